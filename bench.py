@@ -1,0 +1,351 @@
+#!/usr/bin/env python
+"""Benchmark of one MLA decode step on B200 through libmla's C ABI.
+
+A step is the whole hot path over one batch: append the new tokens' latent
+rows (mla_append_latent), absorb the query (mla_absorb_q), split-KV
+attention over the latent cache (mla_decode_attention) and the combine +
+W_UV up-projection (mla_decode_combine).  The default workload is the
+V3-shaped batch-64 x 4096 decode (128 heads, d_c 512, d_R 64, paged cache of
+64-token blocks with a permuted block table).
+
+Prints one JSON line on rank 0.  Under torchrun each rank runs the same
+workload on its own GPU (independent batches, no data-path collective);
+timings are the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mla|reference] [--config NAME]
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MLA decode TFLOP/s & latent-KV GB/s vs B200 roofline (bf16, V3 shapes)"
+UNIT = "TFLOP/s"
+
+
+def _args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="mla", choices=["mla", "reference"])
+    p.add_argument("--config", default="v3_bf16")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        j = json.load(open(path))
+        return dict(hbm_gbs=j["hbm_gbs"], bf16_tflops=j["bf16_tflops"],
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def _config_json(case, n_gpus):
+    d = case.dims
+    sl = case.seqlens
+    return {"workload": f"{case.name}: MLA decode step (append + absorb + split-KV attention + combine/W_UV)",
+            "batch_per_gpu": case.batch, "global_batch": case.batch * n_gpus, "n_q": case.n_q,
+            "seqlens": list(sl), "heads": d.n_heads, "d_c": d.d_c, "d_rope": d.d_rope, "d_nope": d.d_nope,
+            "d_v": d.d_v, "d_model": d.d_model, "block_size": case.block_size,
+            "block_table": "seeded random permutation" if case.paged else "contiguous",
+            "parallelism": f"replicas x{n_gpus} (independent batches per GPU)",
+            "l2": "inputs larger than L2: the latent cache streamed each step exceeds the 126 MB L2"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def __enter__(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.p:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        try:
+            for line in open(self.f.name):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _traffic_for(kernel_file):
+    """dram bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    j = json.load(open(path))
+    ent = j.get(os.path.basename(kernel_file))
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "mla_latent_kv_40_b200", "csrc", os.path.basename(kernel_file))
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    if h != ent.get("source_sha256_16"):
+        return None
+    return ent.get("dram_bytes_per_full_launch")
+
+
+def cpu_baseline(case, target_s=12.0, inp=None):
+    """The fp64 oracle, as it stands, on a bounded sample of the same workload."""
+    import oracle
+    from workloads import make_decode_inputs
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([t.get("num_threads", 1) for t in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    if inp is None:
+        inp = make_decode_inputs(case)
+    d = case.dims
+    H = d.n_heads
+    S0 = int(inp["seqlens"][0])
+    heads, t0, done = [], time.time(), 0
+    flops = 0
+    while time.time() - t0 < target_s and done < H:
+        picks = [(0, j, done) for j in range(case.n_q)]
+        oracle.decode(d, inp["q_nope"], inp["q_pe"], inp["pool"], inp["block_table"], inp["block_size"],
+                      inp["seqlens"], inp["w_uk"], inp["w_uv"], picks=picks)
+        for j in range(case.n_q):
+            vis = S0 - case.n_q + j + 1
+            flops += vis * (2 * (d.d_c + d.d_rope) + 2 * d.d_c) + 2 * d.d_nope * d.d_c + 2 * d.d_c * d.d_v
+        done += 1
+    el = time.time() - t0
+    return {"value": flops / el / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"sequence 0 (S={S0}), {done} of {H} heads, all {case.n_q} query tokens; fp64 unabsorbed "
+                      f"form, FLOPs counted as absorbed-form work; {el:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from workloads import DECODE_CASES, make_decode_inputs
+    case = DECODE_CASES[args.config]
+    inp = make_decode_inputs(case)
+    vals, last = [], None
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(case, target_s=2.0, inp=inp)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            last = r
+    v = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) cache rows and queries)",
+            "config": _config_json(case, 1),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                             "sample": "each step: " + last["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_mla(args):
+    import torch
+    import torch.distributed as dist
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    import mla_latent_kv_40_b200 as mla
+    from workloads import DECODE_CASES, append_flops, decode_flops, latent_bytes, make_decode_step_inputs
+
+    case = DECODE_CASES[args.config]
+    d = case.dims
+    inp = make_decode_step_inputs(case)
+    dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                         rope_base=d.rope_base, rms_eps=d.rms_eps)
+    dev = {k: inp[k].cuda() for k in ("pool", "block_table", "seqlens", "q_nope", "q_pe", "w_uk", "w_uv", "h_new",
+                                      "w_dkv", "w_kr", "gamma", "seq_idx", "pos")}
+    B, n_q, H = case.batch, case.n_q, d.n_heads
+    max_seqlen = int(inp["seqlens"].max())
+    T = B * n_q
+    pool = dev["pool"]
+    c_kv, k_pe = pool, pool[:, d.d_c:]
+    bt = dev["block_table"] if case.paged else None
+    ws = mla.alloc_workspace(mla.mla_decode_workspace_size(dims, B, n_q, max_seqlen))
+    q_abs = torch.empty((B, n_q, H, d.d_c + d.d_rope), dtype=d.torch_dtype, device="cuda")
+    out = torch.empty((B, n_q, H, d.d_v), dtype=d.torch_dtype, device="cuda")
+    lse = torch.empty((B, n_q, H), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def append():
+        mla.mla_append_latent(dims, dev["h_new"], dev["w_dkv"], dev["w_kr"], dev["gamma"], dev["seq_idx"],
+                              dev["pos"], c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status)
+
+    def step(ev=None):
+        append()
+        mla.mla_absorb_q(dims, dev["q_nope"], dev["q_pe"], dev["w_uk"], dev["seqlens"], q_abs)
+        if ev is not None:
+            ev[0].record(stream)
+        mla.mla_decode_attention(dims, q_abs, c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
+                                 dev["seqlens"], max_seqlen, ws, status)
+        if ev is not None:
+            ev[1].record(stream)
+        mla.mla_decode_combine(dims, B, n_q, dev["seqlens"], max_seqlen, dev["w_uv"], out, lse, ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(att_ev[i])
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    att_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in att_ev))
+    clocks = clk.summary()
+
+    # End to end through the public call: pinned host inputs in, result out, copies inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: inp[k].pin_memory() for k in ("h_new", "q_nope", "q_pe", "seqlens", "seq_idx", "pos")}
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+
+        def e2e_step():
+            for k, t in host_in.items():
+                dev[k].copy_(t, non_blocking=True)
+            append()
+            mla.mla_decode(dims, dev["q_nope"], dev["q_pe"], c_kv, k_pe, bt, inp["max_blocks_per_seq"],
+                           inp["num_blocks"], dev["seqlens"], max_seqlen, dev["w_uk"], dev["w_uv"], out, lse, ws,
+                           status)
+            host_out.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps)
+        e2e = {"h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+    fl = decode_flops(d, inp["seqlens"].tolist(), n_q)
+    step_flops = fl["total"] + append_flops(d, T)
+    lat_bytes = latent_bytes(d, inp["seqlens"].tolist())
+    peaks = _peaks()
+    value = step_flops * world / (ms * 1e-3) / 1e12
+    att_gbs = lat_bytes / (att_ms * 1e-3) / 1e9
+    launches_per_step = 1 + mla.mla_decode_launches(dims, n_q)   # append, then absorb + attention + combine
+    t_hbm = lat_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_flop = fl["total"] / (peaks["bf16_tflops"] * 1e12)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if d.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded N(0,1) latent cache rows and queries, N(0,1)/sqrt(fan_in) weights)",
+        "config": _config_json(case, world),
+        "latent_kv_gbs": lat_bytes * world / (ms * 1e-3) / 1e9,
+        "decode_tokens_per_s": T * world / (ms * 1e-3),
+        "step_roofline": {"t_hbm_us": t_hbm * 1e6, "t_tensor_us": t_flop * 1e6,
+                          "frac": max(t_hbm, t_flop) / (ms * 1e-3),
+                          "note": "roofline time = max(latent bytes / HBM, decode FLOPs / bf16 peak) of measured "
+                                  "peaks, over the whole step time"},
+        "roofline": {"kernel": "split-KV attention (mla_decode_attention)", "bound": "hbm",
+                     "achieved": att_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": att_gbs / peaks["hbm_gbs"],
+                     "traffic": _traffic_for("decode_tc.cu" if mla.mla_decode_launches(dims, n_q) != 3 else
+                                             "attn_simt.cu"),
+                     "peak_source": peaks["source"], "kernel_ms": att_ms,
+                     "algorithmic_bytes_per_launch": lat_bytes},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    if e2e:
+        line["e2e"] = {"value": step_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": UNIT,
+                       "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
+                       "ms_per_step": e2e["ms_per_step"]}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(case)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = _args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mla(args)
+
+
+if __name__ == "__main__":
+    main()

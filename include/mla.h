@@ -1,0 +1,227 @@
+/*
+ * mla.h — C ABI of libmla.so: Multi-head Latent Attention (MLA) over a paged
+ * latent KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method (sources by page title and section):
+ *  - "DeepSeek-V3 解读 1: MLA", section "MLA：高层次的思路": each token's hidden
+ *    state h is compressed to a latent c_KV of width d_c; only the latent is
+ *    cached and per-head keys/values are rebuilt from it by W_UK and W_UV.
+ *  - same page, section "为什么需要解耦 RoPE": one extra key k_pe of width d_R,
+ *    shared by every head, carries RoPE; the latent part is never rotated.
+ *  - "Transformer升级之路：21、MLA好在哪里?（下）", section 双重投影: decode may
+ *    fold W_UK into the query (q_lat = q_nope W_UK^T, width d_c) and apply
+ *    W_UV after attention, so every head attends to the same cached rows
+ *    (MQA with K = V = c); prefill uses the decompressed multi-head form.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers, row-major, owned by the caller.
+ *    The library allocates no device memory; scratch space is the caller's
+ *    `workspace`, sized by the matching *_workspace_size call.
+ *  - Float tensors use the element type dims->dtype (MLA_F32: float,
+ *    MLA_BF16: __nv_bfloat16).  lse outputs are always float.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Argument errors are returned before anything is launched.
+ *    Errors found on the device (a block id outside [0, num_blocks), a
+ *    bounded wait that timed out) are written to *dev_status (if non-NULL) with
+ *    an atomic compare-and-swap from 0, so the first error wins; the caller
+ *    zeroes it beforehand and reads it after synchronising.
+ *  - The library keeps no mutable global state; concurrent calls on different
+ *    streams with disjoint outputs and workspaces are safe.
+ *  - There is no CPU fallback: a shape the CUDA kernels do not handle returns
+ *    MLA_ERR_UNSUPPORTED.
+ *
+ * Paged latent cache
+ *  Token i of sequence b lives in pool row r = blk * block_size + i % block_size
+ *  with blk = block_table[b * max_blocks_per_seq + i / block_size]
+ *  (block_table == NULL means the identity table: blk = b * max_blocks_per_seq
+ *  + i / block_size, i.e. each sequence owns a contiguous run of rows).
+ *  c_KV of row r is at c_kv + r * ckv_stride (d_c elements), the rotated RoPE
+ *  key at k_pe + r * kpe_stride (d_R elements).  The fused layout used by the
+ *  fast decode kernel is one pool of rows of d_c + d_R elements with
+ *  k_pe = c_kv + d_c and both strides = d_c + d_R.
+ *
+ * Positions and RoPE
+ *  Positions are 0-based.  Pair (2i, 2i+1) of a RoPE vector at position p is
+ *  rotated by p * theta_i, theta_i = rope_base^(-2i/d_R), with
+ *  [x'; y'] = [[cos, -sin], [sin, cos]] [x; y].  In decode, seqlens[b] counts
+ *  the cached tokens INCLUDING the n_q new ones (already appended), and query
+ *  token j of sequence b sits at position seqlens[b] - n_q + j and attends to
+ *  keys 0 .. seqlens[b] - n_q + j (causal among the new tokens).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MLA_API __attribute__((visibility("default")))
+#else
+#define MLA_API
+#endif
+
+typedef struct CUstream_st *mla_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = -1, /* a NULL required pointer, a non-positive size, inconsistent dims */
+  MLA_ERR_UNSUPPORTED = -2, /* a valid shape the kernels do not implement */
+  MLA_ERR_WORKSPACE = -3,   /* workspace NULL or smaller than *_workspace_size reports */
+  MLA_ERR_CUDA = -4,        /* a CUDA runtime/driver call or a kernel launch failed */
+  MLA_ERR_TIMEOUT = -5,     /* device only: a bounded wait inside a kernel gave up */
+  MLA_ERR_BAD_INDEX = -6    /* device only: a block id outside [0, num_blocks) or a bad position */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+typedef struct {
+  int n_heads;        /* H: query heads */
+  int d_c;            /* latent width (c_KV) */
+  int d_rope;         /* d_R: width of the shared RoPE key and of q_pe; even */
+  int d_nope;         /* per-head query/key width without RoPE */
+  int d_v;            /* per-head value width */
+  int d_model;        /* D: hidden width of h (append only) */
+  int block_size;     /* tokens per cache page, >= 1 */
+  int ckv_stride;     /* elements between consecutive rows of the c_KV pool, >= d_c */
+  int kpe_stride;     /* elements between consecutive rows of the k_pe pool, >= d_rope */
+  float rope_base;    /* RoPE base, e.g. 10000 */
+  float softmax_scale;/* <= 0 selects 1/sqrt(d_nope + d_rope) */
+  float rms_eps;      /* epsilon of the RMSNorm on c_KV, e.g. 1e-6 */
+  int dtype;          /* mla_dtype of every float tensor */
+} mla_dims;
+
+/*
+ * mla_append_latent — write the cache rows of T new tokens.
+ *   "DeepSeek-V3 解读 1: MLA", sections "MLA：高层次的思路" (c_KV = h W_DKV) and
+ *   "为什么需要解耦 RoPE" (k_pe = RoPE(h W_KR), shared by all heads), with an
+ *   RMSNorm over the d_c latent dims: c_KV = gamma * c / sqrt(mean(c^2) + eps).
+ *   h [T, D]; w_dkv [D, d_c]; w_kr [D, d_R]; rms_gamma [d_c] or NULL (= all ones);
+ *   seq_idx [T], pos [T] (int32): sequence and 0-based position of each token.
+ *   Writes c_kv/k_pe rows of (seq_idx[t], pos[t]) through block_table
+ *   ([num_seqs, max_blocks_per_seq] or NULL, see above).  On the device,
+ *   seq_idx outside [0, num_seqs), pos outside [0, max_blocks_per_seq *
+ *   block_size) and block ids outside [0, num_blocks) report
+ *   MLA_ERR_BAD_INDEX and skip that token.
+ *   T == 0 is a no-op.  Rows not named by (seq_idx, pos) are not touched.
+ */
+MLA_API int mla_append_latent(const mla_dims *dims, int T, const void *h, const void *w_dkv,
+                      const void *w_kr, const void *rms_gamma, const int32_t *seq_idx,
+                      const int32_t *pos, void *c_kv, void *k_pe, const int32_t *block_table,
+                      int num_seqs, int max_blocks_per_seq, int num_blocks, int *dev_status,
+                      mla_stream_t stream);
+
+/*
+ * mla_absorb_q — the decode query in latent space.
+ *   "Transformer升级之路：21、MLA好在哪里?（下）", section 双重投影, decoding
+ *   column: q^(s) = x W_q^(s) W_k^(s)T lies in R^{d_c}; here
+ *   q_lat[b,j,s,:] = W_UK[s] q_nope[b,j,s,:] and q_rot = RoPE(q_pe, seqlens[b] - n_q + j).
+ *   q_nope [B, n_q, H, d_nope], q_pe [B, n_q, H, d_R] (not rotated),
+ *   w_uk [H, d_c, d_nope], seqlens [B] (int32, device).
+ *   Writes q_out [B, n_q, H, d_c + d_R] = [q_lat | q_rot] in dims->dtype
+ *   (rounded once, after fp32 accumulation).
+ */
+MLA_API int mla_absorb_q(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                 const void *w_uk, const int32_t *seqlens, void *q_out, mla_stream_t stream);
+
+/*
+ * mla_decode_workspace_size — bytes of scratch mla_decode / mla_decode_latent
+ *   need for B sequences of n_q query tokens whose seqlens are <= max_seqlen.
+ *   Depends on the current device's SM count.
+ */
+MLA_API int mla_decode_workspace_size(const mla_dims *dims, int B, int n_q, int max_seqlen, size_t *bytes);
+
+/*
+ * mla_decode — one batched decode step in matrix-absorbed form.
+ *   Same section 双重投影, decoding column, with the shared RoPE key:
+ *   z_i = scale * (q_lat . c_i + q_rot . kpe_i), softmax over keys
+ *   0 .. seqlens[b] - n_q + j, o_lat = sum_i p_i c_i, out^(s) = o_lat W_UV^(s).
+ *   q_nope [B, n_q, H, d_nope], q_pe [B, n_q, H, d_R] (not rotated);
+ *   cache as described above; seqlens [B] (int32, device, >= n_q, <= max_seqlen);
+ *   w_uk [H, d_c, d_nope]; w_uv [H, d_c, d_v].
+ *   Writes out [B, n_q, H, d_v] and, if non-NULL, lse [B, n_q, H] (float,
+ *   natural log of sum_i exp(z_i)).  workspace: >= mla_decode_workspace_size bytes,
+ *   256-byte aligned.  Errors: INVALID_ARG, UNSUPPORTED (n_q * H > 256),
+ *   WORKSPACE, CUDA; on the device BAD_INDEX, TIMEOUT.
+ */
+MLA_API int mla_decode(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+               const void *c_kv, const void *k_pe, const int32_t *block_table,
+               int max_blocks_per_seq, int num_blocks, const int32_t *seqlens, int max_seqlen,
+               const void *w_uk, const void *w_uv, void *out, float *lse, void *workspace,
+               size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
+ * mla_decode_latent — mla_decode without the W_UV up-projection: writes the
+ *   softmax-weighted latent o_lat [B, n_q, H, d_c] (dims->dtype) and lse.  For
+ *   callers that fold W_UV into their output projection (same page, section
+ *   键值共享: the c -> v map is absorbed on the W_o side).  w_uv is not read.
+ */
+MLA_API int mla_decode_latent(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                      const void *c_kv, const void *k_pe, const int32_t *block_table,
+                      int max_blocks_per_seq, int num_blocks, const int32_t *seqlens,
+                      int max_seqlen, const void *w_uk, void *o_lat, float *lse, void *workspace,
+                      size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
+ * mla_decode_attention / mla_decode_combine — the two halves of mla_decode
+ *   after mla_absorb_q, for callers that schedule the stages themselves.
+ *   mla_decode_attention: q_abs [B, n_q, H, d_c + d_R] is mla_absorb_q's output;
+ *   runs the split-KV attention over the latent cache (scores
+ *   scale * q_abs . [c_i | kpe_i], online softmax, sum_i p_i c_i) and leaves
+ *   per-split partial outputs and log-sum-exps in `workspace` (layout private
+ *   to the library; same size rule as mla_decode).
+ *   mla_decode_combine: merges those partials by their log-sum-exps and, when
+ *   w_uv is non-NULL, applies out^(s) = o_lat W_UV^(s) (out [B, n_q, H, d_v]);
+ *   with w_uv == NULL it writes o_lat [B, n_q, H, d_c].  It must see the same
+ *   dims, B, n_q, seqlens, max_seqlen and workspace as the attention call.
+ */
+MLA_API int mla_decode_attention(const mla_dims *dims, int B, int n_q, const void *q_abs, const void *c_kv,
+                                 const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
+                                 int num_blocks, const int32_t *seqlens, int max_seqlen, void *workspace,
+                                 size_t ws_bytes, int *dev_status, mla_stream_t stream);
+MLA_API int mla_decode_combine(const mla_dims *dims, int B, int n_q, const int32_t *seqlens, int max_seqlen,
+                               const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes,
+                               mla_stream_t stream);
+
+/*
+ * mla_prefill_workspace_size — scratch bytes of mla_prefill for total_tokens
+ *   query tokens in B sequences of at most max_seqlen tokens.
+ */
+MLA_API int mla_prefill_workspace_size(const mla_dims *dims, int B, int total_tokens, int max_seqlen,
+                               size_t *bytes);
+
+/*
+ * mla_prefill — causal prefill in the decompressed multi-head form.
+ *   Same page, section 双重投影, training/prefill column: per head
+ *   k_i = [c_i W_UK^(s) | kpe_i] (width d_nope + d_R), v_i = c_i W_UV^(s) (d_v),
+ *   o_t = softmax_{i<=t}(scale * q_t . k_i) v.
+ *   cu_seqlens [B+1] (int32, device): sequence b owns query rows
+ *   cu_seqlens[b] .. cu_seqlens[b+1]-1, its token t at position t; its cache
+ *   (already appended) holds tokens 0 .. len-1.  q_nope [total, H, d_nope],
+ *   q_pe [total, H, d_R] (not rotated).  Writes out [total, H, d_v] and, if
+ *   non-NULL, lse [total, H].
+ */
+MLA_API int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, int max_seqlen,
+                int total_tokens, const void *q_nope, const void *q_pe, const void *c_kv,
+                const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
+                int num_blocks, const void *w_uk, const void *w_uv, void *out, float *lse,
+                void *workspace, size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
+ * mla_decode_launches — how many kernels one mla_decode call launches for this
+ *   shape (query absorption, attention, combine); for launch accounting in
+ *   profilers and benchmarks.  Writes *count; no device work.
+ */
+MLA_API int mla_decode_launches(const mla_dims *dims, int n_q, int *count);
+
+/* Human-readable text of an mla_status value (static storage). */
+MLA_API const char *mla_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

@@ -1,0 +1,241 @@
+"""Python binding of libmla.so (the MLA latent-KV C ABI declared in include/mla.h).
+
+Argument marshalling only: every function takes torch tensors that already
+live on the GPU, checks their dtype/shape/contiguity, and passes raw device
+pointers plus the current CUDA stream to the C entry point of the same name.
+All compute runs in the library's CUDA kernels.  Importing this module fails
+loudly if the library has not been built; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python mla_latent_kv_40_b200/build.py`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+MLA_F32, MLA_BF16 = 0, 1
+STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_WORKSPACE",
+          -4: "MLA_ERR_CUDA", -5: "MLA_ERR_TIMEOUT", -6: "MLA_ERR_BAD_INDEX"}
+
+
+class MlaError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {code} ({STATUS.get(code, '?')}: {mla_status_string(code)})")
+        self.code = code
+
+
+class mla_dims(ctypes.Structure):
+    _fields_ = [("n_heads", ctypes.c_int), ("d_c", ctypes.c_int), ("d_rope", ctypes.c_int),
+                ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int), ("d_model", ctypes.c_int),
+                ("block_size", ctypes.c_int), ("ckv_stride", ctypes.c_int), ("kpe_stride", ctypes.c_int),
+                ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
+                ("dtype", ctypes.c_int)]
+
+
+def make_dims(n_heads, d_c, d_rope, d_nope, d_v, d_model, block_size, dtype, ckv_stride=None,
+              kpe_stride=None, rope_base=10000.0, softmax_scale=0.0, rms_eps=1e-6) -> mla_dims:
+    """Dims of a fused cache pool by default: rows of d_c + d_rope elements."""
+    w = d_c + d_rope
+    dt = MLA_BF16 if dtype in ("bf16", torch.bfloat16, MLA_BF16) else MLA_F32
+    return mla_dims(n_heads, d_c, d_rope, d_nope, d_v, d_model, block_size,
+                    w if ckv_stride is None else ckv_stride, w if kpe_stride is None else kpe_stride,
+                    rope_base, softmax_scale, rms_eps, dt)
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_D = ctypes.POINTER(mla_dims)
+_SZ = ctypes.POINTER(ctypes.c_size_t)
+_sigs = {
+    "mla_append_latent": [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P],
+    "mla_absorb_q": [_D, _I, _I, _P, _P, _P, _P, _P, _P],
+    "mla_decode_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
+    "mla_decode_latent": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
+    "mla_decode_attention": [_D, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _P, ctypes.c_size_t, _P, _P],
+    "mla_decode_combine": [_D, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P],
+    "mla_prefill_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode_launches": [_D, _I, ctypes.POINTER(ctypes.c_int)],
+    "mla_prefill": [_D, _I, _P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
+}
+for _n, _a in _sigs.items():
+    getattr(_lib, _n).argtypes = _a
+    getattr(_lib, _n).restype = ctypes.c_int
+_lib.mla_status_string.argtypes = [_I]
+_lib.mla_status_string.restype = ctypes.c_char_p
+
+
+def mla_status_string(code: int) -> str:
+    return _lib.mla_status_string(int(code)).decode()
+
+
+def _elem_dtype(dims: mla_dims):
+    return torch.bfloat16 if dims.dtype == MLA_BF16 else torch.float32
+
+
+def _ptr(t, dtype=None, name="", optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dense(t, name):
+    if t is not None and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MlaError(fn, rc)
+
+
+def mla_append_latent(dims, h, w_dkv, w_kr, rms_gamma, seq_idx, pos, c_kv, k_pe, block_table, num_seqs,
+                      max_blocks_per_seq, num_blocks, dev_status=None, stream=None):
+    et = _elem_dtype(dims)
+    T = 0 if h is None else h.shape[0]
+    for n, t in (("h", h), ("w_dkv", w_dkv), ("w_kr", w_kr), ("rms_gamma", rms_gamma), ("seq_idx", seq_idx),
+                 ("pos", pos), ("block_table", block_table)):
+        _dense(t, n)
+    rc = _lib.mla_append_latent(ctypes.byref(dims), T, _ptr(h, et, "h"), _ptr(w_dkv, et, "w_dkv"),
+                                _ptr(w_kr, et, "w_kr"), _ptr(rms_gamma, et, "rms_gamma", True),
+                                _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(pos, torch.int32, "pos"),
+                                _ptr(c_kv, et, "c_kv"), _ptr(k_pe, et, "k_pe"),
+                                _ptr(block_table, torch.int32, "block_table", True), int(num_seqs),
+                                int(max_blocks_per_seq), int(num_blocks),
+                                _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_append_latent", rc)
+
+
+def mla_absorb_q(dims, q_nope, q_pe, w_uk, seqlens, q_out, stream=None):
+    et = _elem_dtype(dims)
+    B, n_q = q_nope.shape[0], q_nope.shape[1]
+    for n, t in (("q_nope", q_nope), ("q_pe", q_pe), ("w_uk", w_uk), ("seqlens", seqlens), ("q_out", q_out)):
+        _dense(t, n)
+    rc = _lib.mla_absorb_q(ctypes.byref(dims), B, n_q, _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"),
+                           _ptr(w_uk, et, "w_uk"), _ptr(seqlens, torch.int32, "seqlens"),
+                           _ptr(q_out, et, "q_out"), _stream(stream))
+    _check("mla_absorb_q", rc)
+
+
+def mla_decode_workspace_size(dims, B, n_q, max_seqlen) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_decode_workspace_size",
+           _lib.mla_decode_workspace_size(ctypes.byref(dims), int(B), int(n_q), int(max_seqlen), ctypes.byref(n)))
+    return int(n.value)
+
+
+def _decode_common(fn, dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                   max_seqlen, w_uk, w_uv, out, lse, workspace, dev_status, stream):
+    et = _elem_dtype(dims)
+    B, n_q = q_nope.shape[0], q_nope.shape[1]
+    for n, t in (("q_nope", q_nope), ("q_pe", q_pe), ("block_table", block_table), ("seqlens", seqlens),
+                 ("w_uk", w_uk), ("w_uv", w_uv), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    args = [ctypes.byref(dims), B, n_q, _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"),
+            _ptr(c_kv, et, "c_kv"), _ptr(k_pe, et, "k_pe"), _ptr(block_table, torch.int32, "block_table", True),
+            int(max_blocks_per_seq), int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"), int(max_seqlen),
+            _ptr(w_uk, et, "w_uk")]
+    if fn == "mla_decode":
+        args.append(_ptr(w_uv, et, "w_uv"))
+    args += [_ptr(out, et, "out"), _ptr(lse, torch.float32, "lse", True), _ptr(workspace, None, "workspace"),
+             ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+             _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream)]
+    _check(fn, getattr(_lib, fn)(*args))
+
+
+def mla_decode(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens, max_seqlen,
+               w_uk, w_uv, out, lse, workspace, dev_status=None, stream=None):
+    _decode_common("mla_decode", dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks,
+                   seqlens, max_seqlen, w_uk, w_uv, out, lse, workspace, dev_status, stream)
+
+
+def mla_decode_latent(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                      max_seqlen, w_uk, o_lat, lse, workspace, dev_status=None, stream=None):
+    _decode_common("mla_decode_latent", dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq,
+                   num_blocks, seqlens, max_seqlen, w_uk, None, o_lat, lse, workspace, dev_status, stream)
+
+
+def mla_decode_attention(dims, q_abs, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens, max_seqlen,
+                         workspace, dev_status=None, stream=None):
+    et = _elem_dtype(dims)
+    B, n_q = q_abs.shape[0], q_abs.shape[1]
+    for n, t in (("q_abs", q_abs), ("block_table", block_table), ("seqlens", seqlens)):
+        _dense(t, n)
+    rc = _lib.mla_decode_attention(ctypes.byref(dims), B, n_q, _ptr(q_abs, et, "q_abs"), _ptr(c_kv, et, "c_kv"),
+                                   _ptr(k_pe, et, "k_pe"), _ptr(block_table, torch.int32, "block_table", True),
+                                   int(max_blocks_per_seq), int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"),
+                                   int(max_seqlen), _ptr(workspace, None, "workspace"),
+                                   ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                   _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_decode_attention", rc)
+
+
+def mla_decode_combine(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, workspace, stream=None):
+    et = _elem_dtype(dims)
+    for n, t in (("seqlens", seqlens), ("w_uv", w_uv), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_decode_combine(ctypes.byref(dims), int(B), int(n_q), _ptr(seqlens, torch.int32, "seqlens"),
+                                 int(max_seqlen), _ptr(w_uv, et, "w_uv", True), _ptr(out, et, "out"),
+                                 _ptr(lse, torch.float32, "lse", True), _ptr(workspace, None, "workspace"),
+                                 ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check("mla_decode_combine", rc)
+
+
+def mla_decode_launches(dims, n_q) -> int:
+    n = ctypes.c_int(0)
+    _check("mla_decode_launches", _lib.mla_decode_launches(ctypes.byref(dims), int(n_q), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_prefill_workspace_size(dims, B, total_tokens, max_seqlen) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_prefill_workspace_size",
+           _lib.mla_prefill_workspace_size(ctypes.byref(dims), int(B), int(total_tokens), int(max_seqlen),
+                                           ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_prefill(dims, cu_seqlens, max_seqlen, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks,
+                w_uk, w_uv, out, lse, workspace, dev_status=None, stream=None):
+    et = _elem_dtype(dims)
+    B = cu_seqlens.shape[0] - 1
+    total = q_nope.shape[0]
+    for n, t in (("cu_seqlens", cu_seqlens), ("q_nope", q_nope), ("q_pe", q_pe), ("block_table", block_table),
+                 ("w_uk", w_uk), ("w_uv", w_uv), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_prefill(ctypes.byref(dims), B, _ptr(cu_seqlens, torch.int32, "cu_seqlens"), int(max_seqlen), total,
+                          _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"), _ptr(c_kv, et, "c_kv"),
+                          _ptr(k_pe, et, "k_pe"), _ptr(block_table, torch.int32, "block_table", True),
+                          int(max_blocks_per_seq), int(num_blocks), _ptr(w_uk, et, "w_uk"), _ptr(w_uv, et, "w_uv"),
+                          _ptr(out, et, "out"), _ptr(lse, torch.float32, "lse", True),
+                          _ptr(workspace, None, "workspace"),
+                          ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                          _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_prefill", rc)
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte aligned uint8 device buffer (torch's caching allocator aligns to 512 B)."""
+    t = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    assert t.data_ptr() % 256 == 0
+    return t

@@ -1,0 +1,261 @@
+// C-ABI entry points of libmla: argument validation, workspace carving and
+// kernel dispatch.  Every step of every call runs in this library's kernels;
+// there is no host-side compute and no CPU fallback.
+#include <cuda_runtime.h>
+
+#include "decode_tc.cuh"
+#include "kernels.cuh"
+
+using namespace mla;
+
+namespace {
+
+constexpr int kSimtChunk = 1024;   // keys per split in the CUDA-core decode path
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool dims_ok(const mla_dims *d) {
+  if (!d) return false;
+  if (d->n_heads <= 0 || d->d_c <= 0 || d->d_rope < 0 || (d->d_rope & 1) || d->d_nope <= 0 ||
+      d->d_v <= 0 || d->block_size <= 0)
+    return false;
+  if (d->ckv_stride < d->d_c || d->kpe_stride < d->d_rope) return false;
+  if (d->dtype != MLA_F32 && d->dtype != MLA_BF16) return false;
+  if (!(d->rope_base > 0.f)) return false;
+  return true;
+}
+
+size_t elem(const mla_dims *d) { return d->dtype == MLA_BF16 ? 2 : 4; }
+
+struct DecodeLayout {
+  size_t q_off, o_off, lse_off, tc_off, total;
+  int max_chunks;
+  bool use_tc;
+};
+
+DecodeLayout decode_layout(const mla_dims *d, int B, int n_q, int max_seqlen) {
+  DecodeLayout L{};
+  const size_t W = (size_t)d->d_c + d->d_rope;
+  const size_t R = (size_t)n_q * d->n_heads;
+  L.use_tc = tc_decode_supported(*d, n_q);
+  L.q_off = 0;
+  size_t off = align256((size_t)B * R * W * elem(d));
+  if (L.use_tc) {
+    L.max_chunks = 0;
+    L.o_off = L.lse_off = off;
+    L.tc_off = off;
+    off += align256(tc_decode_workspace_bytes(*d, B, n_q));
+  } else {
+    L.max_chunks = (max_seqlen + kSimtChunk - 1) / kSimtChunk;
+    L.o_off = off;
+    off += align256((size_t)B * L.max_chunks * R * d->d_c * sizeof(float));
+    L.lse_off = off;
+    off += align256((size_t)B * L.max_chunks * R * sizeof(float));
+    L.tc_off = off;
+  }
+  L.total = off;
+  return L;
+}
+
+int check_decode_args(const mla_dims *dims, int B, int n_q, const void *c_kv, const void *k_pe,
+                      int max_blocks_per_seq, int num_blocks, const int32_t *seqlens, int max_seqlen) {
+  if (!dims_ok(dims)) return MLA_ERR_INVALID_ARG;
+  if (B <= 0 || n_q <= 0 || max_seqlen < n_q || max_blocks_per_seq <= 0 || num_blocks <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!c_kv || (!k_pe && dims->d_rope) || !seqlens) return MLA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * dims->block_size < max_seqlen) return MLA_ERR_INVALID_ARG;
+  if (n_q * dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+int check_ws(const DecodeLayout &L, const void *workspace, size_t ws_bytes) {
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
+  return MLA_OK;
+}
+
+int attention_impl(const mla_dims *dims, int B, int n_q, const void *q_abs, const void *c_kv, const void *k_pe,
+                   const int32_t *block_table, int max_blocks_per_seq, int num_blocks, const int32_t *seqlens,
+                   int max_seqlen, const DecodeLayout &L, char *ws, int *dev_status, cudaStream_t st) {
+  const bool bf16 = dims->dtype == MLA_BF16;
+  CacheView cv{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq,
+               num_blocks, dims->block_size};
+  if (L.use_tc)
+    return launch_tc_attention(*dims, B, n_q, q_abs, cv, seqlens, max_seqlen, ws + L.tc_off, dev_status, st);
+  AttnArgs at{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, q_abs, cv, seqlens, default_scale(*dims),
+              kSimtChunk, L.max_chunks, reinterpret_cast<float *>(ws + L.o_off),
+              reinterpret_cast<float *>(ws + L.lse_off), dev_status};
+  return launch_attn_simt(at, bf16, st);
+}
+
+int combine_impl(const mla_dims *dims, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
+                 void *out, float *lse, const DecodeLayout &L, char *ws, cudaStream_t st) {
+  const bool bf16 = dims->dtype == MLA_BF16;
+  if (L.use_tc) return launch_tc_combine(*dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, ws + L.tc_off, st);
+  CombineArgs cb{B, n_q, dims->n_heads, dims->d_c, dims->d_v, seqlens, kSimtChunk, L.max_chunks,
+                 reinterpret_cast<const float *>(ws + L.o_off), reinterpret_cast<const float *>(ws + L.lse_off),
+                 w_uv, out, lse};
+  return launch_combine(cb, bf16, st);
+}
+
+int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                const void *c_kv, const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
+                int num_blocks, const int32_t *seqlens, int max_seqlen, const void *w_uk,
+                const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes,
+                int *dev_status, cudaStream_t st) {
+  int rc = check_decode_args(dims, B, n_q, c_kv, k_pe, max_blocks_per_seq, num_blocks, seqlens, max_seqlen);
+  if (rc) return rc;
+  if (!q_nope || (!q_pe && dims->d_rope) || !w_uk || !out) return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(dims, B, n_q, max_seqlen);
+  if ((rc = check_ws(L, workspace, ws_bytes))) return rc;
+  char *ws = static_cast<char *>(workspace);
+  void *qbuf = ws + L.q_off;
+  AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
+                q_nope, q_pe, w_uk, seqlens, qbuf, dims->rope_base};
+  if ((rc = launch_absorb(ab, dims->dtype == MLA_BF16, st))) return rc;
+  if ((rc = attention_impl(dims, B, n_q, qbuf, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                           max_seqlen, L, ws, dev_status, st)))
+    return rc;
+  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, ws, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mla_status_string(int s) {
+  switch (s) {
+    case MLA_OK: return "ok";
+    case MLA_ERR_INVALID_ARG: return "invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "unsupported shape";
+    case MLA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case MLA_ERR_CUDA: return "CUDA error";
+    case MLA_ERR_TIMEOUT: return "device wait timed out";
+    case MLA_ERR_BAD_INDEX: return "block id, sequence index or position out of range";
+    default: return "unknown status";
+  }
+}
+
+int mla_append_latent(const mla_dims *dims, int T, const void *h, const void *w_dkv, const void *w_kr,
+                      const void *rms_gamma, const int32_t *seq_idx, const int32_t *pos, void *c_kv,
+                      void *k_pe, const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
+                      int num_blocks, int *dev_status, mla_stream_t stream) {
+  if (!dims_ok(dims) || dims->d_model <= 0 || T < 0) return MLA_ERR_INVALID_ARG;
+  if (T == 0) return MLA_OK;
+  if (!h || !w_dkv || (!w_kr && dims->d_rope) || !seq_idx || !pos || !c_kv || (!k_pe && dims->d_rope))
+    return MLA_ERR_INVALID_ARG;
+  if (num_seqs <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return MLA_ERR_INVALID_ARG;
+  AppendArgs a{T, dims->d_model, dims->d_c, dims->d_rope, h, w_dkv, w_kr, rms_gamma, seq_idx, pos,
+               c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, num_seqs,
+               max_blocks_per_seq, num_blocks, dims->block_size, dims->rms_eps, dims->rope_base,
+               dev_status};
+  return launch_append(a, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_absorb_q(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                 const void *w_uk, const int32_t *seqlens, void *q_out, mla_stream_t stream) {
+  if (!dims_ok(dims) || B <= 0 || n_q <= 0) return MLA_ERR_INVALID_ARG;
+  if (!q_nope || (!q_pe && dims->d_rope) || !w_uk || !seqlens || !q_out) return MLA_ERR_INVALID_ARG;
+  AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
+                q_nope, q_pe, w_uk, seqlens, q_out, dims->rope_base};
+  return launch_absorb(ab, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_workspace_size(const mla_dims *dims, int B, int n_q, int max_seqlen, size_t *bytes) {
+  if (!dims_ok(dims) || B <= 0 || n_q <= 0 || max_seqlen < n_q || !bytes) return MLA_ERR_INVALID_ARG;
+  if (n_q * dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  *bytes = decode_layout(dims, B, n_q, max_seqlen).total;
+  return MLA_OK;
+}
+
+int mla_decode(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+               const void *c_kv, const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
+               int num_blocks, const int32_t *seqlens, int max_seqlen, const void *w_uk,
+               const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes,
+               int *dev_status, mla_stream_t stream) {
+  if (!w_uv) return MLA_ERR_INVALID_ARG;
+  return decode_impl(dims, B, n_q, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq,
+                     num_blocks, seqlens, max_seqlen, w_uk, w_uv, out, lse, workspace, ws_bytes,
+                     dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_latent(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                      const void *c_kv, const void *k_pe, const int32_t *block_table,
+                      int max_blocks_per_seq, int num_blocks, const int32_t *seqlens, int max_seqlen,
+                      const void *w_uk, void *o_lat, float *lse, void *workspace, size_t ws_bytes,
+                      int *dev_status, mla_stream_t stream) {
+  return decode_impl(dims, B, n_q, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq,
+                     num_blocks, seqlens, max_seqlen, w_uk, nullptr, o_lat, lse, workspace, ws_bytes,
+                     dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_attention(const mla_dims *dims, int B, int n_q, const void *q_abs, const void *c_kv,
+                         const void *k_pe, const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                         const int32_t *seqlens, int max_seqlen, void *workspace, size_t ws_bytes,
+                         int *dev_status, mla_stream_t stream) {
+  int rc = check_decode_args(dims, B, n_q, c_kv, k_pe, max_blocks_per_seq, num_blocks, seqlens, max_seqlen);
+  if (rc) return rc;
+  if (!q_abs) return MLA_ERR_INVALID_ARG;
+  const DecodeLayout L = decode_layout(dims, B, n_q, max_seqlen);
+  if ((rc = check_ws(L, workspace, ws_bytes))) return rc;
+  return attention_impl(dims, B, n_q, q_abs, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                        max_seqlen, L, static_cast<char *>(workspace), dev_status,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_combine(const mla_dims *dims, int B, int n_q, const int32_t *seqlens, int max_seqlen,
+                       const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes,
+                       mla_stream_t stream) {
+  if (!dims_ok(dims) || B <= 0 || n_q <= 0 || max_seqlen < n_q || !seqlens || !out) return MLA_ERR_INVALID_ARG;
+  if (n_q * dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  const DecodeLayout L = decode_layout(dims, B, n_q, max_seqlen);
+  int rc = check_ws(L, workspace, ws_bytes);
+  if (rc) return rc;
+  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, static_cast<char *>(workspace),
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_launches(const mla_dims *dims, int n_q, int *count) {
+  if (!dims_ok(dims) || n_q <= 0 || !count) return MLA_ERR_INVALID_ARG;
+  *count = tc_decode_supported(*dims, n_q) ? 1 + tc_decode_kernel_launches() : 3;
+  return MLA_OK;
+}
+
+int mla_prefill_workspace_size(const mla_dims *dims, int B, int total_tokens, int max_seqlen,
+                               size_t *bytes) {
+  if (!dims_ok(dims) || B <= 0 || total_tokens <= 0 || max_seqlen <= 0 || !bytes)
+    return MLA_ERR_INVALID_ARG;
+  const size_t dqk = (size_t)dims->d_nope + dims->d_rope;
+  const size_t rows = (size_t)total_tokens * dims->n_heads;
+  *bytes = 2 * align256(rows * dqk * elem(dims)) + align256(rows * dims->d_v * elem(dims));
+  return MLA_OK;
+}
+
+int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, int max_seqlen, int total_tokens,
+                const void *q_nope, const void *q_pe, const void *c_kv, const void *k_pe,
+                const int32_t *block_table, int max_blocks_per_seq, int num_blocks, const void *w_uk,
+                const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes, int *dev_status,
+                mla_stream_t stream) {
+  if (!dims_ok(dims) || B <= 0 || total_tokens <= 0 || max_seqlen <= 0 || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!cu_seqlens || !q_nope || (!q_pe && dims->d_rope) || !c_kv || (!k_pe && dims->d_rope) || !w_uk ||
+      !w_uv || !out)
+    return MLA_ERR_INVALID_ARG;
+  size_t need = 0;
+  mla_prefill_workspace_size(dims, B, total_tokens, max_seqlen, &need);
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
+  const size_t dqk = (size_t)dims->d_nope + dims->d_rope;
+  const size_t rows = (size_t)total_tokens * dims->n_heads;
+  char *ws = static_cast<char *>(workspace);
+  void *qbuf = ws;
+  void *kbuf = ws + align256(rows * dqk * elem(dims));
+  void *vbuf = ws + 2 * align256(rows * dqk * elem(dims));
+  PrefillArgs a{B, total_tokens, max_seqlen, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope, dims->d_v,
+                cu_seqlens, q_nope, q_pe, w_uk, w_uv,
+                CacheView{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq,
+                          num_blocks, dims->block_size},
+                qbuf, kbuf, vbuf, out, lse, default_scale(*dims), dims->rope_base, dev_status};
+  return launch_prefill_simt(a, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

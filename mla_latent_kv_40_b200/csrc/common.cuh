@@ -1,0 +1,60 @@
+// Shared device helpers of libmla: element conversion, status reporting,
+// paged-row addressing and the RoPE angle.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/mla.h"
+
+namespace mla {
+
+// ---- element types ---------------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// ---- device-side error reporting -------------------------------------------
+// First error wins: the word moves from 0 to the code once.
+__device__ __forceinline__ void report(int *dev_status, int code) {
+  if (dev_status) atomicCAS(dev_status, 0, code);
+}
+
+// ---- paged latent cache ----------------------------------------------------
+// Row of token i of sequence b, or -1 if the block id is out of range.
+__device__ __forceinline__ int64_t cache_row(const int32_t *block_table, int max_blocks_per_seq,
+                                             int num_blocks, int block_size, int b, int i) {
+  if (i < 0) return -1;
+  const int lb = i / block_size;
+  if (lb >= max_blocks_per_seq) return -1;
+  const int blk = block_table ? block_table[(int64_t)b * max_blocks_per_seq + lb]
+                              : b * max_blocks_per_seq + lb;
+  if (blk < 0 || blk >= num_blocks) return -1;
+  return (int64_t)blk * block_size + (i % block_size);
+}
+
+// ---- RoPE ------------------------------------------------------------------
+// cos/sin of p * base^(-2i/d).  The angle is formed and reduced modulo 2*pi in
+// double so that positions up to 2^31 keep full fp32 accuracy in the result.
+__device__ __forceinline__ void rope_cos_sin(int pos, int pair, int d_rope, float base, float *c,
+                                             float *s) {
+  const double theta = pow((double)base, -2.0 * (double)pair / (double)d_rope);
+  double a = (double)pos * theta;
+  const double two_pi = 6.283185307179586476925286766559;
+  a = a - two_pi * floor(a / two_pi);
+  float sf, cf;
+  sincosf((float)a, &sf, &cf);
+  *c = cf;
+  *s = sf;
+}
+
+__host__ __device__ inline float default_scale(const mla_dims &d) {
+  return d.softmax_scale > 0.f ? d.softmax_scale : 1.0f / sqrtf((float)(d.d_nope + d.d_rope));
+}
+
+}  // namespace mla

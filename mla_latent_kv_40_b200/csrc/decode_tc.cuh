@@ -1,0 +1,21 @@
+// Tensor-core (tcgen05) split-KV decode over the latent cache: host interface.
+#pragma once
+
+#include "kernels.cuh"
+
+namespace mla {
+
+// True when the shape runs on the tcgen05 path (bf16, fused 576-wide rows, ...).
+bool tc_decode_supported(const mla_dims &d, int n_q);
+// Kernels the tcgen05 attention + combine launch per call.
+int tc_decode_kernel_launches();
+// Scratch bytes the tcgen05 path needs beyond the absorbed query buffer.
+size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q);
+// Split-KV attention from an absorbed query buffer; partials stay in ws.
+int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, const CacheView &cache,
+                        const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st);
+// Merge of the partials (+ W_UV when w_uv != NULL).
+int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
+                      void *out, float *lse, void *ws, cudaStream_t st);
+
+}  // namespace mla

@@ -1,0 +1,79 @@
+// Argument bundles and launchers of every libmla kernel (host side).
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+struct AppendArgs {
+  int T, d_model, d_c, d_rope;
+  const void *h, *w_dkv, *w_kr, *gamma;
+  const int32_t *seq_idx, *pos;
+  void *c_kv, *k_pe;
+  int64_t ckv_stride, kpe_stride;
+  const int32_t *block_table;
+  int num_seqs, max_blocks_per_seq, num_blocks, block_size;
+  float rms_eps, rope_base;
+  int *dev_status;
+};
+
+struct AbsorbArgs {
+  int B, n_q, H, d_c, d_rope, d_nope;
+  const void *q_nope, *q_pe, *w_uk;
+  const int32_t *seqlens;
+  void *q_out;  // [B, n_q, H, d_c + d_rope]
+  float rope_base;
+};
+
+// Paged-cache view shared by the decode kernels.
+struct CacheView {
+  const void *c_kv, *k_pe;
+  int64_t ckv_stride, kpe_stride;
+  const int32_t *block_table;
+  int max_blocks_per_seq, num_blocks, block_size;
+};
+
+// Split-KV attention over the latent cache (the absorbed decode core).
+struct AttnArgs {
+  int B, n_q, H, d_c, d_rope;
+  const void *q;            // [B, n_q, H, d_c + d_rope]: [q_lat | rotated q_pe]
+  CacheView cache;
+  const int32_t *seqlens;
+  float scale;
+  int chunk;                // keys per split
+  int max_chunks;           // splits allocated per sequence
+  float *o_part;            // [B, max_chunks, n_q*H, d_c], normalised by the split's own sum
+  float *lse_part;          // [B, max_chunks, n_q*H]
+  int *dev_status;
+};
+
+// Merge of the split partials and the per-head up-projection.
+struct CombineArgs {
+  int B, n_q, H, d_c, d_v;
+  const int32_t *seqlens;
+  int chunk, max_chunks;
+  const float *o_part, *lse_part;
+  const void *w_uv;         // [H, d_c, d_v], NULL: write o_lat instead
+  void *out;                // [B, n_q, H, d_v] or o_lat [B, n_q, H, d_c]
+  float *lse;               // [B, n_q, H] or NULL
+};
+
+struct PrefillArgs {
+  int B, total, max_seqlen, H, d_c, d_rope, d_nope, d_v;
+  const int32_t *cu_seqlens;
+  const void *q_nope, *q_pe, *w_uk, *w_uv;
+  CacheView cache;
+  void *qbuf, *kbuf, *vbuf;   // workspace: [total, H, d_nope+d_rope] x2, [total, H, d_v]
+  void *out;
+  float *lse;
+  float scale, rope_base;
+  int *dev_status;
+};
+
+int launch_append(const AppendArgs &a, bool bf16, cudaStream_t st);
+int launch_absorb(const AbsorbArgs &a, bool bf16, cudaStream_t st);
+int launch_attn_simt(const AttnArgs &a, bool bf16, cudaStream_t st);
+int launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st);
+int launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st);
+
+}  // namespace mla

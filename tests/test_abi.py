@@ -1,0 +1,98 @@
+"""CPU checks of the C ABI boundary: the library loads without a GPU, exports
+every symbol include/mla.h declares, and rejects bad arguments on the host
+before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    return sorted(set(re.findall(r"MLA_API\s+(?:const\s+char\s*\*|int)\s*(mla_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ("mla_append_latent", "mla_decode_workspace_size", "mla_decode", "mla_prefill",
+                 "mla_prefill_workspace_size", "mla_status_string", "mla_absorb_q", "mla_decode_latent"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol():
+    import mla_latent_kv_40_b200 as mla
+    lib = ctypes.CDLL(mla.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    import mla_latent_kv_40_b200 as mla
+    for code in range(-6, 1):
+        assert mla.mla_status_string(code) and "unknown" not in mla.mla_status_string(code)
+    assert "unknown" in mla.mla_status_string(-99)
+
+
+def test_dims_struct_matches_header_layout():
+    import mla_latent_kv_40_b200 as mla
+    assert ctypes.sizeof(mla.mla_dims) == 13 * 4
+
+
+def _lib():
+    import mla_latent_kv_40_b200 as mla
+    return mla, mla._lib
+
+
+def test_host_validation_rejects_bad_arguments():
+    mla, lib = _lib()
+    d = mla.make_dims(8, 64, 16, 32, 32, 256, 64, "f32")
+    n = ctypes.c_size_t(0)
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 0, 1, 10, ctypes.byref(n)) == -1
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 1, 2, 1, ctypes.byref(n)) == -1   # max_seqlen < n_q
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 1, 1, 10, None) == -1
+    big = mla.make_dims(200, 64, 16, 32, 32, 256, 64, "f32")
+    assert lib.mla_decode_workspace_size(ctypes.byref(big), 1, 2, 10, ctypes.byref(n)) == -2  # n_q*H > 256
+    odd = mla.make_dims(8, 64, 15, 32, 32, 256, 64, "f32")
+    assert lib.mla_decode_workspace_size(ctypes.byref(odd), 1, 1, 10, ctypes.byref(n)) == -1  # odd d_rope
+    bad = mla.make_dims(8, 64, 16, 32, 32, 256, 64, "f32", ckv_stride=10)
+    assert lib.mla_decode_workspace_size(ctypes.byref(bad), 1, 1, 10, ctypes.byref(n)) == -1  # stride < d_c
+    assert lib.mla_decode_workspace_size(ctypes.byref(d), 1, 1, 10, ctypes.byref(n)) == 0 and n.value > 0
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    # Missing pointers are caught before any launch.
+    rc = lib.mla_decode(ctypes.byref(d), 1, 1, None, fake, fake, fake, None, 4, 4, fake, 10, fake, fake, fake,
+                        None, fake, ctypes.c_size_t(1 << 20), None, None)
+    assert rc == -1
+    # Workspace too small / misaligned.
+    rc = lib.mla_decode(ctypes.byref(d), 1, 1, fake, fake, fake, fake, None, 4, 4, fake, 10, fake, fake, fake,
+                        None, fake, ctypes.c_size_t(16), None, None)
+    assert rc == -3
+    rc = lib.mla_decode(ctypes.byref(d), 1, 1, fake, fake, fake, fake, None, 4, 4, fake, 10, fake, fake, fake,
+                        None, P(0x1001), ctypes.c_size_t(1 << 30), None, None)
+    assert rc == -3
+    # Table too short for max_seqlen.
+    rc = lib.mla_decode(ctypes.byref(d), 1, 1, fake, fake, fake, fake, None, 1, 4, fake, 100, fake, fake, fake,
+                        None, fake, ctypes.c_size_t(1 << 30), None, None)
+    assert rc == -1
+    # Append of zero tokens is a no-op that launches nothing.
+    assert lib.mla_append_latent(ctypes.byref(d), 0, None, None, None, None, None, None, None, None, None,
+                                 1, 1, 1, None, None) == 0
+    assert lib.mla_append_latent(ctypes.byref(d), 3, None, fake, fake, None, fake, fake, fake, fake, None,
+                                 1, 1, 1, None, None) == -1
+    assert lib.mla_prefill_workspace_size(ctypes.byref(d), 1, 0, 10, ctypes.byref(n)) == -1
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    """The product path has no fallback: a missing libmla.so is an ImportError."""
+    import importlib.util
+    import shutil
+    pkg = tmp_path / "mla_latent_kv_40_b200"
+    pkg.mkdir()
+    shutil.copy(os.path.join(ROOT, "mla_latent_kv_40_b200", "__init__.py"), pkg / "__init__.py")
+    spec = importlib.util.spec_from_file_location("mla_copy", pkg / "__init__.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "Dims", "DecodeCase", "PrefillCase", "DECODE_CASES", "PREFILL_CASES",
     "make_decode_inputs", "make_prefill_inputs", "make_append_inputs",
-    "cache_row_of", "latent_bytes", "decode_flops", "prefill_flops",
+    "cache_row_of", "latent_bytes", "decode_flops", "prefill_flops", "make_decode_step_inputs", "append_flops",
 ]
 
 
@@ -296,3 +296,31 @@ def prefill_flops(dims: Dims, seqlens) -> dict:
     tok = sum(int(s) for s in seqlens)
     decomp = tok * H * 2 * dims.d_c * (dims.d_nope + dims.d_v)
     return dict(attention=att, decompress=decomp, total=att + decomp)
+
+
+def make_decode_step_inputs(case: DecodeCase, fill: str = "random") -> dict:
+    """Decode inputs plus the append of this step's new tokens.
+
+    The n_q newest tokens of every sequence (positions S_b - n_q .. S_b - 1) get
+    hidden states h [B*n_q, D] and are appended through the same block table
+    before attention; weights W_DKV, W_KR ~ N(0,1)/sqrt(D), gamma = 1.
+    """
+    inp = make_decode_inputs(case, fill=fill)
+    d = case.dims
+    gen = torch.Generator().manual_seed(case.seed + 500)
+    dt = d.torch_dtype
+    T = case.batch * case.n_q
+    inp["h_new"] = _randn(gen, (T, d.d_model)).to(dt)
+    inp["w_dkv"] = _randn(gen, (d.d_model, d.d_c), 1.0 / math.sqrt(d.d_model)).to(dt)
+    inp["w_kr"] = _randn(gen, (d.d_model, d.d_rope), 1.0 / math.sqrt(d.d_model)).to(dt)
+    inp["gamma"] = torch.ones(d.d_c).to(dt)
+    sl = inp["seqlens"].to(torch.int64)
+    inp["seq_idx"] = torch.arange(case.batch, dtype=torch.int32).repeat_interleave(case.n_q)
+    inp["pos"] = (sl.repeat_interleave(case.n_q) - case.n_q
+                  + torch.arange(case.n_q).repeat(case.batch)).to(torch.int32)
+    return inp
+
+
+def append_flops(dims: Dims, T: int) -> int:
+    """FLOPs of appending T tokens: the [T, D] x [D, d_c + d_R] projection."""
+    return 2 * T * dims.d_model * (dims.d_c + dims.d_rope)
