@@ -73,7 +73,8 @@ typedef enum {
   MLA_ERR_WORKSPACE = -3,   /* workspace NULL or smaller than *_workspace_size reports */
   MLA_ERR_CUDA = -4,        /* a CUDA runtime/driver call or a kernel launch failed */
   MLA_ERR_TIMEOUT = -5,     /* device only: a bounded wait inside a kernel gave up */
-  MLA_ERR_BAD_INDEX = -6    /* device only: a block id outside [0, num_blocks) or a bad position */
+  MLA_ERR_BAD_INDEX = -6,   /* device only: a block id outside [0, num_blocks) or a bad position */
+  MLA_ERR_STATIC_WS = -7    /* the shape needs more scratch than mla_decode_noalloc's built-in buffer */
 } mla_status;
 
 typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
@@ -184,6 +185,35 @@ MLA_API int mla_decode_attention(const mla_dims *dims, int B, int n_q, const voi
                                  size_t ws_bytes, int *dev_status, mla_stream_t stream);
 MLA_API int mla_decode_combine(const mla_dims *dims, int B, int n_q, const int32_t *seqlens, int max_seqlen,
                                const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes,
+                               mla_stream_t stream);
+
+/*
+ * mla_decode_noalloc — mla_decode for callers that cannot allocate device
+ *   memory.  The source pages have no counterpart: this is a deployment
+ *   variant, not part of the method.  Some callers cannot call cudaMalloc or
+ *   hold a workspace of their own: code embedded in a host runtime that owns
+ *   every device allocation and forbids side allocations, or plain C callers
+ *   with no allocator at hand.  This entry point takes the same arguments as
+ *   mla_decode minus the workspace, and uses instead one scratch buffer of
+ *   MLA_NOALLOC_SCRATCH_BYTES (16 MiB) that the library reserves statically
+ *   in device memory; every GPU that loads the library holds it until the
+ *   process exits.  It allocates nothing: no cudaMalloc, no cudaFree, no
+ *   allocating library routine.
+ *   - The first call on each device looks up that device's address of the
+ *     buffer (once per device, with that device current); make that first
+ *     call before any stream capture.
+ *   - Every call on a device shares the one buffer, which keeps the last
+ *     call's contents.  Calls whose executions overlap on the GPU (different
+ *     streams, or several host threads) race on it: serialise them.
+ *   - Shapes whose mla_decode_workspace_size exceeds the buffer return
+ *     MLA_ERR_STATIC_WS before anything is launched.
+ *   Output and errors are otherwise those of mla_decode.
+ */
+#define MLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+MLA_API int mla_decode_noalloc(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                               const void *c_kv, const void *k_pe, const int32_t *block_table,
+                               int max_blocks_per_seq, int num_blocks, const int32_t *seqlens, int max_seqlen,
+                               const void *w_uk, const void *w_uv, void *out, float *lse, int *dev_status,
                                mla_stream_t stream);
 
 /*

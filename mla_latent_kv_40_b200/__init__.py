@@ -21,7 +21,8 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 MLA_F32, MLA_BF16 = 0, 1
 STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_WORKSPACE",
-          -4: "MLA_ERR_CUDA", -5: "MLA_ERR_TIMEOUT", -6: "MLA_ERR_BAD_INDEX"}
+          -4: "MLA_ERR_CUDA", -5: "MLA_ERR_TIMEOUT", -6: "MLA_ERR_BAD_INDEX", -7: "MLA_ERR_STATIC_WS"}
+NOALLOC_SCRATCH_BYTES = 16 << 20   # MLA_NOALLOC_SCRATCH_BYTES in include/mla.h
 
 
 class MlaError(RuntimeError):
@@ -62,6 +63,7 @@ _sigs = {
     "mla_decode_combine": [_D, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_prefill_workspace_size": [_D, _I, _I, _I, _SZ],
     "mla_decode_launches": [_D, _I, ctypes.POINTER(ctypes.c_int)],
+    "mla_decode_noalloc": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P],
     "mla_prefill": [_D, _I, _P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
 }
 for _n, _a in _sigs.items():
@@ -167,6 +169,26 @@ def mla_decode(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, 
                w_uk, w_uv, out, lse, workspace, dev_status=None, stream=None):
     _decode_common("mla_decode", dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks,
                    seqlens, max_seqlen, w_uk, w_uv, out, lse, workspace, dev_status, stream)
+
+
+def mla_decode_noalloc(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                       max_seqlen, w_uk, w_uv, out, lse, dev_status=None, stream=None):
+    """mla_decode without a workspace argument: the library's static device
+    scratch (NOALLOC_SCRATCH_BYTES per GPU) stands in for it.  For callers that
+    cannot allocate; calls that overlap on one GPU race on that scratch."""
+    et = _elem_dtype(dims)
+    B, n_q = q_nope.shape[0], q_nope.shape[1]
+    for n, t in (("q_nope", q_nope), ("q_pe", q_pe), ("block_table", block_table), ("seqlens", seqlens),
+                 ("w_uk", w_uk), ("w_uv", w_uv), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_decode_noalloc(ctypes.byref(dims), B, n_q, _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"),
+                                 _ptr(c_kv, et, "c_kv"), _ptr(k_pe, et, "k_pe"),
+                                 _ptr(block_table, torch.int32, "block_table", True), int(max_blocks_per_seq),
+                                 int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"), int(max_seqlen),
+                                 _ptr(w_uk, et, "w_uk"), _ptr(w_uv, et, "w_uv"), _ptr(out, et, "out"),
+                                 _ptr(lse, torch.float32, "lse", True), _ptr(dev_status, torch.int32, "dev_status", True),
+                                 _stream(stream))
+    _check("mla_decode_noalloc", rc)
 
 
 def mla_decode_latent(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,

@@ -131,6 +131,7 @@ const char *mla_status_string(int s) {
     case MLA_ERR_CUDA: return "CUDA error";
     case MLA_ERR_TIMEOUT: return "device wait timed out";
     case MLA_ERR_BAD_INDEX: return "block id, sequence index or position out of range";
+    case MLA_ERR_STATIC_WS: return "shape needs more scratch than the built-in no-allocation buffer";
     default: return "unknown status";
   }
 }
