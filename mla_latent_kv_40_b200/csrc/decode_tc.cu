@@ -1,17 +1,907 @@
+// Split-KV MLA decode on 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// The absorbed decode form of "Transformer升级之路：21、MLA好在哪里?（下）",
+// section 双重投影, decoding column: all heads of a sequence attend to the same
+// cached rows [c_i | kpe_i] (576 wide), so one 128-row block of queries
+// (head x query token) against a 64-key tile is a dense contraction:
+//   S = Q [128 x 576] . K^T [576 x 64]        (scores)
+//   O += P [128 x 64] . C [64 x 512]          (softmax-weighted latents)
+//
+// Resources decide the shape of the kernel.  O is 128 x 512 fp32 = 256 KB, the
+// whole tensor memory of one SM, and Q is 147 KB of bf16.  So each work unit
+// runs on a cluster of two CTAs on two SMs:
+//   * the score CTA (rank 0) keeps Q in its tensor memory (A operand of a
+//     TS-form MMA), streams full 576-wide key tiles with TMA, computes S into
+//     tensor memory, runs the online softmax in registers and writes P (bf16)
+//     straight into the value CTA's shared memory (distributed shared memory);
+//   * the value CTA (rank 1) streams the 512-wide latent part of the same
+//     tiles with TMA and accumulates O = P . C in all 512 tensor-memory
+//     columns, then normalises and writes the unit's partial output.
+// The score CTA does 53% of the MMA work and the value CTA 47%.
+//
+// Online softmax uses a lazy reference maximum (kept in log2 units): P is
+// exp2(s - m_ref) and m_ref only moves when a tile's maximum exceeds it by more
+// than 8, so the O accumulator is rescaled (tcgen05.ld / st by the value CTA)
+// only on those rare tiles; the final normalisation by the row sum is exact.
+//
+// Work is split evenly over the persistent clusters by 64-key tiles across all
+// (sequence, 128-row block) units; a unit cut between clusters leaves one
+// partial (O / l, lse) per piece, merged by the combine kernel.  Every wait on
+// an mbarrier is bounded in time: on expiry the kernel reports MLA_ERR_TIMEOUT,
+// drains its in-flight copies, frees its tensor memory and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math_constants.h>
+
+#include <mutex>
+
 #include "decode_tc.cuh"
+#include "sm100.cuh"
 
 namespace mla {
+namespace {
 
-bool tc_decode_supported(const mla_dims &, int) { return false; }
-int tc_decode_kernel_launches() { return 2; }
-size_t tc_decode_workspace_bytes(const mla_dims &, int, int) { return 0; }
-int launch_tc_attention(const mla_dims &, int, int, const void *, const CacheView &, const int32_t *, int, void *,
-                        int *, cudaStream_t) {
-  return MLA_ERR_UNSUPPORTED;
+using namespace sm100;
+
+constexpr int kTileKeys = 64;
+constexpr int kDc = 512, kDr = 64, kW = kDc + kDr;
+constexpr int kRows = 128;                         // M of every MMA: query rows per unit
+constexpr int kKStages = 3;                        // key tiles in flight (score CTA)
+constexpr int kVStages = 2;                        // value tiles in flight (value CTA)
+constexpr int kThreads = 256;
+constexpr uint32_t kChunkBytes = kTileKeys * 128;  // one [64 keys x 64 dims] bf16 TMA box, 128B-swizzled
+constexpr uint32_t kKTileBytes = 9 * kChunkBytes;  // 73728
+constexpr uint32_t kVTileBytes = 8 * kChunkBytes;  // 65536
+constexpr uint32_t kPBytes = kRows * kTileKeys * 2;
+constexpr uint32_t kRegionA = kKStages * kKTileBytes;                     // 221184
+constexpr uint32_t kPOff = kVStages * kVTileBytes;                        // P buffers (value CTA)
+static_assert(kPOff + 2 * kPBytes <= kRegionA, "value-CTA tiles must fit the score-CTA region");
+constexpr float kRescaleLog2 = 8.f;
+constexpr uint64_t kWaitNs = 2000000000ull;        // 2 s per wait
+constexpr int kMaxClusters = 128;
+constexpr int kTimeoutRecInts = 1 + 6 * 16;
+
+// TMEM columns
+constexpr uint32_t kQCol = 0;      // score CTA: Q, 288 columns (2 bf16 per column)
+constexpr uint32_t kSCol = 288;    // score CTA: two 64-column S buffers
+// value CTA: O in columns 0..511
+
+// Barrier slots (same indices in both CTAs).
+enum Bar {
+  B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_SFULL = B_KEMPTY + kKStages, B_SEMPTY = B_SFULL + 2,
+  B_QREADY = B_SEMPTY + 2, B_PEMPTY = B_QREADY + 1, B_STATSEMPTY = B_PEMPTY + 2,
+  B_VFULL = B_STATSEMPTY + 1, B_VEMPTY = B_VFULL + kVStages, B_PFULL = B_VEMPTY + kVStages,
+  B_PVDONE = B_PFULL + 2, B_CORR = B_PVDONE + 2, B_STATSFULL = B_CORR + 2,
+  B_OFREE = B_STATSFULL + 1, B_COUNT = B_OFREE + 1
+};
+
+struct SmemB {                       // small region after the tiles
+  float alpha[2][kRows];             // value CTA: per-row rescale factor of each P buffer
+  float stat_l[kRows], stat_m[kRows];// value CTA: row sum and reference max of a finished unit
+  uint64_t bars[B_COUNT];
+  uint32_t tmem_base;
+  int abort;
+  int plan_u0, plan_p0, plan_s0;     // first unit of this cluster, its tile prefix and segment prefix
+  int plan_C;                        // clusters that get work: min(launched clusters, total tiles)
+  int prog[8];                       // per-warp progress (tiles handled), kept for timeout records
+  long long plan_start, plan_end, plan_total;
+};
+constexpr size_t kSmemBytes = 1024 + kRegionA + sizeof(SmemB);
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+struct TcParams {
+  int B, n_q, H, n_rb, U, max_seqlen;
+  const __nv_bfloat16 *q;            // [B, n_q, H, 576]
+  const int32_t *seqlens, *block_table;
+  int max_blocks_per_seq, num_blocks, block_size;
+  float scale_log2;
+  __nv_bfloat16 *o_part;             // [seg][128][512], O / l of each segment
+  float *lse_part;                   // [seg][128]
+  int *seg_info;                     // [U][2]
+  int *timeout_rec;                  // [kTimeoutRecInts]: where bounded waits gave up (diagnostics)
+  int *dev_status;
+};
+
+__device__ __forceinline__ int seq_len_clamped(const TcParams &p, int b) {
+  const int S = p.seqlens[b];
+  return S < 0 ? 0 : (S > p.max_seqlen ? p.max_seqlen : S);
 }
-int launch_tc_combine(const mla_dims &, int, int, const int32_t *, int, const void *, void *, float *, void *,
-                      cudaStream_t) {
-  return MLA_ERR_UNSUPPORTED;
+
+__device__ __forceinline__ int unit_tiles(const TcParams &p, int u) {
+  return (seq_len_clamped(p, u / p.n_rb) + kTileKeys - 1) / kTileKeys;
+}
+
+// Cluster owning global tile t when T tiles are cut into C even ranges
+// [floor(c T / C), floor((c+1) T / C)).
+__device__ __forceinline__ int cluster_of(long long t, long long T, long long C) {
+  return (int)(((t + 1) * C + T - 1) / T - 1);
+}
+
+// Warp-level plan: total tiles, this cluster's range, its first unit and the
+// tile / segment prefixes of that unit.  Every CTA computes the same values.
+__device__ void make_plan(const TcParams &p, SmemB &sb, int cid, int C) {
+  const int lane = threadIdx.x & 31;
+  long long total = 0;
+  for (int u0 = 0; u0 < p.U; u0 += 32) {
+    const int u = u0 + lane;
+    int nt = u < p.U ? unit_tiles(p, u) : 0;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) nt += __shfl_xor_sync(0xffffffffu, nt, o);
+    total += nt;
+  }
+  // With fewer tiles than clusters only the first `total` clusters get work, so
+  // that every active range is non-empty and segment ids have no gaps.
+  C = (int)(total < C ? total : C);
+  const long long start = cid < C ? total * cid / C : 0, end = cid < C ? total * (cid + 1) / C : 0;
+  long long tp = 0, sp = 0;   // running tile / segment prefix
+  int found = -1;
+  long long fp = 0, fs = 0;
+  for (int u0 = 0; u0 < p.U && found < 0; u0 += 32) {
+    const int u = u0 + lane;
+    const int nt = u < p.U ? unit_tiles(p, u) : 0;
+    // inclusive scan of nt
+    int inc = nt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    const long long my_p = tp + inc - nt;
+    int ns = 0;
+    if (nt > 0 && total > 0) ns = cluster_of(my_p + nt - 1, total, C) - cluster_of(my_p, total, C) + 1;
+    int sinc = ns;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, sinc, o);
+      if (lane >= o) sinc += v;
+    }
+    const long long my_s = sp + sinc - ns;
+    const bool hit = u < p.U && nt > 0 && my_p <= start && start < my_p + nt;
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (m) {
+      const int src = __ffs(m) - 1;
+      found = u0 + src;
+      fp = __shfl_sync(0xffffffffu, my_p, src);
+      fs = __shfl_sync(0xffffffffu, my_s, src);
+    }
+    tp += __shfl_sync(0xffffffffu, inc, 31);
+    sp += __shfl_sync(0xffffffffu, sinc, 31);
+  }
+  if (lane == 0) {
+    sb.plan_C = C;
+    sb.plan_total = total;
+    sb.plan_start = start;
+    sb.plan_end = (found < 0 || cid >= C) ? start : end;
+    sb.plan_u0 = found < 0 ? 0 : found;
+    sb.plan_p0 = (int)fp;
+    sb.plan_s0 = (int)fs;
+  }
+}
+
+// Iterates the (unit, tile range) segments of this cluster.
+struct SegIter {
+  int u, prefix, seg_prefix;
+  long long pos, end, total;
+  int C;
+  __device__ bool next(const TcParams &p, int cid, int &b, int &rb, int &t0, int &t1, int &segid, bool &first_of_unit,
+                       int &nseg_unit) {
+    while (pos < end && u < p.U) {
+      const int nt = unit_tiles(p, u);
+      const long long lo = pos > prefix ? pos : prefix;
+      const long long hi = end < (long long)prefix + nt ? end : (long long)prefix + nt;
+      const int c0 = nt > 0 ? cluster_of(prefix, total, C) : 0;
+      const int ns = nt > 0 ? cluster_of((long long)prefix + nt - 1, total, C) - c0 + 1 : 0;
+      if (lo < hi) {
+        b = u / p.n_rb;
+        rb = u % p.n_rb;
+        t0 = (int)(lo - prefix);
+        t1 = (int)(hi - prefix);
+        segid = seg_prefix + (cid - c0);
+        first_of_unit = (lo == prefix);
+        nseg_unit = ns;
+        const int cur_u = u;
+        // advance
+        pos = hi;
+        if (hi == (long long)prefix + nt) {
+          prefix += nt;
+          seg_prefix += ns;
+          u = cur_u + 1;
+        }
+        return true;
+      }
+      prefix += nt;
+      seg_prefix += ns;
+      ++u;
+    }
+    return false;
+  }
+};
+
+// Bounded wait that turns a timeout into the CTA-wide abort state.  The first
+// timeout of each (CTA rank, warp) in the grid is recorded in rec[1 + 6 * (8 * rank + warp) ..]:
+// cluster, barrier slot, parity, source line, the warp's progress counter.
+__device__ __forceinline__ bool wait_or_abort(SmemB &sb, uint32_t bar, uint32_t parity, int *dev_status,
+                                              bool cluster_scope = false, int *rec = nullptr, int tag = 0) {
+  if (*(volatile int *)&sb.abort) return false;
+  if (mbar_wait(bar, parity, kWaitNs, cluster_scope)) return true;
+  *(volatile int *)&sb.abort = 1;
+  report(dev_status, MLA_ERR_TIMEOUT);
+  if (rec) {
+    const int w = (int)(threadIdx.x >> 5);
+    int *e = rec + 1 + 6 * (8 * (int)cluster_ctarank() + w);
+    if (atomicCAS(e, 0, 1) == 0) {
+      e[1] = (int)cluster_id_x();
+      e[2] = (int)((bar - smem_u32(&sb.bars[0])) / 8);
+      e[3] = (int)parity;
+      e[4] = tag;
+      e[5] = sb.prog[w];
+    }
+    atomicAdd(rec, 1);
+  }
+  return false;
+}
+
+// Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, and then
+// every lane observes the completed phase itself (acquire for its own reads).
+// The phase cannot move on in between: the next completion of the same
+// barrier needs an arrival from this warp.
+__device__ __forceinline__ bool warp_wait(SmemB &sb, uint32_t bar, uint32_t parity, int *dev_status,
+                                          bool cluster_scope = false, int *rec = nullptr, int tag = 0) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = wait_or_abort(sb, bar, parity, dev_status, cluster_scope, rec, tag) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_wait(bar, parity, kWaitNs, cluster_scope);
+  return ok != 0;
+}
+
+__device__ __forceinline__ int64_t tile_row(const TcParams &p, int b, int t) {
+  const int key = t * kTileKeys;
+  const int lb = key / p.block_size;
+  if (lb >= p.max_blocks_per_seq) return -1;
+  const int blk = p.block_table ? p.block_table[(int64_t)b * p.max_blocks_per_seq + lb]
+                                : b * p.max_blocks_per_seq + lb;
+  if (blk < 0 || blk >= p.num_blocks) return -1;
+  return (int64_t)blk * p.block_size + (key % p.block_size);
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_pe,
+                     const TcParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *tiles = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemB &sb = *reinterpret_cast<SmemB *>(tiles + kRegionA);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cid = (int)cluster_id_x();
+  const int C = (int)nclusters_x();
+  auto bar = [&](int i) { return smem_u32(&sb.bars[i]); };
+  const uint32_t peer = rank ^ 1u;
+
+  if (threadIdx.x == 0 && cid == 0 && rank == 0)
+    for (int i = 0; i < kTimeoutRecInts; ++i) p.timeout_rec[i] = 0;
+  if (threadIdx.x < 8) sb.prog[threadIdx.x] = 0;
+  if (threadIdx.x == 0) {
+    const uint32_t counts[B_COUNT] = {
+        1, 1, 1,          // K full
+        1, 1, 1,          // K empty
+        1, 1,             // S full
+        4, 4,             // S empty (one per softmax warp)
+        4,                // Q ready
+        1, 1,             // P empty (relay arrives remotely)
+        4,                // stats empty (remote, one per value-CTA epilogue warp)
+        1, 1,             // V full
+        1, 1,             // V empty
+        kRows, kRows,     // P full (remote, every softmax thread)
+        1, 1,             // PV done
+        kRows, kRows,     // tile checked: tail rows zeroed and O rescaled where needed (by tile parity)
+        kRows,            // stats full (remote, every softmax thread)
+        kRows};           // O free
+    for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
+    sb.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 3) {
+    tmem_alloc(smem_u32(&sb.tmem_base), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0) make_plan(p, sb, cid, C);
+  if (threadIdx.x == 32) {
+    tma_prefetch_desc(&map_c);
+    tma_prefetch_desc(&map_pe);
+  }
+  tc_fence_before();
+  cluster_sync();   // barriers initialised in both CTAs before any remote arrive
+  tc_fence_after();
+  const uint32_t tbase = sb.tmem_base;
+
+  SegIter it0;
+  it0.u = sb.plan_u0;
+  it0.prefix = sb.plan_p0;
+  it0.seg_prefix = sb.plan_s0;
+  it0.pos = sb.plan_start;
+  it0.end = sb.plan_end;
+  it0.total = sb.plan_total;
+  it0.C = sb.plan_C;
+
+  int b, rb, t0, t1, segid, nseg;
+  bool first_u;
+
+  if (rank == 0) {
+    // ============================ score CTA ============================
+    if (warp == 0 && lane == 0) {
+      // ---- key-tile producer
+      SegIter it = it0;
+      uint32_t n = 0;
+      uint32_t uses[kKStages] = {0, 0, 0};
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        for (int t = t0; t < t1; ++t, ++n) {
+          sb.prog[warp] = (int)n;
+          const int s = n % kKStages;
+          if (n >= kKStages && !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done0;
+          int64_t row = tile_row(p, b, t);
+          if (row < 0) {
+            report(p.dev_status, MLA_ERR_BAD_INDEX);
+            row = 0;
+          }
+          const uint32_t dst = smem_u32(tiles + s * kKTileBytes);
+          mbar_expect_tx(bar(B_KFULL + s), kKTileBytes);
+          for (int j = 0; j < 8; ++j) tma_load_2d(dst + j * kChunkBytes, &map_c, 64 * j, (int32_t)row, bar(B_KFULL + s));
+          tma_load_2d(dst + 8 * kChunkBytes, &map_pe, 0, (int32_t)row, bar(B_KFULL + s));
+          ++uses[s];
+        }
+      }
+    prod_done0:
+      // Drain: the last load issued on each stage must have landed before exit.
+      for (int s = 0; s < kKStages; ++s)
+        if (uses[s]) mbar_wait(bar(B_KFULL + s), (uses[s] - 1) & 1, kWaitNs);
+    } else if (warp == 1 && lane == 0) {
+      // ---- MMA issuer: S = Q . K^T
+      SegIter it = it0;
+      uint32_t n = 0, ns = 0, uc = 0;
+      const uint32_t idesc = idesc_bf16_f32(kRows, kTileKeys, false, false);
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        if (!wait_or_abort(sb, bar(B_QREADY), uc & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int t = t0; t < t1; ++t, ++n, ++ns) {
+          sb.prog[warp] = (int)n;
+          const int s = n % kKStages;
+          const int sbuf = ns & 1;
+          if (!wait_or_abort(sb, bar(B_KFULL + s), (n / kKStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          if (ns >= 2 && !wait_or_abort(sb, bar(B_SEMPTY + sbuf), ((ns >> 1) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kt = smem_u32(tiles + s * kKTileBytes);
+          const uint32_t d = tbase + kSCol + 64 * sbuf;
+#pragma unroll 4
+          for (int k = 0; k < kW / 16; ++k) {
+            const uint64_t bd = smem_desc_sw128(kt + (k >> 2) * kChunkBytes + (k & 3) * 32, 16, 1024);
+            mma_ts(d, tbase + kQCol + 8 * k, bd, idesc, k > 0);
+          }
+          tc_commit(bar(B_SFULL + sbuf));
+          tc_commit(bar(B_KEMPTY + s));
+        }
+        if (!ok) break;
+        ++uc;
+      }
+    } else if (warp >= 4) {
+      // ---- softmax: thread = one query row (TMEM lane)
+      const int r = (warp - 4) * 32 + lane;
+      const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+      SegIter it = it0;
+      uint32_t ns = 0, np = 0, uc = 0;
+      const uint32_t pbuf_local = smem_u32(tiles + kPOff);
+      const uint32_t pbuf_remote = mapa(pbuf_local, peer);
+      const uint32_t alpha_remote = mapa(smem_u32(&sb.alpha[0][0]), peer);
+      const uint32_t statl_remote = mapa(smem_u32(&sb.stat_l[0]), peer);
+      const uint32_t statm_remote = mapa(smem_u32(&sb.stat_m[0]), peer);
+      const uint32_t pfull_remote = mapa(bar(B_PFULL), peer);
+      const uint32_t statsfull_remote = mapa(bar(B_STATSFULL), peer);
+      const int nrows = p.n_q * p.H;
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        // Q row -> tensor memory (the previous unit's MMAs are complete: its last S was consumed).
+        const int gr = rb * kRows + r;
+        const bool real = gr < nrows;
+        {
+          const uint4 *src = reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * nrows + (real ? gr : 0)) * kW);
+#pragma unroll 1
+          for (int c = 0; c < 9; ++c) {
+            uint32_t v[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              uint4 x = real ? __ldg(src + c * 8 + i) : make_uint4(0, 0, 0, 0);
+              v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+            }
+            tmem_st32(tbase + lane_off + kQCol + 32 * c, v);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_QREADY));
+        }
+        const int S = seq_len_clamped(p, b);
+        const int j = real ? gr / p.H : 0;
+        const int visible = real ? S - p.n_q + j + 1 : 0;
+        float m_ref = -CUDART_INF_F, l = 0.f;
+        bool ok = true;
+        for (int t = t0; t < t1; ++t, ++ns, ++np) {
+          if (lane == 0) sb.prog[warp] = (int)np;
+          const int sbuf = ns & 1;
+          if (!warp_wait(sb, bar(B_SFULL + sbuf), (ns >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t sraw[64];
+          {
+            uint32_t a[32], c2[32];
+            tmem_ld32(tbase + lane_off + kSCol + 64 * sbuf, a);
+            tmem_ld32(tbase + lane_off + kSCol + 64 * sbuf + 32, c2);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { sraw[i] = a[i]; sraw[32 + i] = c2[i]; }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
+          const int nvalid = visible - t * kTileKeys;     // keys k < nvalid are visible
+          float mx = -CUDART_INF_F;
+#pragma unroll
+          for (int k = 0; k < 64; ++k)
+            if (k < nvalid) mx = fmaxf(mx, __uint_as_float(sraw[k]) * p.scale_log2);
+          float alpha = 1.f;
+          const bool need = mx > m_ref + kRescaleLog2;
+          if (need) {
+            alpha = exp2f(m_ref - mx);
+            l *= alpha;
+            m_ref = mx;
+          }
+          uint32_t pk[32];
+          float psum = 0.f;
+#pragma unroll
+          for (int k = 0; k < 64; k += 2) {
+            float p0 = (k < nvalid) ? exp2f(__uint_as_float(sraw[k]) * p.scale_log2 - m_ref) : 0.f;
+            float p1 = (k + 1 < nvalid) ? exp2f(__uint_as_float(sraw[k + 1]) * p.scale_log2 - m_ref) : 0.f;
+            const uint32_t pr = pack_bf16x2(p0, p1);
+            pk[k >> 1] = pr;
+            psum += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xffff0000u);
+          }
+          l += psum;
+          const int pb = np & 1;
+          if (np >= 2 && !warp_wait(sb, bar(B_PEMPTY + pb), ((np >> 1) - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) { ok = false; break; }
+          // P row r -> value CTA, K-major 128B-swizzled [128 rows x 64 keys] tile.
+          const uint32_t rowbase = pbuf_remote + pb * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_cluster_v4(rowbase + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          st_cluster_f32(alpha_remote + (pb * kRows + r) * 4, alpha);
+          fence_proxy_async_cluster();
+          mbar_arrive_cluster(pfull_remote + 8 * pb);
+        }
+        if (!ok) break;
+        // Unit statistics -> value CTA.
+        if (uc > 0 && !warp_wait(sb, bar(B_STATSEMPTY), (uc - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) break;
+        st_cluster_f32(statl_remote + r * 4, l);
+        st_cluster_f32(statm_remote + r * 4, m_ref);
+        mbar_arrive_cluster(statsfull_remote);
+        ++uc;
+      }
+    }
+  } else {
+    // ============================ value CTA ============================
+    if (warp == 0 && lane == 0) {
+      // ---- latent-tile producer (c_KV part only)
+      if (cid == 0) {
+        // Units with no tiles get an empty segment list (their rows combine to zero).
+        for (int u = 0; u < p.U; ++u)
+          if (unit_tiles(p, u) == 0) {
+            p.seg_info[2 * u] = 0;
+            p.seg_info[2 * u + 1] = 0;
+          }
+        for (int bb = 0; bb < p.B; ++bb) {
+          const int S = p.seqlens[bb];
+          if (S < p.n_q || S > p.max_seqlen) report(p.dev_status, MLA_ERR_BAD_INDEX);
+        }
+      }
+      SegIter it = it0;
+      uint32_t n = 0;
+      uint32_t uses[kVStages] = {0, 0};
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        if (first_u) {
+          // This cluster holds the unit's first tile: publish where its partials live.
+          p.seg_info[2 * (b * p.n_rb + rb)] = segid;
+          p.seg_info[2 * (b * p.n_rb + rb) + 1] = nseg;
+        }
+        for (int t = t0; t < t1; ++t, ++n) {
+          sb.prog[warp] = (int)n;
+          const int s = n % kVStages;
+          if (n >= kVStages && !wait_or_abort(sb, bar(B_VEMPTY + s), ((n / kVStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done1;
+          int64_t row = tile_row(p, b, t);
+          if (row < 0) row = 0;   // reported by the score CTA
+          const uint32_t dst = smem_u32(tiles + s * kVTileBytes);
+          mbar_expect_tx(bar(B_VFULL + s), kVTileBytes);
+          for (int j = 0; j < 8; ++j) tma_load_2d(dst + j * kChunkBytes, &map_c, 64 * j, (int32_t)row, bar(B_VFULL + s));
+          ++uses[s];
+        }
+      }
+    prod_done1:
+      for (int s = 0; s < kVStages; ++s)
+        if (uses[s]) mbar_wait(bar(B_VFULL + s), (uses[s] - 1) & 1, kWaitNs);
+    } else if (warp == 1 && lane == 0) {
+      // ---- MMA issuer: O += P . C
+      SegIter it = it0;
+      uint32_t n = 0, np = 0, uc = 0;
+      const uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        if (uc > 0 && !wait_or_abort(sb, bar(B_OFREE), (uc - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
+        bool ok = true;
+        for (int t = t0; t < t1; ++t, ++n, ++np) {
+          if (lane == 0) sb.prog[warp] = (int)n;
+          const int s = n % kVStages, pb = np & 1;
+          if (!wait_or_abort(sb, bar(B_VFULL + s), (n / kVStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          if (!wait_or_abort(sb, bar(B_PFULL + pb), (np >> 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) { ok = false; break; }
+          // The epilogue warps have zeroed tail rows and rescaled O for this tile.
+          // Two slots: the epilogue warps may run up to two tiles ahead of this thread, and one
+          // barrier would then complete two phases before it is observed.
+          if (!wait_or_abort(sb, bar(B_CORR + (n & 1)), (n >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          tc_fence_after();
+          fence_proxy_async_smem();
+          const uint32_t vt = smem_u32(tiles + s * kVTileBytes);
+          const uint32_t pt = smem_u32(tiles + kPOff + pb * kPBytes);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint64_t ad = smem_desc_sw128(pt + ks * 32, 16, 1024);
+              const uint64_t bd = smem_desc_sw128(vt + h * 4 * kChunkBytes + ks * 2048, kChunkBytes, 1024);
+              mma_ss(tbase + 256 * h, ad, bd, idesc, (t != t0 || ks > 0) ? 1u : 0u);
+            }
+          tc_commit(bar(B_PVDONE + pb));
+          tc_commit(bar(B_VEMPTY + s));
+        }
+        if (!ok) break;
+        ++uc;
+      }
+    } else if (warp == 2 && lane == 0) {
+      // ---- relay: a P buffer is free once the MMAs that read it completed
+      SegIter it = it0;
+      uint32_t np = 0;
+      const uint32_t pempty_remote = mapa(bar(B_PEMPTY), peer);
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        bool ok = true;
+        for (int t = t0; t < t1; ++t, ++np) {
+          sb.prog[warp] = (int)np;
+          const int pb = np & 1;
+          if (!wait_or_abort(sb, bar(B_PVDONE + pb), (np >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          mbar_arrive_cluster(pempty_remote + 8 * pb);
+        }
+        if (!ok) break;
+      }
+    } else if (warp >= 4) {
+      // ---- tail zeroing, O rescaling and the unit epilogue
+      const int r = (warp - 4) * 32 + lane;
+      const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+      SegIter it = it0;
+      uint32_t n = 0, np = 0, uc = 0;
+      const uint32_t statsempty_remote = mapa(bar(B_STATSEMPTY), peer);
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        const int S = seq_len_clamped(p, b);
+        bool ok = true;
+        for (int t = t0; t < t1; ++t, ++n, ++np) {
+          if (lane == 0) sb.prog[warp] = (int)n;
+          const int s = n % kVStages, pb = np & 1;
+          if (!warp_wait(sb, bar(B_PFULL + pb), (np >> 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) { ok = false; break; }
+          if ((t + 1) * kTileKeys > S) {
+            // Rows past the sequence end may hold anything (NaN): zero them so 0 * row stays 0.
+            if (!warp_wait(sb, bar(B_VFULL + s), (n / kVStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            const int nv = S - t * kTileKeys;
+            unsigned char *vt = tiles + s * kVTileBytes;
+            const int nrow = kTileKeys - nv;
+            for (int e = threadIdx.x - 128; e < nrow * 8 * 8; e += 128) {
+              const int row = nv + e / 64, rest = e % 64, ch = rest / 8, piece = rest % 8;
+              *reinterpret_cast<uint4 *>(vt + ch * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
+          // Rescale O where this tile moved a row's reference maximum (warp-uniform: tcgen05.ld/st
+          // are warp-collective; rows that did not move carry alpha = 1).
+          const float a = sb.alpha[pb][r];
+          if (__any_sync(0xffffffffu, a != 1.f && t != t0)) {
+            // All earlier PV MMAs must be complete before O is read back.
+            if (!warp_wait(sb, bar(B_PVDONE + ((np - 1) & 1)), ((np - 1) >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 16; ++c) {
+              uint32_t v[32];
+              tmem_ld32(tbase + lane_off + 32 * c, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+              tmem_st32(tbase + lane_off + 32 * c, v);
+            }
+            tmem_wait_st();
+          }
+          tc_fence_before();
+          mbar_arrive(bar(B_CORR + (n & 1)));
+        }
+        if (!ok) break;
+        // Epilogue: wait for the unit's last MMAs and the row statistics.
+        if (!warp_wait(sb, bar(B_PVDONE + ((np - 1) & 1)), ((np - 1) >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
+        if (!warp_wait(sb, bar(B_STATSFULL), uc & 1, p.dev_status, true, p.timeout_rec, __LINE__)) break;
+        tc_fence_after();
+        const float l = sb.stat_l[r], m = sb.stat_m[r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(statsempty_remote);
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16 *dst = p.o_part + ((int64_t)segid * kRows + r) * kDc;
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tbase + lane_off + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; i += 8)
+            *reinterpret_cast<uint4 *>(dst + 32 * c + i) =
+                make_uint4(pack_bf16x2(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
+                           pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
+                           pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
+                           pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
+        }
+        p.lse_part[(int64_t)segid * kRows + r] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+        tc_fence_before();
+        mbar_arrive(bar(B_OFREE));
+        ++uc;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 3) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+  cluster_sync();   // no CTA leaves while its peer may still touch its shared memory
+}
+
+// ------------------------------------------------------------ combine (+ W_UV)
+constexpr int kCombRows = 16;
+constexpr int kCombThreads = 256;
+constexpr int kMaxSegPerUnit = kMaxClusters + 1;
+
+__global__ void __launch_bounds__(kCombThreads)
+tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part, const float *lse_part,
+                  const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out) {
+  extern __shared__ float smem[];
+  float *ol = smem;                         // [kCombRows][512]
+  float *wgt = ol + kCombRows * kDc;        // [kCombRows][kMaxSegPerUnit]
+  int *sinfo = reinterpret_cast<int *>(wgt + kCombRows * kMaxSegPerUnit);   // [kCombRows][3]
+  const int s = blockIdx.x;
+  const int g0 = blockIdx.y * kCombRows;
+  const int rows = B * n_q;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int rr = warp; rr < kCombRows; rr += 8) {
+    const int g = g0 + rr;
+    int s0 = 0, ns = 0, lr = 0;
+    if (g < rows) {
+      const int b = g / n_q, j = g % n_q;
+      const int gr = j * H + s;
+      const int u = b * n_rb + gr / kRows;
+      lr = gr % kRows;
+      s0 = seg_info[2 * u];
+      ns = seg_info[2 * u + 1];
+      ns = ns < 0 ? 0 : (ns > kMaxSegPerUnit ? kMaxSegPerUnit : ns);
+      if (s0 < 0 || s0 + ns > max_segs) { s0 = 0; ns = 0; }
+    }
+    float m = -CUDART_INF_F;
+    for (int k = lane; k < ns; k += 32) m = fmaxf(m, lse_part[(int64_t)(s0 + k) * kRows + lr]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+    for (int k = lane; k < ns; k += 32) {
+      const float e = m == -CUDART_INF_F ? 0.f : __expf(lse_part[(int64_t)(s0 + k) * kRows + lr] - m);
+      wgt[rr * kMaxSegPerUnit + k] = e;
+      sum += e;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    for (int k = lane; k < ns; k += 32) wgt[rr * kMaxSegPerUnit + k] *= inv;
+    if (lane == 0) {
+      sinfo[3 * rr] = s0;
+      sinfo[3 * rr + 1] = ns;
+      sinfo[3 * rr + 2] = lr;
+      if (g < rows && lse_out) lse_out[(int64_t)g * H + s] = sum > 0.f ? m + logf(sum) : -CUDART_INF_F;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < kCombRows * kDc; e += kCombThreads) {
+    const int rr = e / kDc, c = e % kDc;
+    const int s0 = sinfo[3 * rr], ns = sinfo[3 * rr + 1], lr = sinfo[3 * rr + 2];
+    float v = 0.f;
+    for (int k = 0; k < ns; ++k) {
+      const float w = wgt[rr * kMaxSegPerUnit + k];
+      if (w != 0.f) v = fmaf(w, __bfloat162float(o_part[((int64_t)(s0 + k) * kRows + lr) * kDc + c]), v);
+    }
+    ol[e] = v;
+  }
+  __syncthreads();
+  if (!w_uv) {
+    for (int e = tid; e < kCombRows * kDc; e += kCombThreads) {
+      const int rr = e / kDc, c = e % kDc, g = g0 + rr;
+      if (g < rows) out[((int64_t)g * H + s) * kDc + c] = __float2bfloat16_rn(ol[e]);
+    }
+    return;
+  }
+  const __nv_bfloat16 *w = w_uv + (int64_t)s * kDc * d_v;
+  for (int v = tid; v < d_v; v += kCombThreads) {
+    float acc[kCombRows];
+#pragma unroll
+    for (int rr = 0; rr < kCombRows; ++rr) acc[rr] = 0.f;
+    for (int c = 0; c < kDc; ++c) {
+      const float wv = __bfloat162float(w[(int64_t)c * d_v + v]);
+#pragma unroll
+      for (int rr = 0; rr < kCombRows; ++rr) acc[rr] = fmaf(ol[rr * kDc + c], wv, acc[rr]);
+    }
+#pragma unroll
+    for (int rr = 0; rr < kCombRows; ++rr) {
+      const int g = g0 + rr;
+      if (g < rows) out[((int64_t)g * H + s) * d_v + v] = __float2bfloat16_rn(acc[rr]);
+    }
+  }
+}
+
+// ------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+int make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint64_t row_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return MLA_ERR_CUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {64, 64};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+struct WsLayout {
+  size_t seg_info, o_part, lse_part, total;
+};
+
+int clusters_for_device();
+
+// Partials: one per (unit, cluster) piece, at most U + C - 1 pieces for C clusters.
+WsLayout ws_layout(int B, int n_rb) {
+  auto a256 = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t U = (size_t)B * n_rb;
+  const int C = clusters_for_device();
+  const size_t segs = U + (C > 0 ? C : kMaxClusters);
+  WsLayout L;
+  L.seg_info = 0;
+  L.o_part = a256(U * 2 * sizeof(int) + kTimeoutRecInts * sizeof(int));
+  L.lse_part = L.o_part + a256(segs * kRows * kDc * sizeof(__nv_bfloat16));
+  L.total = L.lse_part + a256(segs * kRows * sizeof(float));
+  return L;
+}
+
+// Clusters of two CTAs that fit on the current device at once (0 without a device).
+int clusters_for_device() {
+  static int cached[128] = {0};
+  int dev = 0, ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev <= 0) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
+  if (cached[dev]) return cached[dev];
+  if (cudaFuncSetAttribute(mla_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes))
+    return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * kMaxClusters);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, mla_decode_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    n = sms / 2;
+  }
+  if (n > kMaxClusters) n = kMaxClusters;
+  cached[dev] = n;
+  return n;
+}
+
+}  // namespace
+
+bool tc_decode_supported(const mla_dims &d, int n_q) {
+  return d.dtype == MLA_BF16 && d.d_c == kDc && d.d_rope == kDr && d.block_size % kTileKeys == 0 &&
+         d.ckv_stride % 8 == 0 && d.kpe_stride % 8 == 0 && d.d_v <= 1024 && n_q * d.n_heads <= 2 * kRows;
+}
+
+int tc_decode_kernel_launches() { return 2; }
+
+size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q) {
+  const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
+  return ws_layout(B, n_rb).total;
+}
+
+int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, const CacheView &cache,
+                        const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st) {
+  if ((reinterpret_cast<uintptr_t>(cache.c_kv) & 15) || (reinterpret_cast<uintptr_t>(cache.k_pe) & 15) ||
+      (reinterpret_cast<uintptr_t>(q_abs) & 15))
+    return MLA_ERR_INVALID_ARG;
+  const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
+  const WsLayout L = ws_layout(B, n_rb);
+  char *w = static_cast<char *>(ws);
+  CUtensorMap mc, mpe;
+  const uint64_t rows = (uint64_t)cache.num_blocks * cache.block_size;
+  int rc = make_map(&mc, cache.c_kv, kDc, rows, (uint64_t)cache.ckv_stride * 2);
+  if (rc) return rc;
+  if ((rc = make_map(&mpe, cache.k_pe, kDr, rows, (uint64_t)cache.kpe_stride * 2))) return rc;
+  const int C = clusters_for_device();
+  if (C <= 0) return MLA_ERR_CUDA;
+  TcParams p;
+  p.B = B;
+  p.n_q = n_q;
+  p.H = d.n_heads;
+  p.n_rb = n_rb;
+  p.U = B * n_rb;
+  p.max_seqlen = max_seqlen;
+  p.q = static_cast<const __nv_bfloat16 *>(q_abs);
+  p.seqlens = seqlens;
+  p.block_table = cache.block_table;
+  p.max_blocks_per_seq = cache.max_blocks_per_seq;
+  p.num_blocks = cache.num_blocks;
+  p.block_size = cache.block_size;
+  p.scale_log2 = default_scale(d) * 1.4426950408889634f;
+  p.o_part = reinterpret_cast<__nv_bfloat16 *>(w + L.o_part);
+  p.lse_part = reinterpret_cast<float *>(w + L.lse_part);
+  p.seg_info = reinterpret_cast<int *>(w + L.seg_info);
+  p.timeout_rec = p.seg_info + 2 * p.U;
+  p.dev_status = dev_status;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * C);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  if (cudaLaunchKernelEx(&cfg, mla_decode_tc_kernel, mc, mpe, p) != cudaSuccess) return MLA_ERR_CUDA;
+  return MLA_OK;
+}
+
+int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
+                      void *out, float *lse, void *ws, cudaStream_t st) {
+  (void)seqlens;
+  (void)max_seqlen;
+  const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
+  const WsLayout L = ws_layout(B, n_rb);
+  char *w = static_cast<char *>(ws);
+  const size_t smem = sizeof(float) * (kCombRows * kDc + kCombRows * kMaxSegPerUnit) + sizeof(int) * 3 * kCombRows;
+  if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+    return MLA_ERR_CUDA;
+  const dim3 grid(d.n_heads, (B * n_q + kCombRows - 1) / kCombRows);
+  tc_combine_kernel<<<grid, kCombThreads, smem, st>>>(
+      B, n_q, d.n_heads, n_rb, B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
+      reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part), reinterpret_cast<const float *>(w + L.lse_part),
+      static_cast<const __nv_bfloat16 *>(w_uv), d.d_v, static_cast<__nv_bfloat16 *>(out), lse);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 }  // namespace mla
