@@ -43,42 +43,60 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTileKeys = 64;
+constexpr int kTileKeys = 64;                      // one cache page of keys (a "page tile")
+constexpr int kSuper = 4;                          // page tiles per score tile: N = 256 keys per MMA
 constexpr int kDc = 512, kDr = 64, kW = kDc + kDr;
 constexpr int kRows = 128;                         // M of every MMA: query rows per unit
-constexpr int kKStages = 3;                        // key tiles in flight (score CTA)
-constexpr int kVStages = 2;                        // value tiles in flight (value CTA)
-constexpr int kThreads = 256;
+constexpr int kKStages = 6;                        // score CTA: [256 keys x 64 dims] stages in flight
+constexpr int kVStages = 2;                        // value CTA: [64 keys x 512 dims] stages in flight
+constexpr int kThreads = 384;
+constexpr int kLaunchRegs = 168;                   // per thread at launch (65536 / 384, rounded down to 8)
+constexpr int kLowRegs = 56, kHighRegs = 224;
+static_assert(128 * kLowRegs + 256 * kHighRegs == kThreads * kLaunchRegs, "register split must match the launch");
 constexpr uint32_t kChunkBytes = kTileKeys * 128;  // one [64 keys x 64 dims] bf16 TMA box, 128B-swizzled
-constexpr uint32_t kKTileBytes = 9 * kChunkBytes;  // 73728
-constexpr uint32_t kVTileBytes = 8 * kChunkBytes;  // 65536
-constexpr uint32_t kPBytes = kRows * kTileKeys * 2;
-constexpr uint32_t kRegionA = kKStages * kKTileBytes;                     // 221184
-constexpr uint32_t kPOff = kVStages * kVTileBytes;                        // P buffers (value CTA)
-static_assert(kPOff + 2 * kPBytes <= kRegionA, "value-CTA tiles must fit the score-CTA region");
+constexpr uint32_t kKStageBytes = kSuper * kChunkBytes;            // 32768
+constexpr uint32_t kVTileBytes = 8 * kChunkBytes;                  // 65536
+constexpr uint32_t kPBytes = kRows * kTileKeys * 2;                // 16384
+constexpr int kPSlots = 5;                         // P page tiles in flight from the score CTA to the value CTA
+constexpr uint32_t kPTxBytes = kPBytes + kRows * 4 + 4 * 4;       // P tile + alpha column + 4 warp flags
+constexpr uint32_t kQpeOff = 0;                                    // score CTA: Q rope part, [128 x 64] bf16
+constexpr uint32_t kKOff = kRows * 128;                            // score CTA: key stages
+constexpr uint32_t kPOff = kVStages * kVTileBytes;                 // value CTA: P slots
+constexpr uint32_t kRegionA = kKOff + kKStages * kKStageBytes;     // 212992
+static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint64_t kWaitNs = 2000000000ull;        // 2 s per wait
 constexpr int kMaxClusters = 128;
 constexpr int kTimeoutRecInts = 1 + 6 * 16;
 
 // TMEM columns
-constexpr uint32_t kQCol = 0;      // score CTA: Q, 288 columns (2 bf16 per column)
-constexpr uint32_t kSCol = 288;    // score CTA: two 64-column S buffers
+constexpr uint32_t kQCol = 0;      // score CTA: latent part of Q, 256 columns (2 bf16 per column)
+constexpr uint32_t kSCol = 256;    // score CTA: S, 256 columns (one score tile)
 // value CTA: O in columns 0..511
 
 // Barrier slots (same indices in both CTAs).
 enum Bar {
-  B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_SFULL = B_KEMPTY + kKStages, B_SEMPTY = B_SFULL + 2,
-  B_QREADY = B_SEMPTY + 2, B_PEMPTY = B_QREADY + 1, B_STATSEMPTY = B_PEMPTY + 2,
+  B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_SFULL = B_KEMPTY + kKStages, B_SEMPTY = B_SFULL + 1,
+  B_QREADY = B_SEMPTY + 1, B_PEMPTY = B_QREADY + 1, B_STATSEMPTY = B_PEMPTY + kPSlots,
   B_VFULL = B_STATSEMPTY + 1, B_VEMPTY = B_VFULL + kVStages, B_PFULL = B_VEMPTY + kVStages,
-  B_PVDONE = B_PFULL + 2, B_CORR = B_PVDONE + 2, B_STATSFULL = B_CORR + 2,
+  B_PVDONE = B_PFULL + kPSlots, B_REQ = B_PVDONE + kPSlots, B_REQDONE = B_REQ + 1, B_STATSFULL = B_REQDONE + 1,
   B_OFREE = B_STATSFULL + 1, B_COUNT = B_OFREE + 1
 };
 
+// A request from the value CTA's MMA thread to its epilogue warps.
+struct Req {
+  int kind;        // 0: fix up a tile before its MMA, 1: unit epilogue
+  int vstage, slot, nvalid, tail, rescale, segid, last_slot, last_parity;
+};
+
 struct SmemB {                       // small region after the tiles
-  float alpha[2][kRows];             // value CTA: per-row rescale factor of each P buffer
+  float alpha[kPSlots][kRows];       // value CTA: per-row rescale factor of each P slot
+  uint32_t flags[kPSlots][4];        // value CTA: per softmax warp, "some row of this tile rescaled"
   float stat_l[kRows], stat_m[kRows];// value CTA: row sum and reference max of a finished unit
+  float xmax[2][2][kRows];           // score CTA: the two softmax halves' tile maxima (double-buffered)
+  float xl[2][kRows];                // score CTA: the two halves' row sums at the end of a unit
   uint64_t bars[B_COUNT];
+  Req req;
   uint32_t tmem_base;
   int abort;
   int plan_u0, plan_p0, plan_s0;     // first unit of this cluster, its tile prefix and segment prefix
@@ -281,22 +299,18 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
     for (int i = 0; i < kTimeoutRecInts; ++i) p.timeout_rec[i] = 0;
   if (threadIdx.x < 8) sb.prog[threadIdx.x] = 0;
   if (threadIdx.x == 0) {
-    const uint32_t counts[B_COUNT] = {
-        1, 1, 1,          // K full
-        1, 1, 1,          // K empty
-        1, 1,             // S full
-        4, 4,             // S empty (one per softmax warp)
-        4,                // Q ready
-        1, 1,             // P empty (relay arrives remotely)
-        4,                // stats empty (remote, one per value-CTA epilogue warp)
-        1, 1,             // V full
-        1, 1,             // V empty
-        kRows, kRows,     // P full (remote, every softmax thread)
-        1, 1,             // PV done
-        kRows, kRows,     // tile checked: tail rows zeroed and O rescaled where needed (by tile parity)
-        kRows,            // stats full (remote, every softmax thread)
-        kRows};           // O free
+    uint32_t counts[B_COUNT];
+    for (int i = 0; i < B_COUNT; ++i) counts[i] = 1;
+    counts[B_SEMPTY] = 8;                             // one per softmax warp
+    counts[B_QREADY] = 8;
+    counts[B_STATSEMPTY] = 4;                         // remote, one per value-CTA epilogue warp
+    // P full: one local arrival (the relay arms the expected bytes); the bytes arrive by st.async.
+    counts[B_REQDONE] = kRows;
+    counts[B_STATSFULL] = kRows;                      // remote, every softmax thread
+    counts[B_OFREE] = kRows;
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
+    if (rank == 1)
+      for (int i = 0; i < kPSlots; ++i) mbar_expect_tx(bar(B_PFULL + i), kPTxBytes);
     sb.abort = 0;
     fence_mbar_init();
   }
@@ -326,166 +340,90 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   int b, rb, t0, t1, segid, nseg;
   bool first_u;
 
-  if (rank == 0) {
-    // ============================ score CTA ============================
-    if (warp == 0 && lane == 0) {
-      // ---- key-tile producer
+  // Register split: the launch gives every thread kLaunchRegs (checked on the host before launch);
+  // warpgroup 0 (producer, MMA issuer, relay) gives registers up to warpgroups 1-2 (softmax /
+  // epilogue).  128 * kLowRegs + 256 * kHighRegs == 384 * kLaunchRegs.
+  // Register split (warpgroup-uniform): the launch gives every thread kLaunchRegs (checked on the
+  // host); warpgroup 0 (producers, MMA issuers, relay) hands registers to warpgroups 1-2 (softmax
+  // and epilogue warps).  128 * kLowRegs + 256 * kHighRegs == 384 * kLaunchRegs.
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+    if (rank == 0) {
+      if (warp == 0 && lane == 0) {
+      // ---- key producer: a score tile is up to 4 pages (256 keys); it is streamed as 9 stages of
+      // [256 keys x 64 dims] (8 latent chunks, then the RoPE key), one TMA box per page.
       SegIter it = it0;
       uint32_t n = 0;
-      uint32_t uses[kKStages] = {0, 0, 0};
+      uint32_t uses[kKStages] = {0, 0, 0, 0, 0, 0};
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        for (int t = t0; t < t1; ++t, ++n) {
-          sb.prog[warp] = (int)n;
-          const int s = n % kKStages;
-          if (n >= kKStages && !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done0;
-          int64_t row = tile_row(p, b, t);
-          if (row < 0) {
-            report(p.dev_status, MLA_ERR_BAD_INDEX);
-            row = 0;
+        for (int T = t0; T < t1; T += kSuper) {
+          const int npg = min(kSuper, t1 - T);
+          int32_t rows[kSuper];
+#pragma unroll
+          for (int pg = 0; pg < kSuper; ++pg) {
+            int64_t row = pg < npg ? tile_row(p, b, T + pg) : 0;
+            if (row < 0) {
+              report(p.dev_status, MLA_ERR_BAD_INDEX);
+              row = 0;
+            }
+            rows[pg] = (int32_t)row;
           }
-          const uint32_t dst = smem_u32(tiles + s * kKTileBytes);
-          mbar_expect_tx(bar(B_KFULL + s), kKTileBytes);
-          for (int j = 0; j < 8; ++j) tma_load_2d(dst + j * kChunkBytes, &map_c, 64 * j, (int32_t)row, bar(B_KFULL + s));
-          tma_load_2d(dst + 8 * kChunkBytes, &map_pe, 0, (int32_t)row, bar(B_KFULL + s));
-          ++uses[s];
+          for (int j = 0; j < 9; ++j, ++n) {
+            sb.prog[warp] = (int)n;
+            const int s = n % kKStages;
+            if (n >= kKStages && !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done0;
+            const uint32_t dst = smem_u32(tiles + kKOff + s * kKStageBytes);
+            mbar_expect_tx(bar(B_KFULL + s), npg * kChunkBytes);
+            for (int pg = 0; pg < npg; ++pg) {
+              if (j < 8) tma_load_2d(dst + pg * kChunkBytes, &map_c, 64 * j, rows[pg], bar(B_KFULL + s));
+              else tma_load_2d(dst + pg * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
+            }
+            ++uses[s];
+          }
         }
       }
     prod_done0:
       // Drain: the last load issued on each stage must have landed before exit.
       for (int s = 0; s < kKStages; ++s)
         if (uses[s]) mbar_wait(bar(B_KFULL + s), (uses[s] - 1) & 1, kWaitNs);
-    } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: S = Q . K^T
+      } else if (warp == 1 && lane == 0) {
+      // ---- MMA issuer: S [128 x N] = Q . K^T, N = 64 * pages (256 for a full score tile).
+      // The latent part of Q is the A operand from tensor memory; the RoPE part is in shared memory.
       SegIter it = it0;
       uint32_t n = 0, ns = 0, uc = 0;
-      const uint32_t idesc = idesc_bf16_f32(kRows, kTileKeys, false, false);
-      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+      bool ok = true;
+      while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         if (!wait_or_abort(sb, bar(B_QREADY), uc & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
         tc_fence_after();
-        bool ok = true;
-        for (int t = t0; t < t1; ++t, ++n, ++ns) {
-          sb.prog[warp] = (int)n;
-          const int s = n % kKStages;
-          const int sbuf = ns & 1;
-          if (!wait_or_abort(sb, bar(B_KFULL + s), (n / kKStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-          if (ns >= 2 && !wait_or_abort(sb, bar(B_SEMPTY + sbuf), ((ns >> 1) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+        for (int T = t0; T < t1; T += kSuper, ++ns) {
+          const int npg = min(kSuper, t1 - T);
+          const uint32_t idesc = idesc_bf16_f32(kRows, kTileKeys * npg, false, false);
+          if (ns > 0 && !wait_or_abort(sb, bar(B_SEMPTY), (ns - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t kt = smem_u32(tiles + s * kKTileBytes);
-          const uint32_t d = tbase + kSCol + 64 * sbuf;
-#pragma unroll 4
-          for (int k = 0; k < kW / 16; ++k) {
-            const uint64_t bd = smem_desc_sw128(kt + (k >> 2) * kChunkBytes + (k & 3) * 32, 16, 1024);
-            mma_ts(d, tbase + kQCol + 8 * k, bd, idesc, k > 0);
-          }
-          tc_commit(bar(B_SFULL + sbuf));
-          tc_commit(bar(B_KEMPTY + s));
-        }
-        if (!ok) break;
-        ++uc;
-      }
-    } else if (warp >= 4) {
-      // ---- softmax: thread = one query row (TMEM lane)
-      const int r = (warp - 4) * 32 + lane;
-      const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-      SegIter it = it0;
-      uint32_t ns = 0, np = 0, uc = 0;
-      const uint32_t pbuf_local = smem_u32(tiles + kPOff);
-      const uint32_t pbuf_remote = mapa(pbuf_local, peer);
-      const uint32_t alpha_remote = mapa(smem_u32(&sb.alpha[0][0]), peer);
-      const uint32_t statl_remote = mapa(smem_u32(&sb.stat_l[0]), peer);
-      const uint32_t statm_remote = mapa(smem_u32(&sb.stat_m[0]), peer);
-      const uint32_t pfull_remote = mapa(bar(B_PFULL), peer);
-      const uint32_t statsfull_remote = mapa(bar(B_STATSFULL), peer);
-      const int nrows = p.n_q * p.H;
-      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        // Q row -> tensor memory (the previous unit's MMAs are complete: its last S was consumed).
-        const int gr = rb * kRows + r;
-        const bool real = gr < nrows;
-        {
-          const uint4 *src = reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * nrows + (real ? gr : 0)) * kW);
-#pragma unroll 1
-          for (int c = 0; c < 9; ++c) {
-            uint32_t v[32];
+          for (int j = 0; j < 9; ++j, ++n) {
+            sb.prog[warp] = (int)n;
+            const int s = n % kKStages;
+            if (!wait_or_abort(sb, bar(B_KFULL + s), (n / kKStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t kt = smem_u32(tiles + kKOff + s * kKStageBytes);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              uint4 x = real ? __ldg(src + c * 8 + i) : make_uint4(0, 0, 0, 0);
-              v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = smem_desc_sw128(kt + kk * 32, 16, 1024);
+              if (j < 8)
+                mma_ts(tbase + kSCol, tbase + kQCol + 32 * j + 8 * kk, bd, idesc, (j | kk) ? 1u : 0u);
+              else
+                mma_ss(tbase + kSCol, smem_desc_sw128(smem_u32(tiles + kQpeOff) + kk * 32, 16, 1024), bd, idesc, 1u);
             }
-            tmem_st32(tbase + lane_off + kQCol + 32 * c, v);
+            tc_commit(bar(B_KEMPTY + s));
           }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_QREADY));
+          if (!ok) break;
+          tc_commit(bar(B_SFULL));
         }
-        const int S = seq_len_clamped(p, b);
-        const int j = real ? gr / p.H : 0;
-        const int visible = real ? S - p.n_q + j + 1 : 0;
-        float m_ref = -CUDART_INF_F, l = 0.f;
-        bool ok = true;
-        for (int t = t0; t < t1; ++t, ++ns, ++np) {
-          if (lane == 0) sb.prog[warp] = (int)np;
-          const int sbuf = ns & 1;
-          if (!warp_wait(sb, bar(B_SFULL + sbuf), (ns >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-          tc_fence_after();
-          uint32_t sraw[64];
-          {
-            uint32_t a[32], c2[32];
-            tmem_ld32(tbase + lane_off + kSCol + 64 * sbuf, a);
-            tmem_ld32(tbase + lane_off + kSCol + 64 * sbuf + 32, c2);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) { sraw[i] = a[i]; sraw[32 + i] = c2[i]; }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
-          const int nvalid = visible - t * kTileKeys;     // keys k < nvalid are visible
-          float mx = -CUDART_INF_F;
-#pragma unroll
-          for (int k = 0; k < 64; ++k)
-            if (k < nvalid) mx = fmaxf(mx, __uint_as_float(sraw[k]) * p.scale_log2);
-          float alpha = 1.f;
-          const bool need = mx > m_ref + kRescaleLog2;
-          if (need) {
-            alpha = exp2f(m_ref - mx);
-            l *= alpha;
-            m_ref = mx;
-          }
-          uint32_t pk[32];
-          float psum = 0.f;
-#pragma unroll
-          for (int k = 0; k < 64; k += 2) {
-            float p0 = (k < nvalid) ? exp2f(__uint_as_float(sraw[k]) * p.scale_log2 - m_ref) : 0.f;
-            float p1 = (k + 1 < nvalid) ? exp2f(__uint_as_float(sraw[k + 1]) * p.scale_log2 - m_ref) : 0.f;
-            const uint32_t pr = pack_bf16x2(p0, p1);
-            pk[k >> 1] = pr;
-            psum += __uint_as_float(pr << 16) + __uint_as_float(pr & 0xffff0000u);
-          }
-          l += psum;
-          const int pb = np & 1;
-          if (np >= 2 && !warp_wait(sb, bar(B_PEMPTY + pb), ((np >> 1) - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) { ok = false; break; }
-          // P row r -> value CTA, K-major 128B-swizzled [128 rows x 64 keys] tile.
-          const uint32_t rowbase = pbuf_remote + pb * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_cluster_v4(rowbase + ((c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-          st_cluster_f32(alpha_remote + (pb * kRows + r) * 4, alpha);
-          fence_proxy_async_cluster();
-          mbar_arrive_cluster(pfull_remote + 8 * pb);
-        }
-        if (!ok) break;
-        // Unit statistics -> value CTA.
-        if (uc > 0 && !warp_wait(sb, bar(B_STATSEMPTY), (uc - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) break;
-        st_cluster_f32(statl_remote + r * 4, l);
-        st_cluster_f32(statm_remote + r * 4, m_ref);
-        mbar_arrive_cluster(statsfull_remote);
         ++uc;
       }
-    }
-  } else {
-    // ============================ value CTA ============================
-    if (warp == 0 && lane == 0) {
+      }
+    } else {
+      if (warp == 0 && lane == 0) {
       // ---- latent-tile producer (c_KV part only)
       if (cid == 0) {
         // Units with no tiles get an empty segment list (their rows combine to zero).
@@ -523,23 +461,36 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
     prod_done1:
       for (int s = 0; s < kVStages; ++s)
         if (uses[s]) mbar_wait(bar(B_VFULL + s), (uses[s] - 1) & 1, kWaitNs);
-    } else if (warp == 1 && lane == 0) {
+      } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer: O += P . C
       SegIter it = it0;
-      uint32_t n = 0, np = 0, uc = 0;
+      uint32_t n = 0, np = 0, uc = 0, nfix = 0;
       const uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
-      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+      bool ok = true;
+      while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         if (uc > 0 && !wait_or_abort(sb, bar(B_OFREE), (uc - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
-        bool ok = true;
+        const int S = seq_len_clamped(p, b);
         for (int t = t0; t < t1; ++t, ++n, ++np) {
-          if (lane == 0) sb.prog[warp] = (int)n;
-          const int s = n % kVStages, pb = np & 1;
-          if (!wait_or_abort(sb, bar(B_VFULL + s), (n / kVStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-          if (!wait_or_abort(sb, bar(B_PFULL + pb), (np >> 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) { ok = false; break; }
-          // The epilogue warps have zeroed tail rows and rescaled O for this tile.
-          // Two slots: the epilogue warps may run up to two tiles ahead of this thread, and one
-          // barrier would then complete two phases before it is observed.
-          if (!wait_or_abort(sb, bar(B_CORR + (n & 1)), (n >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          sb.prog[warp] = (int)n;
+          const int s = n % kVStages, pb = np % kPSlots;
+          if (!wait_or_abort(sb, bar(B_VFULL + s), (n / kVStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__) ||
+              !wait_or_abort(sb, bar(B_PFULL + pb), (np / kPSlots) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
+            ok = false;
+            break;
+          }
+          const bool tail = (t + 1) * kTileKeys > S;
+          const uint32_t *fl = sb.flags[pb];
+          const bool resc = t != t0 && (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
+          if (tail || resc) {
+            // Rare: let the epilogue warps zero the rows past the end and/or rescale O first.
+            // A rescale reads O back, so every earlier MMA must have completed.
+            if (resc && !wait_or_abort(sb, bar(B_PVDONE + (np - 1) % kPSlots), ((np - 1) / kPSlots) & 1, p.dev_status,
+                                       false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            sb.req = Req{0, s, pb, S - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
+            mbar_arrive(bar(B_REQ));
+            if (!wait_or_abort(sb, bar(B_REQDONE), nfix & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            ++nfix;
+          }
           tc_fence_after();
           fence_proxy_async_smem();
           const uint32_t vt = smem_u32(tiles + s * kVTileBytes);
@@ -556,97 +507,243 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           tc_commit(bar(B_VEMPTY + s));
         }
         if (!ok) break;
+        // Unit epilogue request: the epilogue warps wait for the last MMAs themselves.
+        const uint32_t last = np - 1;
+        sb.req = Req{1, 0, 0, 0, 0, 0, segid, (int)(last % kPSlots), (int)((last / kPSlots) & 1)};
+        mbar_arrive(bar(B_REQ));
         ++uc;
       }
-    } else if (warp == 2 && lane == 0) {
-      // ---- relay: a P buffer is free once the MMAs that read it completed
+      } else if (warp == 2 && lane == 0) {
+      // ---- relay: a P slot is free once the MMAs that read it completed
+      // Each slot's P-full phase is armed with the bytes the score CTA will send
+      // before that CTA may send them (initially, then when the slot frees up).
       SegIter it = it0;
       uint32_t np = 0;
       const uint32_t pempty_remote = mapa(bar(B_PEMPTY), peer);
-      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        bool ok = true;
+      bool ok = true;
+      while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         for (int t = t0; t < t1; ++t, ++np) {
           sb.prog[warp] = (int)np;
-          const int pb = np & 1;
-          if (!wait_or_abort(sb, bar(B_PVDONE + pb), (np >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          const int pb = np % kPSlots;
+          if (!wait_or_abort(sb, bar(B_PVDONE + pb), (np / kPSlots) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bar(B_PFULL + pb), kPTxBytes);
           mbar_arrive_cluster(pempty_remote + 8 * pb);
         }
-        if (!ok) break;
       }
-    } else if (warp >= 4) {
-      // ---- tail zeroing, O rescaling and the unit epilogue
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
+    if (rank == 0) {
+      // ---- softmax: 8 warps; warp (quadrant q, half h) owns rows 32q..32q+31 (its TMEM lanes)
+      // and the score columns 128h..128h+127 of each score tile.
+      const int q4 = warp & 3, h = (warp - 4) >> 2;
+      const int r = q4 * 32 + lane;
+      const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+      SegIter it = it0;
+      uint32_t ns = 0, np = 0, uc = 0;
+      const uint32_t pbuf_remote = mapa(smem_u32(tiles + kPOff), peer);
+      const uint32_t alpha_remote = mapa(smem_u32(&sb.alpha[0][0]), peer);
+      const uint32_t flags_remote = mapa(smem_u32(&sb.flags[0][0]), peer);
+      const uint32_t statl_remote = mapa(smem_u32(&sb.stat_l[0]), peer);
+      const uint32_t statm_remote = mapa(smem_u32(&sb.stat_m[0]), peer);
+      const uint32_t pfull_remote = mapa(bar(B_PFULL), peer);
+      const uint32_t statsfull_remote = mapa(bar(B_STATSFULL), peer);
+      const int nrows = p.n_q * p.H;
+      // No early exit in this region: the eight warps meet at named barriers, so on a timeout they
+      // keep walking the same (now wait-free: every wait returns at once) loop to the end.
+      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        // Q row -> half h loads latent dims 256h..256h+255 into TMEM columns 128h..; half 0 also
+        // puts the RoPE dims into the shared [128 x 64] A tile.  The previous unit's MMAs are
+        // complete (its last S was consumed), so both may be overwritten.
+        const int gr = rb * kRows + r;
+        const bool real = gr < nrows;
+        {
+          const uint4 *src = reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * nrows + (real ? gr : 0)) * kW);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              uint4 x = real ? __ldg(src + h * 32 + c * 8 + i) : make_uint4(0, 0, 0, 0);
+              v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+            }
+            tmem_st32(tbase + lane_off + kQCol + 128 * h + 32 * c, v);
+          }
+          if (h == 0) {
+            unsigned char *qpe = tiles + kQpeOff + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4 *>(qpe + ((c ^ (r & 7)) << 4)) = real ? __ldg(src + 64 + c) : make_uint4(0, 0, 0, 0);
+            fence_proxy_async_smem();
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_QREADY));
+        }
+        const int S = seq_len_clamped(p, b);
+        const int j = real ? gr / p.H : 0;
+        const int visible = real ? S - p.n_q + j + 1 : 0;
+        float m_ref = -CUDART_INF_F, l = 0.f;
+        for (int T = t0; T < t1; T += kSuper, ++ns) {
+          if (lane == 0) sb.prog[warp] = (int)np;
+          const int npg = min(kSuper, t1 - T);
+          warp_wait(sb, bar(B_SFULL), ns & 1, p.dev_status, false, p.timeout_rec, __LINE__);
+          tc_fence_after();
+          uint32_t sc[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tbase + lane_off + kSCol + 128 * h + 32 * c, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sc[32 * c + i] = v[i];
+          }
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(B_SEMPTY));
+          // Keys of my columns: 64T + 128h + k; valid while below the row's causal limit and
+          // inside the pages this score tile holds.
+          const int nvalid = min(visible - (T * kTileKeys + 128 * h), npg * kTileKeys - 128 * h);
+          float mx = -CUDART_INF_F;
+#pragma unroll
+          for (int k = 0; k < 128; ++k)
+            if (k < nvalid) mx = fmaxf(mx, __uint_as_float(sc[k]) * p.scale_log2);
+          sb.xmax[ns & 1][h][r] = mx;
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          mx = fmaxf(mx, sb.xmax[ns & 1][h ^ 1][r]);
+          float alpha = 1.f;
+          const bool need = mx > m_ref + kRescaleLog2;
+          if (need) {
+            alpha = exp2f(m_ref - mx);
+            l *= alpha;
+            m_ref = mx;
+          }
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int g = 2 * h + i;              // page of this score tile
+            if (g >= npg) break;
+            const uint32_t pn = np + g;
+            const int pb = pn % kPSlots;
+            if (pn >= kPSlots) warp_wait(sb, bar(B_PEMPTY + pb), ((pn / kPSlots) - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__);
+            // P rows -> value CTA, K-major 128B-swizzled [128 rows x 64 keys] tile, by asynchronous
+            // remote stores that complete on the value CTA's P-full barrier (armed by its relay),
+            // 8 keys (16 bytes) at a time.  The first page of a score tile also carries the tile's
+            // O rescale factors.
+            const uint32_t pfull = pfull_remote + 8 * pb;
+            const uint32_t rowbase = pbuf_remote + pb * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+            float psum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int kk = 64 * i + 8 * c + 2 * e;
+                const float p0 = (kk < nvalid) ? exp2f(__uint_as_float(sc[kk]) * p.scale_log2 - m_ref) : 0.f;
+                const float p1 = (kk + 1 < nvalid) ? exp2f(__uint_as_float(sc[kk + 1]) * p.scale_log2 - m_ref) : 0.f;
+                pk[e] = pack_bf16x2(p0, p1);
+                psum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+              }
+              st_async_v4(rowbase + ((c ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3], pfull);
+            }
+            l += psum;
+            st_async_b32(alpha_remote + (pb * kRows + r) * 4, __float_as_uint(g == 0 ? alpha : 1.f), pfull);
+            const unsigned moved = __ballot_sync(0xffffffffu, need && g == 0 && T != t0);
+            if (lane == 0) st_async_b32(flags_remote + (pb * 4 + q4) * 4, moved ? 1u : 0u, pfull);
+          }
+          np += npg;
+        }
+        // Unit statistics: combine the halves' row sums, then send them to the value CTA.
+        sb.xl[h][r] = l;
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        if (h == 0) {
+          l += sb.xl[1][r];
+          if (uc > 0) warp_wait(sb, bar(B_STATSEMPTY), (uc - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__);
+          st_cluster_f32(statl_remote + r * 4, l);
+          st_cluster_f32(statm_remote + r * 4, m_ref);
+          mbar_arrive_cluster(statsfull_remote);
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // xl may be reused by the next unit
+        ++uc;
+      }
+    } else if (warp < 8) {
+      // ---- epilogue warps: tile fix-ups on request, then each unit's epilogue
       const int r = (warp - 4) * 32 + lane;
       const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
       SegIter it = it0;
-      uint32_t n = 0, np = 0, uc = 0;
+      uint32_t nreq = 0, uc = 0;
       const uint32_t statsempty_remote = mapa(bar(B_STATSEMPTY), peer);
-      while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        const int S = seq_len_clamped(p, b);
-        bool ok = true;
-        for (int t = t0; t < t1; ++t, ++n, ++np) {
-          if (lane == 0) sb.prog[warp] = (int)n;
-          const int s = n % kVStages, pb = np & 1;
-          if (!warp_wait(sb, bar(B_PFULL + pb), (np >> 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) { ok = false; break; }
-          if ((t + 1) * kTileKeys > S) {
-            // Rows past the sequence end may hold anything (NaN): zero them so 0 * row stays 0.
-            if (!warp_wait(sb, bar(B_VFULL + s), (n / kVStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            const int nv = S - t * kTileKeys;
-            unsigned char *vt = tiles + s * kVTileBytes;
-            const int nrow = kTileKeys - nv;
-            for (int e = threadIdx.x - 128; e < nrow * 8 * 8; e += 128) {
-              const int row = nv + e / 64, rest = e % 64, ch = rest / 8, piece = rest % 8;
-              *reinterpret_cast<uint4 *>(vt + ch * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+      bool ok = true;
+      while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        for (;;) {
+          if (lane == 0) sb.prog[warp] = (int)nreq;
+          if (!warp_wait(sb, bar(B_REQ), nreq & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          ++nreq;
+          const Req q = sb.req;
+          if (q.kind == 0) {
+            if (q.tail) {
+              // Rows past the sequence end may hold anything (NaN): zero them so 0 * row stays 0.
+              unsigned char *vt = tiles + q.vstage * kVTileBytes;
+              const int nrow = kTileKeys - q.nvalid;
+              for (int e = threadIdx.x - 128; e < nrow * 64; e += 128) {
+                const int row = q.nvalid + e / 64, rest = e % 64, ch = rest / 8, piece = rest % 8;
+                *reinterpret_cast<uint4 *>(vt + ch * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+              }
+              fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
-          }
-          // Rescale O where this tile moved a row's reference maximum (warp-uniform: tcgen05.ld/st
-          // are warp-collective; rows that did not move carry alpha = 1).
-          const float a = sb.alpha[pb][r];
-          if (__any_sync(0xffffffffu, a != 1.f && t != t0)) {
-            // All earlier PV MMAs must be complete before O is read back.
-            if (!warp_wait(sb, bar(B_PVDONE + ((np - 1) & 1)), ((np - 1) >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            tc_fence_after();
+            if (q.rescale) {
+              tc_fence_after();
+              const float a = sb.alpha[q.slot][r];
 #pragma unroll 1
-            for (int c = 0; c < 16; ++c) {
-              uint32_t v[32];
-              tmem_ld32(tbase + lane_off + 32 * c, v);
-              tmem_wait_ld();
+              for (int c = 0; c < 16; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tbase + lane_off + 32 * c, v);
+                tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-              tmem_st32(tbase + lane_off + 32 * c, v);
+                for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+                tmem_st32(tbase + lane_off + 32 * c, v);
+              }
+              tmem_wait_st();
+              tc_fence_before();
             }
-            tmem_wait_st();
+            mbar_arrive(bar(B_REQDONE));
+            continue;
           }
+          // Unit epilogue: the unit's last MMAs and the row statistics.
+          if (!warp_wait(sb, bar(B_PVDONE + q.last_slot), q.last_parity, p.dev_status, false, p.timeout_rec, __LINE__) ||
+              !warp_wait(sb, bar(B_STATSFULL), uc & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float l = sb.stat_l[r], m = sb.stat_m[r];
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(statsempty_remote);
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          __nv_bfloat16 *dst = p.o_part + ((int64_t)q.segid * kRows + r) * kDc;
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tbase + lane_off + 32 * c, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+              *reinterpret_cast<uint4 *>(dst + 32 * c + i) =
+                  make_uint4(pack_bf16x2(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
+                             pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
+                             pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
+                             pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
+          }
+          p.lse_part[(int64_t)q.segid * kRows + r] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
           tc_fence_before();
-          mbar_arrive(bar(B_CORR + (n & 1)));
+          mbar_arrive(bar(B_OFREE));
+          ++uc;
+          break;
         }
-        if (!ok) break;
-        // Epilogue: wait for the unit's last MMAs and the row statistics.
-        if (!warp_wait(sb, bar(B_PVDONE + ((np - 1) & 1)), ((np - 1) >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
-        if (!warp_wait(sb, bar(B_STATSFULL), uc & 1, p.dev_status, true, p.timeout_rec, __LINE__)) break;
-        tc_fence_after();
-        const float l = sb.stat_l[r], m = sb.stat_m[r];
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(statsempty_remote);
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16 *dst = p.o_part + ((int64_t)segid * kRows + r) * kDc;
-#pragma unroll 1
-        for (int c = 0; c < 16; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tbase + lane_off + 32 * c, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; i += 8)
-            *reinterpret_cast<uint4 *>(dst + 32 * c + i) =
-                make_uint4(pack_bf16x2(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
-                           pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
-                           pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
-                           pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
-        }
-        p.lse_part[(int64_t)segid * kRows + r] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
-        tc_fence_before();
-        mbar_arrive(bar(B_OFREE));
-        ++uc;
       }
     }
   }
@@ -806,6 +903,9 @@ int clusters_for_device() {
   if (cached[dev]) return cached[dev];
   if (cudaFuncSetAttribute(mla_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes))
     return 0;
+  // The in-kernel register split assumes exactly kLaunchRegs per thread; never launch otherwise.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, mla_decode_tc_kernel) != cudaSuccess || fa.numRegs != kLaunchRegs) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * kMaxClusters);
   cfg.blockDim = dim3(kThreads);
