@@ -199,15 +199,23 @@ def run_mla(args):
     case = DECODE_CASES[args.config]
     d = case.dims
     inp = make_decode_step_inputs(case)
+    # bf16 pools with 64-token pages use the tiled page layout (pages move by contiguous bulk copies);
+    # the seeded row pool is packed into it once, before anything is timed.
+    tiled = d.dtype == "bf16" and case.block_size % 64 == 0 and (d.d_c + d.d_rope) % 64 == 0
     dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
-                         rope_base=d.rope_base, rms_eps=d.rms_eps)
+                         rope_base=d.rope_base, rms_eps=d.rms_eps, cache_layout=1 if tiled else 0)
     dev = {k: inp[k].cuda() for k in ("pool", "block_table", "seqlens", "q_nope", "q_pe", "w_uk", "w_uv", "h_new",
                                       "w_dkv", "w_kr", "gamma", "seq_idx", "pos")}
+    if tiled:
+        packed = torch.empty_like(dev["pool"])
+        mla.mla_cache_pack(dims, dev["pool"], packed)
+        torch.cuda.synchronize()
+        dev["pool"] = packed
     B, n_q, H = case.batch, case.n_q, d.n_heads
     max_seqlen = int(inp["seqlens"].max())
     T = B * n_q
     pool = dev["pool"]
-    c_kv, k_pe = pool, pool[:, d.d_c:]
+    c_kv, k_pe = (pool, pool) if tiled else (pool, pool[:, d.d_c:])
     bt = dev["block_table"] if case.paged else None
     ws = mla.alloc_workspace(mla.mla_decode_workspace_size(dims, B, n_q, max_seqlen))
     q_abs = torch.empty((B, n_q, H, d.d_c + d.d_rope), dtype=d.torch_dtype, device="cuda")
@@ -216,9 +224,13 @@ def run_mla(args):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
 
+    app_ws_bytes = mla.mla_append_workspace_size(dims, T)
+    app_ws = mla.alloc_workspace(app_ws_bytes) if app_ws_bytes else None
+
     def append():
         mla.mla_append_latent(dims, dev["h_new"], dev["w_dkv"], dev["w_kr"], dev["gamma"], dev["seq_idx"],
-                              dev["pos"], c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status)
+                              dev["pos"], c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status,
+                              workspace=app_ws)
 
     def step(ev=None):
         append()

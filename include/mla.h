@@ -35,10 +35,21 @@
  *  with blk = block_table[b * max_blocks_per_seq + i / block_size]
  *  (block_table == NULL means the identity table: blk = b * max_blocks_per_seq
  *  + i / block_size, i.e. each sequence owns a contiguous run of rows).
- *  c_KV of row r is at c_kv + r * ckv_stride (d_c elements), the rotated RoPE
- *  key at k_pe + r * kpe_stride (d_R elements).  The fused layout used by the
- *  fast decode kernel is one pool of rows of d_c + d_R elements with
- *  k_pe = c_kv + d_c and both strides = d_c + d_R.
+ *  Two pool layouts (mla_dims.cache_layout):
+ *  - MLA_CACHE_ROWS: c_KV of row r is at c_kv + r * ckv_stride (d_c elements),
+ *    the rotated RoPE key at k_pe + r * kpe_stride (d_R elements).  One pool of
+ *    rows of d_c + d_R elements has k_pe = c_kv + d_c and both strides d_c + d_R.
+ *  - MLA_CACHE_TILED: one pool at c_kv (k_pe and the strides are ignored), in
+ *    pages of 64 tokens; block_size must be a multiple of 64 and block blk
+ *    holds pages blk*block_size/64 .. +block_size/64-1, i.e. row r lies in page
+ *    r / 64 as token t = r % 64.  A page is W/64 chunks (W = d_c + d_R, a
+ *    multiple of 64) of 8 KB; chunk c holds dims 64c .. 64c+63 of its 64 tokens,
+ *    token t at byte 128 t of the chunk, and its 16-byte group g (dims 8g ..
+ *    8g+7 of the chunk) at byte 16 * (g XOR (t mod 8)) of that 128-byte line.
+ *    c_KV dims come first, then the RoPE key.  This is the order in which the
+ *    tensor cores read a page (128-byte swizzled, K-major), so a page moves
+ *    with plain contiguous bulk copies.  bf16 only.  mla_cache_pack /
+ *    mla_cache_unpack convert between a row pool and this layout.
  *
  * Positions and RoPE
  *  Positions are 0-based.  Pair (2i, 2i+1) of a RoPE vector at position p is
@@ -79,6 +90,8 @@ typedef enum {
 
 typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
 
+typedef enum { MLA_CACHE_ROWS = 0, MLA_CACHE_TILED = 1 } mla_cache_layout;
+
 typedef struct {
   int n_heads;        /* H: query heads */
   int d_c;            /* latent width (c_KV) */
@@ -93,6 +106,7 @@ typedef struct {
   float softmax_scale;/* <= 0 selects 1/sqrt(d_nope + d_rope) */
   float rms_eps;      /* epsilon of the RMSNorm on c_KV, e.g. 1e-6 */
   int dtype;          /* mla_dtype of every float tensor */
+  int cache_layout;   /* mla_cache_layout of the latent pool */
 } mla_dims;
 
 /*
@@ -112,8 +126,18 @@ typedef struct {
 MLA_API int mla_append_latent(const mla_dims *dims, int T, const void *h, const void *w_dkv,
                       const void *w_kr, const void *rms_gamma, const int32_t *seq_idx,
                       const int32_t *pos, void *c_kv, void *k_pe, const int32_t *block_table,
-                      int num_seqs, int max_blocks_per_seq, int num_blocks, int *dev_status,
-                      mla_stream_t stream);
+                      int num_seqs, int max_blocks_per_seq, int num_blocks, void *workspace,
+                      size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
+ * mla_append_workspace_size — scratch bytes that let mla_append_latent run
+ *   the down-projection on tensor cores, split over d_model (bf16 shapes with
+ *   d_model a multiple of 64, d_c a multiple of 64, d_R <= 64).  0 when the
+ *   shape has no such path.  mla_append_latent with workspace == NULL (or a
+ *   smaller one) runs the CUDA-core path instead; both give the same rows up
+ *   to the order of fp32 additions.
+ */
+MLA_API int mla_append_workspace_size(const mla_dims *dims, int T, size_t *bytes);
 
 /*
  * mla_absorb_q — the decode query in latent space.
@@ -246,6 +270,19 @@ MLA_API int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, 
  *   profilers and benchmarks.  Writes *count; no device work.
  */
 MLA_API int mla_decode_launches(const mla_dims *dims, int n_q, int *count);
+
+/*
+ * mla_cache_pack / mla_cache_unpack — convert a latent pool between the row
+ *   layout and the tiled page layout (see "Paged latent cache" above).
+ *   rows: [num_rows, d_c + d_R] bf16, row-major (c_KV then the RoPE key);
+ *   tiled: num_rows / 64 pages.  num_rows must be a multiple of 64; dims->dtype
+ *   must be MLA_BF16 and d_c + d_R a multiple of 64.  The two buffers must not
+ *   overlap.  Pure data movement: unpack(pack(x)) == x bit for bit.
+ */
+MLA_API int mla_cache_pack(const mla_dims *dims, const void *rows, void *tiled, int64_t num_rows,
+                           mla_stream_t stream);
+MLA_API int mla_cache_unpack(const mla_dims *dims, const void *tiled, void *rows, int64_t num_rows,
+                             mla_stream_t stream);
 
 /* Human-readable text of an mla_status value (static storage). */
 MLA_API const char *mla_status_string(int status);

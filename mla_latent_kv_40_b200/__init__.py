@@ -20,6 +20,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 MLA_F32, MLA_BF16 = 0, 1
+MLA_CACHE_ROWS, MLA_CACHE_TILED = 0, 1
 STATUS = {0: "MLA_OK", -1: "MLA_ERR_INVALID_ARG", -2: "MLA_ERR_UNSUPPORTED", -3: "MLA_ERR_WORKSPACE",
           -4: "MLA_ERR_CUDA", -5: "MLA_ERR_TIMEOUT", -6: "MLA_ERR_BAD_INDEX", -7: "MLA_ERR_STATIC_WS"}
 NOALLOC_SCRATCH_BYTES = 16 << 20   # MLA_NOALLOC_SCRATCH_BYTES in include/mla.h
@@ -36,17 +37,17 @@ class mla_dims(ctypes.Structure):
                 ("d_nope", ctypes.c_int), ("d_v", ctypes.c_int), ("d_model", ctypes.c_int),
                 ("block_size", ctypes.c_int), ("ckv_stride", ctypes.c_int), ("kpe_stride", ctypes.c_int),
                 ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("cache_layout", ctypes.c_int)]
 
 
 def make_dims(n_heads, d_c, d_rope, d_nope, d_v, d_model, block_size, dtype, ckv_stride=None,
-              kpe_stride=None, rope_base=10000.0, softmax_scale=0.0, rms_eps=1e-6) -> mla_dims:
-    """Dims of a fused cache pool by default: rows of d_c + d_rope elements."""
+              kpe_stride=None, rope_base=10000.0, softmax_scale=0.0, rms_eps=1e-6, cache_layout=MLA_CACHE_ROWS) -> mla_dims:
+    """Dims of a fused row pool (rows of d_c + d_rope elements) by default, or of a tiled page pool."""
     w = d_c + d_rope
     dt = MLA_BF16 if dtype in ("bf16", torch.bfloat16, MLA_BF16) else MLA_F32
     return mla_dims(n_heads, d_c, d_rope, d_nope, d_v, d_model, block_size,
                     w if ckv_stride is None else ckv_stride, w if kpe_stride is None else kpe_stride,
-                    rope_base, softmax_scale, rms_eps, dt)
+                    rope_base, softmax_scale, rms_eps, dt, int(cache_layout))
 
 
 _P = ctypes.c_void_p
@@ -54,7 +55,8 @@ _I = ctypes.c_int
 _D = ctypes.POINTER(mla_dims)
 _SZ = ctypes.POINTER(ctypes.c_size_t)
 _sigs = {
-    "mla_append_latent": [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P],
+    "mla_append_latent": [_D, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, ctypes.c_size_t, _P, _P],
+    "mla_append_workspace_size": [_D, _I, _SZ],
     "mla_absorb_q": [_D, _I, _I, _P, _P, _P, _P, _P, _P],
     "mla_decode_workspace_size": [_D, _I, _I, _I, _SZ],
     "mla_decode": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
@@ -63,6 +65,8 @@ _sigs = {
     "mla_decode_combine": [_D, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_prefill_workspace_size": [_D, _I, _I, _I, _SZ],
     "mla_decode_launches": [_D, _I, ctypes.POINTER(ctypes.c_int)],
+    "mla_cache_pack": [_D, _P, _P, ctypes.c_int64, _P],
+    "mla_cache_unpack": [_D, _P, _P, ctypes.c_int64, _P],
     "mla_decode_noalloc": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P],
     "mla_prefill": [_D, _I, _P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
 }
@@ -111,20 +115,30 @@ def _check(fn, rc):
         raise MlaError(fn, rc)
 
 
+def mla_append_workspace_size(dims, T) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_append_workspace_size", _lib.mla_append_workspace_size(ctypes.byref(dims), int(T), ctypes.byref(n)))
+    return int(n.value)
+
+
 def mla_append_latent(dims, h, w_dkv, w_kr, rms_gamma, seq_idx, pos, c_kv, k_pe, block_table, num_seqs,
-                      max_blocks_per_seq, num_blocks, dev_status=None, stream=None):
+                      max_blocks_per_seq, num_blocks, dev_status=None, stream=None, workspace=None):
+    """workspace: None runs the CUDA-core path; a buffer of mla_append_workspace_size bytes
+    lets bf16 shapes run the tensor-core projection."""
     et = _elem_dtype(dims)
     T = 0 if h is None else h.shape[0]
     for n, t in (("h", h), ("w_dkv", w_dkv), ("w_kr", w_kr), ("rms_gamma", rms_gamma), ("seq_idx", seq_idx),
                  ("pos", pos), ("block_table", block_table)):
         _dense(t, n)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = _lib.mla_append_latent(ctypes.byref(dims), T, _ptr(h, et, "h"), _ptr(w_dkv, et, "w_dkv"),
                                 _ptr(w_kr, et, "w_kr"), _ptr(rms_gamma, et, "rms_gamma", True),
                                 _ptr(seq_idx, torch.int32, "seq_idx"), _ptr(pos, torch.int32, "pos"),
                                 _ptr(c_kv, et, "c_kv"), _ptr(k_pe, et, "k_pe"),
                                 _ptr(block_table, torch.int32, "block_table", True), int(num_seqs),
-                                int(max_blocks_per_seq), int(num_blocks),
-                                _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+                                int(max_blocks_per_seq), int(num_blocks), _ptr(workspace, None, "workspace", True),
+                                ctypes.c_size_t(ws_bytes), _ptr(dev_status, torch.int32, "dev_status", True),
+                                _stream(stream))
     _check("mla_append_latent", rc)
 
 
@@ -254,6 +268,22 @@ def mla_prefill(dims, cu_seqlens, max_seqlen, q_nope, q_pe, c_kv, k_pe, block_ta
                           ctypes.c_size_t(workspace.numel() * workspace.element_size()),
                           _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
     _check("mla_prefill", rc)
+
+
+def mla_cache_pack(dims, rows, tiled, stream=None):
+    """Row pool [num_rows, d_c + d_rope] (bf16) -> tiled page pool of the same byte size."""
+    _dense(rows, "rows")
+    _check("mla_cache_pack", _lib.mla_cache_pack(ctypes.byref(dims), _ptr(rows, torch.bfloat16, "rows"),
+                                                 _ptr(tiled, torch.bfloat16, "tiled"), int(rows.shape[0]),
+                                                 _stream(stream)))
+
+
+def mla_cache_unpack(dims, tiled, rows, stream=None):
+    """Tiled page pool -> row pool [num_rows, d_c + d_rope] (bf16)."""
+    _dense(rows, "rows")
+    _check("mla_cache_unpack", _lib.mla_cache_unpack(ctypes.byref(dims), _ptr(tiled, torch.bfloat16, "tiled"),
+                                                     _ptr(rows, torch.bfloat16, "rows"), int(rows.shape[0]),
+                                                     _stream(stream)))
 
 
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:

@@ -19,7 +19,14 @@ bool dims_ok(const mla_dims *d) {
   if (d->n_heads <= 0 || d->d_c <= 0 || d->d_rope < 0 || (d->d_rope & 1) || d->d_nope <= 0 ||
       d->d_v <= 0 || d->block_size <= 0)
     return false;
-  if (d->ckv_stride < d->d_c || d->kpe_stride < d->d_rope) return false;
+  if (d->cache_layout == MLA_CACHE_TILED) {
+    // Tiled pages: bf16, 64-token pages inside blocks, rows a whole number of 64-dim chunks.
+    if (d->dtype != MLA_BF16 || d->block_size % 64 != 0 || (d->d_c + d->d_rope) % 64 != 0) return false;
+  } else if (d->cache_layout == MLA_CACHE_ROWS) {
+    if (d->ckv_stride < d->d_c || d->kpe_stride < d->d_rope) return false;
+  } else {
+    return false;
+  }
   if (d->dtype != MLA_F32 && d->dtype != MLA_BF16) return false;
   if (!(d->rope_base > 0.f)) return false;
   return true;
@@ -62,7 +69,7 @@ int check_decode_args(const mla_dims *dims, int B, int n_q, const void *c_kv, co
   if (!dims_ok(dims)) return MLA_ERR_INVALID_ARG;
   if (B <= 0 || n_q <= 0 || max_seqlen < n_q || max_blocks_per_seq <= 0 || num_blocks <= 0)
     return MLA_ERR_INVALID_ARG;
-  if (!c_kv || (!k_pe && dims->d_rope) || !seqlens) return MLA_ERR_INVALID_ARG;
+  if (!c_kv || (!k_pe && dims->d_rope && dims->cache_layout == MLA_CACHE_ROWS) || !seqlens) return MLA_ERR_INVALID_ARG;
   if ((int64_t)max_blocks_per_seq * dims->block_size < max_seqlen) return MLA_ERR_INVALID_ARG;
   if (n_q * dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
@@ -78,7 +85,7 @@ int attention_impl(const mla_dims *dims, int B, int n_q, const void *q_abs, cons
                    int max_seqlen, const DecodeLayout &L, char *ws, int *dev_status, cudaStream_t st) {
   const bool bf16 = dims->dtype == MLA_BF16;
   CacheView cv{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq,
-               num_blocks, dims->block_size};
+               num_blocks, dims->block_size, dims->cache_layout, dims->d_c, dims->d_c + dims->d_rope};
   if (L.use_tc)
     return launch_tc_attention(*dims, B, n_q, q_abs, cv, seqlens, max_seqlen, ws + L.tc_off, dev_status, st);
   AttnArgs at{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, q_abs, cv, seqlens, default_scale(*dims),
@@ -111,7 +118,9 @@ int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const 
   void *qbuf = ws + L.q_off;
   AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
                 q_nope, q_pe, w_uk, seqlens, qbuf, dims->rope_base};
-  if ((rc = launch_absorb(ab, dims->dtype == MLA_BF16, st))) return rc;
+  if ((rc = absorb_mma_supported(ab, dims->dtype == MLA_BF16) ? launch_absorb_mma(ab, st)
+                                                               : launch_absorb(ab, dims->dtype == MLA_BF16, st)))
+    return rc;
   if ((rc = attention_impl(dims, B, n_q, qbuf, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
                            max_seqlen, L, ws, dev_status, st)))
     return rc;
@@ -136,20 +145,44 @@ const char *mla_status_string(int s) {
   }
 }
 
+static AppendArgs append_args(const mla_dims *dims, int T, const void *h, const void *w_dkv, const void *w_kr,
+                              const void *rms_gamma, const int32_t *seq_idx, const int32_t *pos, void *c_kv, void *k_pe,
+                              const int32_t *block_table, int num_seqs, int max_blocks_per_seq, int num_blocks,
+                              int *dev_status) {
+  return AppendArgs{T, dims->d_model, dims->d_c, dims->d_rope, h, w_dkv, w_kr, rms_gamma, seq_idx, pos,
+                    c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, num_seqs,
+                    max_blocks_per_seq, num_blocks, dims->block_size, dims->cache_layout, dims->rms_eps,
+                    dims->rope_base, dev_status};
+}
+
+int mla_append_workspace_size(const mla_dims *dims, int T, size_t *bytes) {
+  if (!dims_ok(dims) || dims->d_model <= 0 || T < 0 || !bytes) return MLA_ERR_INVALID_ARG;
+  AppendArgs a = append_args(dims, T, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                             nullptr, 1, 1, 1, nullptr);
+  *bytes = (T > 0 && append_mma_supported(a, dims->dtype == MLA_BF16))
+               ? append_mma_workspace(T, dims->d_model, dims->d_c + dims->d_rope, nullptr, nullptr)
+               : 0;
+  return MLA_OK;
+}
+
 int mla_append_latent(const mla_dims *dims, int T, const void *h, const void *w_dkv, const void *w_kr,
                       const void *rms_gamma, const int32_t *seq_idx, const int32_t *pos, void *c_kv,
                       void *k_pe, const int32_t *block_table, int num_seqs, int max_blocks_per_seq,
-                      int num_blocks, int *dev_status, mla_stream_t stream) {
+                      int num_blocks, void *workspace, size_t ws_bytes, int *dev_status, mla_stream_t stream) {
   if (!dims_ok(dims) || dims->d_model <= 0 || T < 0) return MLA_ERR_INVALID_ARG;
   if (T == 0) return MLA_OK;
-  if (!h || !w_dkv || (!w_kr && dims->d_rope) || !seq_idx || !pos || !c_kv || (!k_pe && dims->d_rope))
+  if (!h || !w_dkv || (!w_kr && dims->d_rope) || !seq_idx || !pos || !c_kv ||
+      (!k_pe && dims->d_rope && dims->cache_layout == MLA_CACHE_ROWS))
     return MLA_ERR_INVALID_ARG;
   if (num_seqs <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0) return MLA_ERR_INVALID_ARG;
-  AppendArgs a{T, dims->d_model, dims->d_c, dims->d_rope, h, w_dkv, w_kr, rms_gamma, seq_idx, pos,
-               c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, num_seqs,
-               max_blocks_per_seq, num_blocks, dims->block_size, dims->rms_eps, dims->rope_base,
-               dev_status};
-  return launch_append(a, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+  const AppendArgs a = append_args(dims, T, h, w_dkv, w_kr, rms_gamma, seq_idx, pos, c_kv, k_pe, block_table,
+                                   num_seqs, max_blocks_per_seq, num_blocks, dev_status);
+  const bool bf16 = dims->dtype == MLA_BF16;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (workspace && append_mma_supported(a, bf16) && !(reinterpret_cast<uintptr_t>(workspace) & 15) &&
+      ws_bytes >= append_mma_workspace(T, dims->d_model, dims->d_c + dims->d_rope, nullptr, nullptr))
+    return launch_append_mma(a, workspace, st);
+  return launch_append(a, bf16, st);
 }
 
 int mla_absorb_q(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
@@ -158,7 +191,9 @@ int mla_absorb_q(const mla_dims *dims, int B, int n_q, const void *q_nope, const
   if (!q_nope || (!q_pe && dims->d_rope) || !w_uk || !seqlens || !q_out) return MLA_ERR_INVALID_ARG;
   AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
                 q_nope, q_pe, w_uk, seqlens, q_out, dims->rope_base};
-  return launch_absorb(ab, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return absorb_mma_supported(ab, dims->dtype == MLA_BF16) ? launch_absorb_mma(ab, st)
+                                                           : launch_absorb(ab, dims->dtype == MLA_BF16, st);
 }
 
 int mla_decode_workspace_size(const mla_dims *dims, int B, int n_q, int max_seqlen, size_t *bytes) {
@@ -239,7 +274,8 @@ int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, int max_
   if (!dims_ok(dims) || B <= 0 || total_tokens <= 0 || max_seqlen <= 0 || max_blocks_per_seq <= 0 ||
       num_blocks <= 0)
     return MLA_ERR_INVALID_ARG;
-  if (!cu_seqlens || !q_nope || (!q_pe && dims->d_rope) || !c_kv || (!k_pe && dims->d_rope) || !w_uk ||
+  if (!cu_seqlens || !q_nope || (!q_pe && dims->d_rope) || !c_kv ||
+      (!k_pe && dims->d_rope && dims->cache_layout == MLA_CACHE_ROWS) || !w_uk ||
       !w_uv || !out)
     return MLA_ERR_INVALID_ARG;
   size_t need = 0;
@@ -254,9 +290,30 @@ int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, int max_
   PrefillArgs a{B, total_tokens, max_seqlen, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope, dims->d_v,
                 cu_seqlens, q_nope, q_pe, w_uk, w_uv,
                 CacheView{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq,
-                          num_blocks, dims->block_size},
+                          num_blocks, dims->block_size, dims->cache_layout, dims->d_c, dims->d_c + dims->d_rope},
                 qbuf, kbuf, vbuf, out, lse, default_scale(*dims), dims->rope_base, dev_status};
   return launch_prefill_simt(a, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+static int cache_convert(const mla_dims *dims, const void *src, void *dst, int64_t num_rows, bool to_tiled,
+                         mla_stream_t stream) {
+  if (!dims || dims->dtype != MLA_BF16 || dims->d_c <= 0 || dims->d_rope < 0 || (dims->d_c + dims->d_rope) % 64)
+    return MLA_ERR_INVALID_ARG;
+  if (!src || !dst || num_rows < 0 || num_rows % 64) return MLA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) return MLA_ERR_INVALID_ARG;
+  const int W = dims->d_c + dims->d_rope;
+  const uintptr_t bytes = (uintptr_t)num_rows * W * 2;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(src), b = reinterpret_cast<uintptr_t>(dst);
+  if (a < b + bytes && b < a + bytes) return MLA_ERR_INVALID_ARG;   // overlapping buffers
+  return launch_cache_convert(src, dst, num_rows, W, to_tiled, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_cache_pack(const mla_dims *dims, const void *rows, void *tiled, int64_t num_rows, mla_stream_t stream) {
+  return cache_convert(dims, rows, tiled, num_rows, true, stream);
+}
+
+int mla_cache_unpack(const mla_dims *dims, const void *tiled, void *rows, int64_t num_rows, mla_stream_t stream) {
+  return cache_convert(dims, tiled, rows, num_rows, false, stream);
 }
 
 }  // extern "C"

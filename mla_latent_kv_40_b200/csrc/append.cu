@@ -87,19 +87,20 @@ append_latent_kernel(AppendArgs a) {
     if (lane == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
     return;
   }
-  T *ckv = static_cast<T *>(a.c_kv) + row * a.ckv_stride;
-  T *kpe = static_cast<T *>(a.k_pe) + row * a.kpe_stride;
+  auto at = [&](int d) {
+    return latent_elem<T>(a.c_kv, a.k_pe, a.ckv_stride, a.kpe_stride, a.layout, a.d_c, W, row, d);
+  };
   const T *g = static_cast<const T *>(a.gamma);
   for (int j = lane; j < a.d_c; j += 32) {
     const float gj = g ? to_f32(g[j]) : 1.f;
-    ckv[j] = from_f32<T>(c[j] * inv * gj);
+    *at(j) = from_f32<T>(c[j] * inv * gj);
   }
   for (int i = lane; i < a.d_rope / 2; i += 32) {
     float cs_, sn_;
     rope_cos_sin(p, i, a.d_rope, a.rope_base, &cs_, &sn_);
     const float x = c[a.d_c + 2 * i], y = c[a.d_c + 2 * i + 1];
-    kpe[2 * i] = from_f32<T>(x * cs_ - y * sn_);
-    kpe[2 * i + 1] = from_f32<T>(x * sn_ + y * cs_);
+    *at(a.d_c + 2 * i) = from_f32<T>(x * cs_ - y * sn_);
+    *at(a.d_c + 2 * i + 1) = from_f32<T>(x * sn_ + y * cs_);
   }
 }
 

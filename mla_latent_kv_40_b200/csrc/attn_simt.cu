@@ -68,8 +68,6 @@ attn_simt_kernel(AttnArgs a) {
 #pragma unroll
     for (int i = 0; i < kMaxDcPerThr; ++i) acc[r][i] = 0.f;
 
-  const T *ckv = static_cast<const T *>(a.cache.c_kv);
-  const T *kpe = static_cast<const T *>(a.cache.k_pe);
   for (int k0 = k_begin; k0 < k_end; k0 += kKeyTile) {
     __syncthreads();
     // Stage the tile's rows; rows past the end are zero (and masked below).
@@ -83,9 +81,7 @@ attn_simt_kernel(AttnArgs a) {
       }
       for (int d = lane; d < W; d += 32) {
         float v = 0.f;
-        if (row >= 0)
-          v = d < a.d_c ? to_f32(ckv[row * a.cache.ckv_stride + d])
-                        : to_f32(kpe[row * a.cache.kpe_stride + (d - a.d_c)]);
+        if (row >= 0) v = a.cache.load<T>(row, d);
         ks[kk * ldk + d] = v;
       }
     }

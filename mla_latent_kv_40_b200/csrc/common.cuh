@@ -38,6 +38,27 @@ __device__ __forceinline__ int64_t cache_row(const int32_t *block_table, int max
   return (int64_t)blk * block_size + (i % block_size);
 }
 
+// ---- latent pool layouts -----------------------------------------------------
+// Byte offset of element (row r, dim d) in a tiled pool whose rows are W
+// elements wide: 64-token pages of W/64 chunks; chunk c = d / 64 holds token t
+// at byte 128 t and its 16-byte group g = (d / 8) % 8 at 16 * (g ^ (t % 8)).
+__host__ __device__ __forceinline__ int64_t tiled_byte_offset(int64_t r, int d, int W) {
+  const int64_t page = r >> 6;
+  const int t = (int)(r & 63);
+  const int c = d >> 6, g = (d >> 3) & 7, e = d & 7;
+  return page * (int64_t)W * 128 + (int64_t)c * 8192 + t * 128 + ((g ^ (t & 7)) << 4) + e * 2;
+}
+
+// Address of element (row r, dim d), d in [0, d_c + d_rope): c_KV dims first,
+// then the RoPE key, in either pool layout.
+template <typename T>
+__device__ __forceinline__ T *latent_elem(void *c_kv, void *k_pe, int64_t ckv_stride, int64_t kpe_stride, int layout,
+                                          int d_c, int W, int64_t r, int d) {
+  if (layout == MLA_CACHE_TILED)
+    return reinterpret_cast<T *>(static_cast<char *>(c_kv) + tiled_byte_offset(r, d, W));
+  return d < d_c ? static_cast<T *>(c_kv) + r * ckv_stride + d : static_cast<T *>(k_pe) + r * kpe_stride + (d - d_c);
+}
+
 // ---- RoPE ------------------------------------------------------------------
 // cos/sin of p * base^(-2i/d).  The angle is formed and reduced modulo 2*pi in
 // double so that positions up to 2^31 keep full fp32 accuracy in the result.

@@ -33,9 +33,11 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "decode_tc.cuh"
+#include "mma_tile.cuh"
 #include "sm100.cuh"
 
 namespace mla {
@@ -48,22 +50,23 @@ constexpr int kSuper = 4;                          // page tiles per score tile:
 constexpr int kDc = 512, kDr = 64, kW = kDc + kDr;
 constexpr int kRows = 128;                         // M of every MMA: query rows per unit
 constexpr int kKStages = 6;                        // score CTA: [256 keys x 64 dims] stages in flight
-constexpr int kVStages = 2;                        // value CTA: [64 keys x 512 dims] stages in flight
+constexpr int kVStages = 4;                        // value CTA: [64 keys x 256 dims] half-page stages in flight
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;                   // per thread at launch (65536 / 384, rounded down to 8)
 constexpr int kLowRegs = 56, kHighRegs = 224;
 static_assert(128 * kLowRegs + 256 * kHighRegs == kThreads * kLaunchRegs, "register split must match the launch");
 constexpr uint32_t kChunkBytes = kTileKeys * 128;  // one [64 keys x 64 dims] bf16 TMA box, 128B-swizzled
 constexpr uint32_t kKStageBytes = kSuper * kChunkBytes;            // 32768
-constexpr uint32_t kVTileBytes = 8 * kChunkBytes;                  // 65536
+constexpr uint32_t kVStageBytes = 4 * kChunkBytes;                 // 32768
 constexpr uint32_t kPBytes = kRows * kTileKeys * 2;                // 16384
 constexpr int kPSlots = 5;                         // P page tiles in flight from the score CTA to the value CTA
 constexpr uint32_t kPTxBytes = kPBytes + kRows * 4 + 4 * 4;       // P tile + alpha column + 4 warp flags
 constexpr uint32_t kQpeOff = 0;                                    // score CTA: Q rope part, [128 x 64] bf16
 constexpr uint32_t kKOff = kRows * 128;                            // score CTA: key stages
-constexpr uint32_t kPOff = kVStages * kVTileBytes;                 // value CTA: P slots
+constexpr uint32_t kPOff = kVStages * kVStageBytes;                // value CTA: P slots
 constexpr uint32_t kRegionA = kKOff + kKStages * kKStageBytes;     // 212992
 static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
+constexpr int kPrefetchPages = 8;                  // score CTA: pages prefetched into L2 ahead of the smem stream
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint64_t kWaitNs = 2000000000ull;        // 2 s per wait
 constexpr int kMaxClusters = 128;
@@ -86,7 +89,7 @@ enum Bar {
 // A request from the value CTA's MMA thread to its epilogue warps.
 struct Req {
   int kind;        // 0: fix up a tile before its MMA, 1: unit epilogue
-  int vstage, slot, nvalid, tail, rescale, segid, last_slot, last_parity;
+  int vstage0, vstage1, slot, nvalid, tail, rescale, segid, last_slot, last_parity;
 };
 
 struct SmemB {                       // small region after the tiles
@@ -118,6 +121,9 @@ struct TcParams {
   int *seg_info;                     // [U][2]
   int *timeout_rec;                  // [kTimeoutRecInts]: where bounded waits gave up (diagnostics)
   int *dev_status;
+  const unsigned char *tiled;        // tiled page pool (pages move by bulk copy), or NULL: row pool via TMA maps
+  const unsigned char *row_pool;     // row pool base (c_kv) for L2 prefetch
+  int rows_contig;                   // row pool with fused 576-wide rows: a page is 73728 contiguous bytes
 };
 
 __device__ __forceinline__ int seq_len_clamped(const TcParams &p, int b) {
@@ -282,6 +288,32 @@ __device__ __forceinline__ int64_t tile_row(const TcParams &p, int b, int t) {
   return (int64_t)blk * p.block_size + (key % p.block_size);
 }
 
+// Pool rows of a sequence's pages, looked up a warp-load at a time: lane l keeps the
+// rows of pages base + l and base + 32 + l.  Warp-collective; pages must be asked
+// for in non-decreasing order per sequence, at most 32 pages behind the newest.
+struct PageRows {
+  int b = -1, base = 0;
+  int64_t r0 = -1, r1 = -1;
+  __device__ void load(const TcParams &p) {
+    const int lane = threadIdx.x & 31;
+    r0 = tile_row(p, b, base + lane);
+    r1 = tile_row(p, b, base + 32 + lane);
+  }
+  __device__ int64_t get(const TcParams &p, int seq, int page) {
+    if (seq != b || page < base || page >= base + 96) {
+      b = seq;
+      base = page;
+      load(p);
+    } else if (page >= base + 64) {
+      base += 32;
+      r0 = r1;
+      r1 = tile_row(p, b, base + 32 + (threadIdx.x & 31));
+    }
+    const int k = page - base;
+    return __shfl_sync(0xffffffffu, k < 32 ? r0 : r1, k & 31);
+  }
+};
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_pe,
                      const TcParams p) {
@@ -319,7 +351,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
     tmem_relinquish();
   }
   if (warp == 0) make_plan(p, sb, cid, C);
-  if (threadIdx.x == 32) {
+  if (threadIdx.x == 32 && !p.tiled) {
     tma_prefetch_desc(&map_c);
     tma_prefetch_desc(&map_pe);
   }
@@ -349,34 +381,50 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (rank == 0) {
-      if (warp == 0 && lane == 0) {
-      // ---- key producer: a score tile is up to 4 pages (256 keys); it is streamed as 9 stages of
-      // [256 keys x 64 dims] (8 latent chunks, then the RoPE key), one TMA box per page.
+      if (warp == 0) {
+      // ---- key producer (whole warp: lookups in warp-wide batches, lane 0 issues): a score tile
+      // is up to 4 pages (256 keys), streamed as 9 stages of [256 keys x 64 dims] (8 latent chunks,
+      // then the RoPE key).  Pages further ahead are prefetched into L2 (a page is contiguous in a
+      // tiled pool and in a fused row pool), so the shared-memory stages wait on L2, not DRAM.
       SegIter it = it0;
+      PageRows pr;
       uint32_t n = 0;
       uint32_t uses[kKStages] = {0, 0, 0, 0, 0, 0};
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
+        int pf = t0 + kSuper;   // next page to prefetch
         for (int T = t0; T < t1; T += kSuper) {
           const int npg = min(kSuper, t1 - T);
           int32_t rows[kSuper];
 #pragma unroll
           for (int pg = 0; pg < kSuper; ++pg) {
-            int64_t row = pg < npg ? tile_row(p, b, T + pg) : 0;
+            int64_t row = pg < npg ? pr.get(p, b, T + pg) : 0;
             if (row < 0) {
-              report(p.dev_status, MLA_ERR_BAD_INDEX);
+              if (lane == 0) report(p.dev_status, MLA_ERR_BAD_INDEX);
               row = 0;
             }
             rows[pg] = (int32_t)row;
           }
+          const int pf_end = min(t1, T + kSuper + kPrefetchPages);
+          for (; pf < pf_end; ++pf) {
+            const int64_t prow = pr.get(p, b, pf);
+            if (prow < 0 || lane != 0) continue;
+            if (p.tiled) prefetch_l2(p.tiled + (prow / kTileKeys) * (9 * kChunkBytes), 9 * kChunkBytes);
+            else if (p.rows_contig) prefetch_l2(p.row_pool + prow * (int64_t)kW * 2, kTileKeys * kW * 2);
+          }
           for (int j = 0; j < 9; ++j, ++n) {
-            sb.prog[warp] = (int)n;
+            if (lane == 0) sb.prog[warp] = (int)n;
             const int s = n % kKStages;
-            if (n >= kKStages && !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done0;
-            const uint32_t dst = smem_u32(tiles + kKOff + s * kKStageBytes);
-            mbar_expect_tx(bar(B_KFULL + s), npg * kChunkBytes);
-            for (int pg = 0; pg < npg; ++pg) {
-              if (j < 8) tma_load_2d(dst + pg * kChunkBytes, &map_c, 64 * j, rows[pg], bar(B_KFULL + s));
-              else tma_load_2d(dst + pg * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
+            if (n >= kKStages && !warp_wait(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done0;
+            if (lane == 0) {
+              const uint32_t dst = smem_u32(tiles + kKOff + s * kKStageBytes);
+              mbar_expect_tx(bar(B_KFULL + s), npg * kChunkBytes);
+              for (int pg = 0; pg < npg; ++pg) {
+                if (p.tiled)   // chunk j of a page is 8 KB, already in the order the MMA reads it
+                  bulk_load(dst + pg * kChunkBytes, p.tiled + (int64_t)(rows[pg] / kTileKeys) * (9 * kChunkBytes) + j * kChunkBytes,
+                            kChunkBytes, bar(B_KFULL + s));
+                else if (j < 8) tma_load_2d(dst + pg * kChunkBytes, &map_c, 64 * j, rows[pg], bar(B_KFULL + s));
+                else tma_load_2d(dst + pg * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
+              }
             }
             ++uses[s];
           }
@@ -384,8 +432,9 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       }
     prod_done0:
       // Drain: the last load issued on each stage must have landed before exit.
-      for (int s = 0; s < kKStages; ++s)
-        if (uses[s]) mbar_wait(bar(B_KFULL + s), (uses[s] - 1) & 1, kWaitNs);
+      if (lane == 0)
+        for (int s = 0; s < kKStages; ++s)
+          if (uses[s]) mbar_wait(bar(B_KFULL + s), (uses[s] - 1) & 1, kWaitNs);
       } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer: S [128 x N] = Q . K^T, N = 64 * pages (256 for a full score tile).
       // The latent part of Q is the A operand from tensor memory; the RoPE part is in shared memory.
@@ -423,44 +472,56 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       }
       }
     } else {
-      if (warp == 0 && lane == 0) {
-      // ---- latent-tile producer (c_KV part only)
+      if (warp == 0) {
+      // ---- latent producer (whole warp: lookups in warp-wide batches, lane 0 issues): each page's
+      // c_KV part is streamed as two half-page stages [64 keys x 256 dims], one per PV MMA group.
       if (cid == 0) {
         // Units with no tiles get an empty segment list (their rows combine to zero).
-        for (int u = 0; u < p.U; ++u)
+        for (int u = lane; u < p.U; u += 32)
           if (unit_tiles(p, u) == 0) {
             p.seg_info[2 * u] = 0;
             p.seg_info[2 * u + 1] = 0;
           }
-        for (int bb = 0; bb < p.B; ++bb) {
+        for (int bb = lane; bb < p.B; bb += 32) {
           const int S = p.seqlens[bb];
           if (S < p.n_q || S > p.max_seqlen) report(p.dev_status, MLA_ERR_BAD_INDEX);
         }
       }
       SegIter it = it0;
+      PageRows pr;
       uint32_t n = 0;
-      uint32_t uses[kVStages] = {0, 0};
+      uint32_t uses[kVStages] = {0, 0, 0, 0};
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        if (first_u) {
+        if (first_u && lane == 0) {
           // This cluster holds the unit's first tile: publish where its partials live.
           p.seg_info[2 * (b * p.n_rb + rb)] = segid;
           p.seg_info[2 * (b * p.n_rb + rb) + 1] = nseg;
         }
-        for (int t = t0; t < t1; ++t, ++n) {
-          sb.prog[warp] = (int)n;
-          const int s = n % kVStages;
-          if (n >= kVStages && !wait_or_abort(sb, bar(B_VEMPTY + s), ((n / kVStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done1;
-          int64_t row = tile_row(p, b, t);
+        for (int t = t0; t < t1; ++t) {
+          int64_t row = pr.get(p, b, t);
           if (row < 0) row = 0;   // reported by the score CTA
-          const uint32_t dst = smem_u32(tiles + s * kVTileBytes);
-          mbar_expect_tx(bar(B_VFULL + s), kVTileBytes);
-          for (int j = 0; j < 8; ++j) tma_load_2d(dst + j * kChunkBytes, &map_c, 64 * j, (int32_t)row, bar(B_VFULL + s));
-          ++uses[s];
+          for (int h = 0; h < 2; ++h, ++n) {
+            if (lane == 0) sb.prog[warp] = (int)n;
+            const int s = n % kVStages;
+            if (n >= kVStages && !warp_wait(sb, bar(B_VEMPTY + s), ((n / kVStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done1;
+            if (lane == 0) {
+              const uint32_t dst = smem_u32(tiles + s * kVStageBytes);
+              mbar_expect_tx(bar(B_VFULL + s), kVStageBytes);
+              if (p.tiled)   // latent chunks 4h .. 4h+3 of the page: 32 contiguous KB
+                bulk_load(dst, p.tiled + (row / kTileKeys) * (9 * kChunkBytes) + h * kVStageBytes, kVStageBytes,
+                          bar(B_VFULL + s));
+              else
+                for (int j = 0; j < 4; ++j)
+                  tma_load_2d(dst + j * kChunkBytes, &map_c, 64 * (4 * h + j), (int32_t)row, bar(B_VFULL + s));
+            }
+            ++uses[s];
+          }
         }
       }
     prod_done1:
-      for (int s = 0; s < kVStages; ++s)
-        if (uses[s]) mbar_wait(bar(B_VFULL + s), (uses[s] - 1) & 1, kWaitNs);
+      if (lane == 0)
+        for (int s = 0; s < kVStages; ++s)
+          if (uses[s]) mbar_wait(bar(B_VFULL + s), (uses[s] - 1) & 1, kWaitNs);
       } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer: O += P . C
       SegIter it = it0;
@@ -470,46 +531,57 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         if (uc > 0 && !wait_or_abort(sb, bar(B_OFREE), (uc - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
         const int S = seq_len_clamped(p, b);
-        for (int t = t0; t < t1; ++t, ++n, ++np) {
+        for (int t = t0; t < t1; ++t, n += 2, ++np) {
           sb.prog[warp] = (int)n;
-          const int s = n % kVStages, pb = np % kPSlots;
-          if (!wait_or_abort(sb, bar(B_VFULL + s), (n / kVStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__) ||
-              !wait_or_abort(sb, bar(B_PFULL + pb), (np / kPSlots) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
+          const int pb = np % kPSlots;
+          const int sv[2] = {(int)(n % kVStages), (int)((n + 1) % kVStages)};
+          const uint32_t pv[2] = {(n / kVStages) & 1, ((n + 1) / kVStages) & 1};
+          if (!wait_or_abort(sb, bar(B_PFULL + pb), (np / kPSlots) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
             ok = false;
             break;
           }
           const bool tail = (t + 1) * kTileKeys > S;
           const uint32_t *fl = sb.flags[pb];
           const bool resc = t != t0 && (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
+          bool have_v = false;
           if (tail || resc) {
             // Rare: let the epilogue warps zero the rows past the end and/or rescale O first.
             // A rescale reads O back, so every earlier MMA must have completed.
+            if (!wait_or_abort(sb, bar(B_VFULL + sv[0]), pv[0], p.dev_status, false, p.timeout_rec, __LINE__) ||
+                !wait_or_abort(sb, bar(B_VFULL + sv[1]), pv[1], p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            have_v = true;
             if (resc && !wait_or_abort(sb, bar(B_PVDONE + (np - 1) % kPSlots), ((np - 1) / kPSlots) & 1, p.dev_status,
                                        false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            sb.req = Req{0, s, pb, S - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
+            sb.req = Req{0, sv[0], sv[1], pb, S - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
             mbar_arrive(bar(B_REQ));
             if (!wait_or_abort(sb, bar(B_REQDONE), nfix & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
             ++nfix;
           }
-          tc_fence_after();
-          fence_proxy_async_smem();
-          const uint32_t vt = smem_u32(tiles + s * kVTileBytes);
           const uint32_t pt = smem_u32(tiles + kPOff + pb * kPBytes);
-#pragma unroll
-          for (int h = 0; h < 2; ++h)
+          // O[:, 256h .. 256h+255] += P . C[:, 256h ..]: one half-page stage per group of 4 MMAs.
+          for (int h = 0; h < 2; ++h) {
+            if (!have_v && !wait_or_abort(sb, bar(B_VFULL + sv[h]), pv[h], p.dev_status, false, p.timeout_rec, __LINE__)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            fence_proxy_async_smem();
+            const uint32_t vt = smem_u32(tiles + sv[h] * kVStageBytes);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
               const uint64_t ad = smem_desc_sw128(pt + ks * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(vt + h * 4 * kChunkBytes + ks * 2048, kChunkBytes, 1024);
+              const uint64_t bd = smem_desc_sw128(vt + ks * 2048, kChunkBytes, 1024);
               mma_ss(tbase + 256 * h, ad, bd, idesc, (t != t0 || ks > 0) ? 1u : 0u);
             }
+            tc_commit(bar(B_VEMPTY + sv[h]));
+          }
+          if (!ok) break;
           tc_commit(bar(B_PVDONE + pb));
-          tc_commit(bar(B_VEMPTY + s));
         }
         if (!ok) break;
         // Unit epilogue request: the epilogue warps wait for the last MMAs themselves.
         const uint32_t last = np - 1;
-        sb.req = Req{1, 0, 0, 0, 0, 0, segid, (int)(last % kPSlots), (int)((last / kPSlots) & 1)};
+        sb.req = Req{1, 0, 0, 0, 0, 0, 0, segid, (int)(last % kPSlots), (int)((last / kPSlots) & 1)};
         mbar_arrive(bar(B_REQ));
         ++uc;
       }
@@ -687,11 +759,11 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           if (q.kind == 0) {
             if (q.tail) {
               // Rows past the sequence end may hold anything (NaN): zero them so 0 * row stays 0.
-              unsigned char *vt = tiles + q.vstage * kVTileBytes;
               const int nrow = kTileKeys - q.nvalid;
               for (int e = threadIdx.x - 128; e < nrow * 64; e += 128) {
                 const int row = q.nvalid + e / 64, rest = e % 64, ch = rest / 8, piece = rest % 8;
-                *reinterpret_cast<uint4 *>(vt + ch * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+                unsigned char *vt = tiles + (ch < 4 ? q.vstage0 : q.vstage1) * kVStageBytes;
+                *reinterpret_cast<uint4 *>(vt + (ch & 3) * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
               }
               fence_proxy_async_smem();
             }
@@ -758,21 +830,40 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
 }
 
 // ------------------------------------------------------------ combine (+ W_UV)
-constexpr int kCombRows = 16;
+// CTA = (head s, 64 query rows (b, j)).  The split partials of each row are
+// merged by their log-sum-exps into a bf16 [64 x 512] tile in shared memory,
+// which is then multiplied by W_UV[s] ([512 x d_v], streamed in 64-row
+// slices) on warp-level tensor cores: out^(s) = o_lat W_UV^(s).
+constexpr int kCombRows = 64;
 constexpr int kCombThreads = 256;
 constexpr int kMaxSegPerUnit = kMaxClusters + 1;
+constexpr int kOlLd = kDc + 8;             // padded bf16 row of the merged tile
+constexpr int kWLd = 128 + 8;              // padded bf16 row of a W_UV slice
 
 __global__ void __launch_bounds__(kCombThreads)
-tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part, const float *lse_part,
-                  const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out) {
-  extern __shared__ float smem[];
-  float *ol = smem;                         // [kCombRows][512]
-  float *wgt = ol + kCombRows * kDc;        // [kCombRows][kMaxSegPerUnit]
-  int *sinfo = reinterpret_cast<int *>(wgt + kCombRows * kMaxSegPerUnit);   // [kCombRows][3]
+tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part,
+                  const float *lse_part, const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out) {
+  extern __shared__ __align__(16) unsigned char csm[];
+  __nv_bfloat16 *ol = reinterpret_cast<__nv_bfloat16 *>(csm);                     // [64][kOlLd]
+  __nv_bfloat16 *wsl = ol + kCombRows * kOlLd;                                     // [2][64][kWLd]
+  float *wgt = reinterpret_cast<float *>(wsl + 2 * 64 * kWLd);                     // [64][kMaxSegPerUnit]
+  int *sinfo = reinterpret_cast<int *>(wgt + kCombRows * kMaxSegPerUnit);          // [64][3]
   const int s = blockIdx.x;
   const int g0 = blockIdx.y * kCombRows;
   const int rows = B * n_q;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // W_UV slices stream in while the partials are merged.
+  const __nv_bfloat16 *w = w_uv ? w_uv + (int64_t)s * kDc * d_v : nullptr;
+  auto load_w = [&](int buf, int k0) {
+    for (int c = tid; c < 64 * 16; c += kCombThreads) {       // 64 rows x 128 cols = 1024 chunks of 16 B
+      const int r = c >> 4, q = c & 15;
+      mma::cp16(wsl + (buf * 64 + r) * kWLd + q * 8, w + (int64_t)(k0 + r) * d_v + q * 8, true);
+    }
+    mma::cp_commit();
+  };
+  if (w) load_w(0, 0);
+
   for (int rr = warp; rr < kCombRows; rr += 8) {
     const int g = g0 + rr;
     int s0 = 0, ns = 0, lr = 0;
@@ -799,6 +890,7 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
 #pragma unroll
     for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    __syncwarp();
     for (int k = lane; k < ns; k += 32) wgt[rr * kMaxSegPerUnit + k] *= inv;
     if (lane == 0) {
       sinfo[3 * rr] = s0;
@@ -808,40 +900,76 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
     }
   }
   __syncthreads();
-  for (int e = tid; e < kCombRows * kDc; e += kCombThreads) {
-    const int rr = e / kDc, c = e % kDc;
+  // Merge, 8 latent columns (16 bytes of every partial) per step.
+  for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
+    const int rr = e / (kDc / 8), c8 = (e % (kDc / 8)) * 8;
     const int s0 = sinfo[3 * rr], ns = sinfo[3 * rr + 1], lr = sinfo[3 * rr + 2];
-    float v = 0.f;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int k = 0; k < ns; ++k) {
-      const float w = wgt[rr * kMaxSegPerUnit + k];
-      if (w != 0.f) v = fmaf(w, __bfloat162float(o_part[((int64_t)(s0 + k) * kRows + lr) * kDc + c]), v);
+      const float wk = wgt[rr * kMaxSegPerUnit + k];
+      if (wk == 0.f) continue;
+      const uint4 x = *reinterpret_cast<const uint4 *>(o_part + ((int64_t)(s0 + k) * kRows + lr) * kDc + c8);
+      const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(xh[i]);
+        v[2 * i] = fmaf(wk, f.x, v[2 * i]);
+        v[2 * i + 1] = fmaf(wk, f.y, v[2 * i + 1]);
+      }
     }
-    ol[e] = v;
+    uint4 packed;
+    __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ph[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<uint4 *>(ol + rr * kOlLd + c8) = packed;
   }
   __syncthreads();
-  if (!w_uv) {
-    for (int e = tid; e < kCombRows * kDc; e += kCombThreads) {
-      const int rr = e / kDc, c = e % kDc, g = g0 + rr;
-      if (g < rows) out[((int64_t)g * H + s) * kDc + c] = __float2bfloat16_rn(ol[e]);
+  if (!w) {   // latent output: o_lat itself
+    for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
+      const int rr = e / (kDc / 8), c8 = (e % (kDc / 8)) * 8, g = g0 + rr;
+      if (g < rows) *reinterpret_cast<uint4 *>(out + ((int64_t)g * H + s) * kDc + c8) = *reinterpret_cast<const uint4 *>(ol + rr * kOlLd + c8);
     }
     return;
   }
-  const __nv_bfloat16 *w = w_uv + (int64_t)s * kDc * d_v;
-  for (int v = tid; v < d_v; v += kCombThreads) {
-    float acc[kCombRows];
+  // out [64 x 128] = ol [64 x 512] . W_UV[s] [512 x 128]; warp (wr, wc) owns rows 16wr.. and columns 64wc..
+  const int wr = warp & 3, wc = warp >> 2;
+  float acc[8][4];
 #pragma unroll
-    for (int rr = 0; rr < kCombRows; ++rr) acc[rr] = 0.f;
-    for (int c = 0; c < kDc; ++c) {
-      const float wv = __bfloat162float(w[(int64_t)c * d_v + v]);
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int rr = 0; rr < kCombRows; ++rr) acc[rr] = fmaf(ol[rr * kDc + c], wv, acc[rr]);
+    for (int k = 0; k < 4; ++k) acc[i][k] = 0.f;
+  for (int k0 = 0, buf = 0; k0 < kDc; k0 += 64, buf ^= 1) {
+    if (k0 + 64 < kDc) {
+      load_w(buf ^ 1, k0 + 64);
+      mma::cp_wait<1>();
+    } else {
+      mma::cp_wait<0>();
     }
+    __syncthreads();
 #pragma unroll
-    for (int rr = 0; rr < kCombRows; ++rr) {
-      const int g = g0 + rr;
-      if (g < rows) out[((int64_t)g * H + s) * d_v + v] = __float2bfloat16_rn(acc[rr]);
+    for (int kk = 0; kk < 64; kk += 16) {
+      uint32_t a[4];
+      mma::load_a(ol, kOlLd, wr * 16, k0 + kk, a);
+#pragma unroll
+      for (int nt = 0; nt < 8; nt += 2) {
+        uint32_t bb[4];
+        mma::load_b2(wsl + buf * 64 * kWLd, kWLd, kk, wc * 64 + nt * 8, true, bb);
+        mma::mma16816(acc[nt], a, bb[0], bb[1]);
+        mma::mma16816(acc[nt + 1], a, bb[2], bb[3]);
+      }
     }
+    __syncthreads();
   }
+  const int gq = lane >> 2, q = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int g = g0 + wr * 16 + gq + 8 * hf;
+      if (g < rows)
+        *reinterpret_cast<__nv_bfloat162 *>(out + ((int64_t)g * H + s) * d_v + wc * 64 + nt * 8 + 2 * q) =
+            __floats2bfloat162_rn(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+    }
 }
 
 // ------------------------------------------------------------ host side
@@ -932,8 +1060,9 @@ int clusters_for_device() {
 }  // namespace
 
 bool tc_decode_supported(const mla_dims &d, int n_q) {
-  return d.dtype == MLA_BF16 && d.d_c == kDc && d.d_rope == kDr && d.block_size % kTileKeys == 0 &&
-         d.ckv_stride % 8 == 0 && d.kpe_stride % 8 == 0 && d.d_v <= 1024 && n_q * d.n_heads <= 2 * kRows;
+  const bool layout_ok = d.cache_layout == MLA_CACHE_TILED || (d.ckv_stride % 8 == 0 && d.kpe_stride % 8 == 0);
+  return d.dtype == MLA_BF16 && d.d_c == kDc && d.d_rope == kDr && d.block_size % kTileKeys == 0 && layout_ok &&
+         d.d_v == 128 && n_q * d.n_heads <= 2 * kRows;
 }
 
 int tc_decode_kernel_launches() { return 2; }
@@ -945,17 +1074,22 @@ size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q) {
 
 int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, const CacheView &cache,
                         const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st) {
-  if ((reinterpret_cast<uintptr_t>(cache.c_kv) & 15) || (reinterpret_cast<uintptr_t>(cache.k_pe) & 15) ||
+  const bool tiled = cache.layout == MLA_CACHE_TILED;
+  if ((reinterpret_cast<uintptr_t>(cache.c_kv) & 15) || (!tiled && (reinterpret_cast<uintptr_t>(cache.k_pe) & 15)) ||
       (reinterpret_cast<uintptr_t>(q_abs) & 15))
     return MLA_ERR_INVALID_ARG;
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
   const WsLayout L = ws_layout(B, n_rb);
   char *w = static_cast<char *>(ws);
   CUtensorMap mc, mpe;
-  const uint64_t rows = (uint64_t)cache.num_blocks * cache.block_size;
-  int rc = make_map(&mc, cache.c_kv, kDc, rows, (uint64_t)cache.ckv_stride * 2);
-  if (rc) return rc;
-  if ((rc = make_map(&mpe, cache.k_pe, kDr, rows, (uint64_t)cache.kpe_stride * 2))) return rc;
+  memset(&mc, 0, sizeof(mc));
+  memset(&mpe, 0, sizeof(mpe));
+  if (!tiled) {   // row pool: 2-D TMA boxes of [64 rows x 64 dims]
+    const uint64_t rows = (uint64_t)cache.num_blocks * cache.block_size;
+    int rc = make_map(&mc, cache.c_kv, kDc, rows, (uint64_t)cache.ckv_stride * 2);
+    if (rc) return rc;
+    if ((rc = make_map(&mpe, cache.k_pe, kDr, rows, (uint64_t)cache.kpe_stride * 2))) return rc;
+  }
   const int C = clusters_for_device();
   if (C <= 0) return MLA_ERR_CUDA;
   TcParams p;
@@ -972,6 +1106,10 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
   p.num_blocks = cache.num_blocks;
   p.block_size = cache.block_size;
   p.scale_log2 = default_scale(d) * 1.4426950408889634f;
+  p.tiled = tiled ? static_cast<const unsigned char *>(cache.c_kv) : nullptr;
+  p.row_pool = static_cast<const unsigned char *>(cache.c_kv);
+  p.rows_contig = !tiled && cache.ckv_stride == kW && cache.kpe_stride == kW &&
+                  static_cast<const char *>(cache.k_pe) == static_cast<const char *>(cache.c_kv) + 2 * kDc;
   p.o_part = reinterpret_cast<__nv_bfloat16 *>(w + L.o_part);
   p.lse_part = reinterpret_cast<float *>(w + L.lse_part);
   p.seg_info = reinterpret_cast<int *>(w + L.seg_info);
@@ -993,7 +1131,9 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
   const WsLayout L = ws_layout(B, n_rb);
   char *w = static_cast<char *>(ws);
-  const size_t smem = sizeof(float) * (kCombRows * kDc + kCombRows * kMaxSegPerUnit) + sizeof(int) * 3 * kCombRows;
+  const size_t smem = sizeof(__nv_bfloat16) * (kCombRows * kOlLd + 2 * 64 * kWLd) +
+                      sizeof(float) * kCombRows * kMaxSegPerUnit + sizeof(int) * 3 * kCombRows;
+  if (w_uv && d.d_v != 128) return MLA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid(d.n_heads, (B * n_q + kCombRows - 1) / kCombRows);

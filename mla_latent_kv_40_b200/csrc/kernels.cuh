@@ -13,6 +13,7 @@ struct AppendArgs {
   int64_t ckv_stride, kpe_stride;
   const int32_t *block_table;
   int num_seqs, max_blocks_per_seq, num_blocks, block_size;
+  int layout;
   float rms_eps, rope_base;
   int *dev_status;
 };
@@ -31,6 +32,14 @@ struct CacheView {
   int64_t ckv_stride, kpe_stride;
   const int32_t *block_table;
   int max_blocks_per_seq, num_blocks, block_size;
+  int layout;                    // mla_cache_layout
+  int d_c, W;                    // latent width and full row width d_c + d_rope
+
+  template <typename T>
+  __device__ __forceinline__ float load(int64_t row, int d) const {
+    return to_f32(*latent_elem<const T>(const_cast<void *>(c_kv), const_cast<void *>(k_pe), ckv_stride, kpe_stride,
+                                        layout, d_c, W, row, d));
+  }
 };
 
 // Split-KV attention over the latent cache (the absorbed decode core).
@@ -75,5 +84,12 @@ int launch_absorb(const AbsorbArgs &a, bool bf16, cudaStream_t st);
 int launch_attn_simt(const AttnArgs &a, bool bf16, cudaStream_t st);
 int launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st);
 int launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st);
+// bf16 tensor-core (mma.sync) projections.
+size_t append_mma_workspace(int T, int d_model, int W, int *nsplit, int *k_per_split);
+bool append_mma_supported(const AppendArgs &a, bool bf16);
+int launch_append_mma(const AppendArgs &a, void *ws, cudaStream_t st);
+bool absorb_mma_supported(const AbsorbArgs &a, bool bf16);
+int launch_absorb_mma(const AbsorbArgs &a, cudaStream_t st);
+int launch_cache_convert(const void *src, void *dst, int64_t num_rows, int W, bool to_tiled, cudaStream_t st);
 
 }  // namespace mla

@@ -58,8 +58,6 @@ prefill_decompress_kernel(PrefillArgs a) {
   const int t0 = blockIdx.y * kDecRows;
   const int tid = threadIdx.x;
   const int dqk = a.d_nope + a.d_rope;
-  const T *ckv = static_cast<const T *>(a.cache.c_kv);
-  const T *kpe = static_cast<const T *>(a.cache.k_pe);
   __shared__ int64_t rows[kDecRows];
   if (tid < kDecRows) {
     const int t = t0 + tid;
@@ -79,7 +77,7 @@ prefill_decompress_kernel(PrefillArgs a) {
   __syncthreads();
   for (int e = tid; e < kDecRows * a.d_c; e += kPfThreads) {
     const int r = e / a.d_c, c = e % a.d_c;
-    cs[e] = rows[r] >= 0 ? to_f32(ckv[rows[r] * a.cache.ckv_stride + c]) : 0.f;
+    cs[e] = rows[r] >= 0 ? a.cache.load<T>(rows[r], c) : 0.f;
   }
   __syncthreads();
   T *kb = static_cast<T *>(a.kbuf);
@@ -110,7 +108,7 @@ prefill_decompress_kernel(PrefillArgs a) {
     const int r = e / a.d_rope, d = e % a.d_rope;
     const int t = t0 + r;
     if (t < a.total && rows[r] >= 0)
-      kb[((int64_t)t * a.H + s) * dqk + a.d_nope + d] = kpe[rows[r] * a.cache.kpe_stride + d];
+      kb[((int64_t)t * a.H + s) * dqk + a.d_nope + d] = from_f32<T>(a.cache.load<T>(rows[r], a.d_c + d));
   }
 }
 

@@ -26,25 +26,43 @@ def check_close(got, ref, dtype: str, what: str = ""):
     return dict(maxabs=maxabs, rel_l2=rel)
 
 
-def dims_of(mla, d, block_size):
+def dims_of(mla, d, block_size, layout=0):
     return mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, block_size, d.dtype,
-                         rope_base=d.rope_base, rms_eps=d.rms_eps)
+                         rope_base=d.rope_base, rms_eps=d.rms_eps, cache_layout=layout)
+
+
+def tiled_ok(d, block_size):
+    """The tiled page layout needs bf16, 64-token pages inside blocks and 64-dim chunks."""
+    return d.dtype == "bf16" and block_size % 64 == 0 and (d.d_c + d.d_rope) % 64 == 0
+
+
+def device_pool(mla, d, block_size, pool_rows_cpu, layout):
+    """The latent pool on the device in the requested layout: (c_kv, k_pe, keepalive)."""
+    rows = pool_rows_cpu.cuda()
+    if layout == 0:
+        return rows, rows[:, d.d_c:], rows
+    tiled = torch.empty_like(rows)
+    mla.mla_cache_pack(dims_of(mla, d, block_size, 1), rows, tiled)
+    return tiled, tiled, tiled
 
 
 def to_dev(inp, keys):
     return {k: inp[k].cuda() for k in keys}
 
 
-def gpu_decode(mla, inp, latent=False, status=None):
-    """Run mla_decode (or mla_decode_latent) on the device; returns CPU (out, lse, dev_status)."""
+def gpu_decode(mla, inp, latent=False, status=None, layout=None):
+    """Run mla_decode (or mla_decode_latent) on the device; returns CPU (out, lse, dev_status).
+
+    layout: 0 row pool, 1 tiled page pool; default tiled where the shape allows it."""
     d = inp["dims"]
     bs = inp["block_size"]
-    dims = dims_of(mla, d, bs)
-    dev = to_dev(inp, ["q_nope", "q_pe", "pool", "block_table", "seqlens", "w_uk", "w_uv"])
+    if layout is None:
+        layout = 1 if tiled_ok(d, bs) else 0
+    dims = dims_of(mla, d, bs, layout)
+    dev = to_dev(inp, ["q_nope", "q_pe", "block_table", "seqlens", "w_uk", "w_uv"])
     B, n_q, H = inp["q_nope"].shape[:3]
     max_seqlen = int(inp["seqlens"].max())
-    pool = dev["pool"]
-    c_kv, k_pe = pool, pool[:, d.d_c:]
+    c_kv, k_pe, _keep = device_pool(mla, d, bs, inp["pool"], layout)
     width = d.d_c if latent else d.d_v
     out = torch.full((B, n_q, H, width), float("nan"), dtype=d.torch_dtype, device="cuda")
     lse = torch.full((B, n_q, H), float("nan"), dtype=torch.float32, device="cuda")

@@ -18,7 +18,8 @@ def _declared():
 def test_header_declares_the_boundary():
     names = _declared()
     for want in ("mla_append_latent", "mla_decode_workspace_size", "mla_decode", "mla_prefill",
-                 "mla_prefill_workspace_size", "mla_status_string", "mla_absorb_q", "mla_decode_latent"):
+                 "mla_prefill_workspace_size", "mla_status_string", "mla_absorb_q", "mla_decode_latent",
+                 "mla_cache_pack", "mla_cache_unpack"):
         assert want in names
 
 
@@ -31,14 +32,14 @@ def test_library_exports_every_declared_symbol():
 
 def test_status_strings():
     import mla_latent_kv_40_b200 as mla
-    for code in range(-6, 1):
+    for code in range(-7, 1):
         assert mla.mla_status_string(code) and "unknown" not in mla.mla_status_string(code)
     assert "unknown" in mla.mla_status_string(-99)
 
 
 def test_dims_struct_matches_header_layout():
     import mla_latent_kv_40_b200 as mla
-    assert ctypes.sizeof(mla.mla_dims) == 13 * 4
+    assert ctypes.sizeof(mla.mla_dims) == 14 * 4
 
 
 def _lib():
@@ -79,10 +80,25 @@ def test_host_validation_rejects_bad_arguments():
     assert rc == -1
     # Append of zero tokens is a no-op that launches nothing.
     assert lib.mla_append_latent(ctypes.byref(d), 0, None, None, None, None, None, None, None, None, None,
-                                 1, 1, 1, None, None) == 0
+                                 1, 1, 1, None, ctypes.c_size_t(0), None, None) == 0
     assert lib.mla_append_latent(ctypes.byref(d), 3, None, fake, fake, None, fake, fake, fake, fake, None,
-                                 1, 1, 1, None, None) == -1
+                                 1, 1, 1, None, ctypes.c_size_t(0), None, None) == -1
+    # The tensor-core append needs scratch for bf16 shapes only.
+    assert lib.mla_append_workspace_size(ctypes.byref(d), 64, ctypes.byref(n)) == 0 and n.value == 0
+    v3 = mla.make_dims(128, 512, 64, 128, 128, 7168, 64, "bf16")
+    assert lib.mla_append_workspace_size(ctypes.byref(v3), 64, ctypes.byref(n)) == 0 and n.value > 0
     assert lib.mla_prefill_workspace_size(ctypes.byref(d), 1, 0, 10, ctypes.byref(n)) == -1
+    # Tiled page pools: bf16 only, blocks of whole 64-token pages, rows of whole 64-dim chunks.
+    t_ok = mla.make_dims(128, 512, 64, 128, 128, 7168, 64, "bf16", cache_layout=1)
+    assert lib.mla_decode_workspace_size(ctypes.byref(t_ok), 2, 1, 100, ctypes.byref(n)) == 0
+    for bad_t in (mla.make_dims(128, 512, 64, 128, 128, 7168, 64, "f32", cache_layout=1),
+                  mla.make_dims(128, 512, 64, 128, 128, 7168, 32, "bf16", cache_layout=1),
+                  mla.make_dims(128, 500, 64, 128, 128, 7168, 64, "bf16", cache_layout=1),
+                  mla.make_dims(128, 512, 64, 128, 128, 7168, 64, "bf16", cache_layout=2)):
+        assert lib.mla_decode_workspace_size(ctypes.byref(bad_t), 2, 1, 100, ctypes.byref(n)) == -1
+    # Pack / unpack: row counts in whole pages, distinct buffers.
+    assert lib.mla_cache_pack(ctypes.byref(t_ok), fake, P(0x100000000), 100, None) == -1
+    assert lib.mla_cache_pack(ctypes.byref(t_ok), fake, fake, 64, None) == -1
 
 
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):

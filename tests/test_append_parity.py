@@ -17,25 +17,29 @@ CASES = {
 }
 
 
-def _run(mla, inp, paged: bool, pool_rows: int, dims_):
+def _run(mla, inp, paged: bool, pool_rows: int, dims_, mma: bool = True):
     d = inp["dims"]
     dev = {k: inp[k].cuda() for k in ("h", "w_dkv", "w_kr", "gamma", "seq_idx", "pos", "block_table")}
     pool = torch.full((pool_rows, d.d_c + d.d_rope), float("nan"), dtype=d.torch_dtype, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     bt = dev["block_table"] if paged else None
+    nws = mla.mla_append_workspace_size(dims_, inp["h"].shape[0]) if mma else 0
+    ws = mla.alloc_workspace(nws) if nws else None
     mla.mla_append_latent(dims_, dev["h"], dev["w_dkv"], dev["w_kr"], dev["gamma"], dev["seq_idx"], dev["pos"],
                           pool, pool[:, d.d_c:], bt, inp["seqlens"].numel(), inp["max_blocks_per_seq"],
-                          pool_rows // inp["block_size"], st)
+                          pool_rows // inp["block_size"], st, workspace=ws)
     torch.cuda.synchronize()
     return pool.cpu(), int(st.item())
 
 
+@pytest.mark.parametrize("mma", [True, False])
 @pytest.mark.parametrize("name", list(CASES))
-def test_append_content_and_layout(lib, name):
+def test_append_content_and_layout(lib, name, mma):
+    """mma=True: tensor-core projection (bf16 shapes, with workspace); False: the CUDA-core kernel."""
     d, T, seqlens, bs = CASES[name]
     inp = make_append_inputs(d, T, torch.tensor(seqlens, dtype=torch.int32), bs, True, seed=300 + T)
     dims_ = dims_of(lib, d, bs)
-    pool, st = _run(lib, inp, True, inp["num_blocks"] * bs, dims_)
+    pool, st = _run(lib, inp, True, inp["num_blocks"] * bs, dims_, mma)
     assert st == 0
     c_ref, k_ref = oracle.append_latent(inp["h"], inp["w_dkv"], inp["w_kr"], inp["gamma"], inp["pos"],
                                         d.rms_eps, d.rope_base)

@@ -43,6 +43,17 @@ def test_decode_small_all_outputs(lib, name):
     assert np.max(np.abs(lse - ref_lse)) <= _lse_tol(inp["dims"].dtype)
 
 
+@pytest.mark.parametrize("name", ["small_v3_bf16", "small_v3_nq2_bf16", "small_v2lite_bf16", "small_v3_contig_bf16"])
+def test_decode_small_row_pool(lib, name):
+    """The same outputs from a row-layout pool (2-D TMA path of the tensor-core kernel)."""
+    inp = make_decode_inputs(DECODE_CASES[name])
+    out, lse, st = gpu_decode(lib, inp, layout=0)
+    assert st == 0
+    ref, ref_lse = _oracle(inp)
+    check_close(out, ref, inp["dims"].dtype, name + " rows")
+    assert np.max(np.abs(lse - ref_lse)) <= _lse_tol(inp["dims"].dtype)
+
+
 @pytest.mark.parametrize("name", ["small_f32", "small_v3_nq2_bf16", "small_v2lite_bf16"])
 def test_decode_latent_small(lib, name):
     inp = make_decode_inputs(DECODE_CASES[name])
