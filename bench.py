@@ -315,7 +315,8 @@ def run_mla(args):
     peaks = _peaks()
     value = step_flops * world / (ms * 1e-3) / 1e12
     att_gbs = lat_bytes / (att_ms * 1e-3) / 1e9
-    launches_per_step = 1 + mla.mla_decode_launches(dims, n_q)   # append, then absorb + attention + combine
+    # append (projection + finish with a workspace, one fused kernel without), then absorb + attention + combine
+    launches_per_step = (2 if app_ws is not None else 1) + mla.mla_decode_launches(dims, n_q)
     t_hbm = lat_bytes / (peaks["hbm_gbs"] * 1e9)
     t_flop = fl["total"] / (peaks["bf16_tflops"] * 1e12)
     line = {

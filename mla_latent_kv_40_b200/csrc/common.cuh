@@ -62,16 +62,24 @@ __device__ __forceinline__ T *latent_elem(void *c_kv, void *k_pe, int64_t ckv_st
 // ---- RoPE ------------------------------------------------------------------
 // cos/sin of p * base^(-2i/d).  The angle is formed and reduced modulo 2*pi in
 // double so that positions up to 2^31 keep full fp32 accuracy in the result.
-__device__ __forceinline__ void rope_cos_sin(int pos, int pair, int d_rope, float base, float *c,
-                                             float *s) {
-  const double theta = pow((double)base, -2.0 * (double)pair / (double)d_rope);
+// theta_i = base^(-2i / d_R), in double so that pos * theta_i keeps its fractional turns.
+__device__ __forceinline__ double rope_theta(int pair, int d_rope, float base) {
+  return pow((double)base, -2.0 * (double)pair / (double)d_rope);
+}
+
+__device__ __forceinline__ void rope_cos_sin_theta(int pos, double theta, float *c, float *s) {
   double a = (double)pos * theta;
-  const double two_pi = 6.283185307179586476925286766559;
-  a = a - two_pi * floor(a / two_pi);
+  const double two_pi = 6.283185307179586476925286766559, inv_two_pi = 0.15915494309189533576888376337251;
+  a = fma(-two_pi, floor(a * inv_two_pi), a);   // reduced to [0, 2*pi) up to one ulp of a at the ends
   float sf, cf;
   sincosf((float)a, &sf, &cf);
   *c = cf;
   *s = sf;
+}
+
+__device__ __forceinline__ void rope_cos_sin(int pos, int pair, int d_rope, float base, float *c,
+                                             float *s) {
+  rope_cos_sin_theta(pos, rope_theta(pair, d_rope, base), c, s);
 }
 
 __host__ __device__ inline float default_scale(const mla_dims &d) {

@@ -66,7 +66,10 @@ constexpr uint32_t kKOff = kRows * 128;                            // score CTA:
 constexpr uint32_t kPOff = kVStages * kVStageBytes;                // value CTA: P slots
 constexpr uint32_t kRegionA = kKOff + kKStages * kKStageBytes;     // 212992
 static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
-constexpr int kPrefetchPages = 8;                  // score CTA: pages prefetched into L2 ahead of the smem stream
+#ifndef MLA_TC_PREFETCH_PAGES
+#define MLA_TC_PREFETCH_PAGES 0
+#endif
+constexpr int kPrefetchPages = MLA_TC_PREFETCH_PAGES;  // score CTA: pages prefetched into L2 ahead of the smem stream
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint64_t kWaitNs = 2000000000ull;        // 2 s per wait
 constexpr int kMaxClusters = 128;
@@ -404,7 +407,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             }
             rows[pg] = (int32_t)row;
           }
-          const int pf_end = min(t1, T + kSuper + kPrefetchPages);
+          const int pf_end = kPrefetchPages > 0 ? min(t1, T + kSuper + kPrefetchPages) : pf;
           for (; pf < pf_end; ++pf) {
             const int64_t prow = pr.get(p, b, pf);
             if (prow < 0 || lane != 0) continue;
@@ -839,14 +842,15 @@ constexpr int kCombThreads = 256;
 constexpr int kMaxSegPerUnit = kMaxClusters + 1;
 constexpr int kOlLd = kDc + 8;             // padded bf16 row of the merged tile
 constexpr int kWLd = 128 + 8;              // padded bf16 row of a W_UV slice
+constexpr int kWSlices = 4;                // W_UV slices of 64 rows in flight
 
 __global__ void __launch_bounds__(kCombThreads)
 tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part,
                   const float *lse_part, const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out) {
   extern __shared__ __align__(16) unsigned char csm[];
   __nv_bfloat16 *ol = reinterpret_cast<__nv_bfloat16 *>(csm);                     // [64][kOlLd]
-  __nv_bfloat16 *wsl = ol + kCombRows * kOlLd;                                     // [2][64][kWLd]
-  float *wgt = reinterpret_cast<float *>(wsl + 2 * 64 * kWLd);                     // [64][kMaxSegPerUnit]
+  __nv_bfloat16 *wsl = ol + kCombRows * kOlLd;                                     // [kWSlices][64][kWLd]
+  float *wgt = reinterpret_cast<float *>(wsl + kWSlices * 64 * kWLd);              // [64][kMaxSegPerUnit]
   int *sinfo = reinterpret_cast<int *>(wgt + kCombRows * kMaxSegPerUnit);          // [64][3]
   const int s = blockIdx.x;
   const int g0 = blockIdx.y * kCombRows;
@@ -862,9 +866,13 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
     }
     mma::cp_commit();
   };
-  if (w) load_w(0, 0);
+  if (w)
+    for (int i = 0; i < kWSlices - 1; ++i) load_w(i, 64 * i);
 
-  for (int rr = warp; rr < kCombRows; rr += 8) {
+  // Merge weights: four threads per row, so every row's segment info and log-sum-exps are
+  // fetched at once rather than one row after another.
+  {
+    const int rr = tid >> 2, sub = tid & 3;
     const int g = g0 + rr;
     int s0 = 0, ns = 0, lr = 0;
     if (g < rows) {
@@ -878,21 +886,24 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
       if (s0 < 0 || s0 + ns > max_segs) { s0 = 0; ns = 0; }
     }
     float m = -CUDART_INF_F;
-    for (int k = lane; k < ns; k += 32) m = fmaxf(m, lse_part[(int64_t)(s0 + k) * kRows + lr]);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int k = sub; k < ns; k += 4) {
+      const float l = lse_part[(int64_t)(s0 + k) * kRows + lr];
+      wgt[rr * kMaxSegPerUnit + k] = l;
+      m = fmaxf(m, l);
+    }
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
     float sum = 0.f;
-    for (int k = lane; k < ns; k += 32) {
-      const float e = m == -CUDART_INF_F ? 0.f : __expf(lse_part[(int64_t)(s0 + k) * kRows + lr] - m);
+    for (int k = sub; k < ns; k += 4) {
+      const float e = m == -CUDART_INF_F ? 0.f : __expf(wgt[rr * kMaxSegPerUnit + k] - m);
       wgt[rr * kMaxSegPerUnit + k] = e;
       sum += e;
     }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
     const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    __syncwarp();
-    for (int k = lane; k < ns; k += 32) wgt[rr * kMaxSegPerUnit + k] *= inv;
-    if (lane == 0) {
+    for (int k = sub; k < ns; k += 4) wgt[rr * kMaxSegPerUnit + k] *= inv;
+    if (sub == 0) {
       sinfo[3 * rr] = s0;
       sinfo[3 * rr + 1] = ns;
       sinfo[3 * rr + 2] = lr;
@@ -900,28 +911,59 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
     }
   }
   __syncthreads();
-  // Merge, 8 latent columns (16 bytes of every partial) per step.
-  for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
-    const int rr = e / (kDc / 8), c8 = (e % (kDc / 8)) * 8;
-    const int s0 = sinfo[3 * rr], ns = sinfo[3 * rr + 1], lr = sinfo[3 * rr + 2];
-    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int k = 0; k < ns; ++k) {
-      const float wk = wgt[rr * kMaxSegPerUnit + k];
-      if (wk == 0.f) continue;
-      const uint4 x = *reinterpret_cast<const uint4 *>(o_part + ((int64_t)(s0 + k) * kRows + lr) * kDc + c8);
-      const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x);
+  // Merge, 8 latent columns (16 bytes of every partial) per item.  A thread owns one column
+  // group and, per pass, 8 rows; it walks the segments outermost so that its 8 loads of one
+  // segment are independent and in flight together.
+  {
+    constexpr int kGroups = kDc / 8;                         // 64 column groups
+    constexpr int kRowStep = kCombThreads / kGroups;         // 4
+    constexpr int kItems = 8;
+    constexpr int kPasses = kCombRows / (kRowStep * kItems); // 2
+    const int c8 = (tid % kGroups) * 8, rr0 = tid / kGroups;
+#pragma unroll 1
+    for (int pass = 0; pass < kPasses; ++pass) {
+      float v[kItems][8];
+      int nsr[kItems];
+      int maxns = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(xh[i]);
-        v[2 * i] = fmaf(wk, f.x, v[2 * i]);
-        v[2 * i + 1] = fmaf(wk, f.y, v[2 * i + 1]);
+      for (int i = 0; i < kItems; ++i) {
+        nsr[i] = sinfo[3 * (rr0 + kRowStep * (i + kItems * pass)) + 1];
+        maxns = max(maxns, nsr[i]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[i][k] = 0.f;
+      }
+      for (int k = 0; k < maxns; ++k) {
+        uint4 x[kItems];
+#pragma unroll
+        for (int i = 0; i < kItems; ++i) {
+          const int rr = rr0 + kRowStep * (i + kItems * pass);
+          x[i] = k < nsr[i] ? *reinterpret_cast<const uint4 *>(
+                                  o_part + ((int64_t)(sinfo[3 * rr] + k) * kRows + sinfo[3 * rr + 2]) * kDc + c8)
+                            : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int i = 0; i < kItems; ++i) {
+          const int rr = rr0 + kRowStep * (i + kItems * pass);
+          const float wk = k < nsr[i] ? wgt[rr * kMaxSegPerUnit + k] : 0.f;
+          const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[i]);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float2 f = __bfloat1622float2(xh[e2]);
+            v[i][2 * e2] = fmaf(wk, f.x, v[i][2 * e2]);
+            v[i][2 * e2 + 1] = fmaf(wk, f.y, v[i][2 * e2 + 1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kItems; ++i) {
+        const int rr = rr0 + kRowStep * (i + kItems * pass);
+        uint4 packed;
+        __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) ph[e2] = __floats2bfloat162_rn(v[i][2 * e2], v[i][2 * e2 + 1]);
+        *reinterpret_cast<uint4 *>(ol + rr * kOlLd + c8) = packed;
       }
     }
-    uint4 packed;
-    __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) ph[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-    *reinterpret_cast<uint4 *>(ol + rr * kOlLd + c8) = packed;
   }
   __syncthreads();
   if (!w) {   // latent output: o_lat itself
@@ -938,18 +980,17 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int k = 0; k < 4; ++k) acc[i][k] = 0.f;
-  for (int k0 = 0, buf = 0; k0 < kDc; k0 += 64, buf ^= 1) {
-    if (k0 + 64 < kDc) {
-      load_w(buf ^ 1, k0 + 64);
-      mma::cp_wait<1>();
-    } else {
-      mma::cp_wait<0>();
-    }
+  for (int it = 0; it < kDc / 64; ++it) {
+    const int buf = it % kWSlices;
+    // Keep kWSlices - 1 slices in flight: issue slice it + 3 (or an empty group), then wait for slice it.
+    if (it + kWSlices - 1 < kDc / 64) load_w((it + kWSlices - 1) % kWSlices, 64 * (it + kWSlices - 1));
+    else mma::cp_commit();
+    mma::cp_wait<kWSlices - 1>();
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < 64; kk += 16) {
       uint32_t a[4];
-      mma::load_a(ol, kOlLd, wr * 16, k0 + kk, a);
+      mma::load_a(ol, kOlLd, wr * 16, 64 * it + kk, a);
 #pragma unroll
       for (int nt = 0; nt < 8; nt += 2) {
         uint32_t bb[4];
@@ -1131,7 +1172,7 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
   const WsLayout L = ws_layout(B, n_rb);
   char *w = static_cast<char *>(ws);
-  const size_t smem = sizeof(__nv_bfloat16) * (kCombRows * kOlLd + 2 * 64 * kWLd) +
+  const size_t smem = sizeof(__nv_bfloat16) * (kCombRows * kOlLd + kWSlices * 64 * kWLd) +
                       sizeof(float) * kCombRows * kMaxSegPerUnit + sizeof(int) * 3 * kCombRows;
   if (w_uv && d.d_v != 128) return MLA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))

@@ -97,50 +97,72 @@ append_proj_kernel(const __nv_bfloat16 *h, const __nv_bfloat16 *w_dkv, const __n
   }
 }
 
-// One warp per token: sum the splits, RMSNorm over d_c, RoPE the shared key, scatter.
-__global__ void __launch_bounds__(256)
+// One CTA per token, one thread per pair of columns: sum the splits (independent loads, so
+// they are in flight together), RMSNorm over d_c, RoPE the shared key, scatter.
+constexpr int kFinThreads = 288;   // (d_c + d_R) / 2 column pairs of the V3 and V2-Lite rows
+
+__global__ void __launch_bounds__(kFinThreads)
 append_finish_kernel(AppendArgs a, const float *part, int nsplit) {
-  extern __shared__ float cs[];                  // [8 warps][W]
-  const int W = a.d_c + a.d_rope;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tok = blockIdx.x * 8 + warp;
-  if (tok >= a.T) return;
-  float *c = cs + warp * W;
+  __shared__ float red[kFinThreads / 32];
+  const int W = a.d_c + a.d_rope, npair = W / 2;
+  const int tok = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t split_stride = (int64_t)a.T * W / 2;   // in float2
+  const float2 *pp = reinterpret_cast<const float2 *>(part) + (int64_t)tok * npair;
+  constexpr int kMaxPairsPerThr = 2;
+  float2 v[kMaxPairsPerThr];
   float ss = 0.f;
-  for (int j = lane; j < W; j += 32) {
-    float v = 0.f;
-    for (int s = 0; s < nsplit; ++s) v += part[((int64_t)s * a.T + tok) * W + j];
-    c[j] = v;
-    if (j < a.d_c) ss += v * v;
+#pragma unroll
+  for (int i = 0; i < kMaxPairsPerThr; ++i) {
+    const int j2 = tid + i * kFinThreads;
+    float2 acc = make_float2(0.f, 0.f);
+    if (j2 < npair) {
+#pragma unroll 8
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float2 x = pp[sp * split_stride + j2];
+        acc.x += x.x;
+        acc.y += x.y;
+      }
+      if (2 * j2 < a.d_c) ss += acc.x * acc.x + acc.y * acc.y;
+    }
+    v[i] = acc;
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  __syncwarp();
-  const float inv = rsqrtf(ss / (float)a.d_c + a.rms_eps);
+  if (lane == 0) red[warp] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kFinThreads / 32; ++w) tot += red[w];
+  const float inv = rsqrtf(tot / (float)a.d_c + a.rms_eps);
   const int b = a.seq_idx[tok], p = a.pos[tok];
   if (b < 0 || b >= a.num_seqs || p < 0 || (int64_t)p >= (int64_t)a.max_blocks_per_seq * a.block_size) {
-    if (lane == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
+    if (tid == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
     return;
   }
   const int64_t row = cache_row(a.block_table, a.max_blocks_per_seq, a.num_blocks, a.block_size, b, p);
   if (row < 0) {
-    if (lane == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
+    if (tid == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
     return;
   }
   auto at = [&](int d) {
     return latent_elem<__nv_bfloat16>(a.c_kv, a.k_pe, a.ckv_stride, a.kpe_stride, a.layout, a.d_c, W, row, d);
   };
   const __nv_bfloat16 *gm = static_cast<const __nv_bfloat16 *>(a.gamma);
-  for (int j = lane; j < a.d_c; j += 32) {
-    const float gj = gm ? __bfloat162float(gm[j]) : 1.f;
-    *at(j) = __float2bfloat16_rn(c[j] * inv * gj);
-  }
-  for (int i = lane; i < a.d_rope / 2; i += 32) {
-    float cs_, sn_;
-    rope_cos_sin(p, i, a.d_rope, a.rope_base, &cs_, &sn_);
-    const float x = c[a.d_c + 2 * i], y = c[a.d_c + 2 * i + 1];
-    *at(a.d_c + 2 * i) = __float2bfloat16_rn(x * cs_ - y * sn_);
-    *at(a.d_c + 2 * i + 1) = __float2bfloat16_rn(x * sn_ + y * cs_);
+#pragma unroll
+  for (int i = 0; i < kMaxPairsPerThr; ++i) {
+    const int j2 = tid + i * kFinThreads, j = 2 * j2;
+    if (j2 >= npair) continue;
+    if (j < a.d_c) {
+      const float g0 = gm ? __bfloat162float(gm[j]) : 1.f, g1 = gm ? __bfloat162float(gm[j + 1]) : 1.f;
+      *at(j) = __float2bfloat16_rn(v[i].x * inv * g0);
+      *at(j + 1) = __float2bfloat16_rn(v[i].y * inv * g1);
+    } else {
+      float cs_, sn_;
+      rope_cos_sin(p, (j - a.d_c) / 2, a.d_rope, a.rope_base, &cs_, &sn_);
+      *at(j) = __float2bfloat16_rn(v[i].x * cs_ - v[i].y * sn_);
+      *at(j + 1) = __float2bfloat16_rn(v[i].x * sn_ + v[i].y * cs_);
+    }
   }
 }
 
@@ -158,7 +180,8 @@ size_t append_mma_workspace(int T, int d_model, int W, int *nsplit, int *k_per_s
 }
 
 bool append_mma_supported(const AppendArgs &a, bool bf16) {
-  return bf16 && a.d_model % kBK == 0 && a.d_c % 64 == 0 && a.d_rope <= 64 && a.d_rope % 8 == 0;
+  return bf16 && a.d_model % kBK == 0 && a.d_c % 64 == 0 && a.d_rope <= 64 && a.d_rope % 8 == 0 &&
+         a.d_c + a.d_rope <= 2 * 2 * kFinThreads;
 }
 
 int launch_append_mma(const AppendArgs &a, void *ws, cudaStream_t st) {
@@ -171,10 +194,7 @@ int launch_append_mma(const AppendArgs &a, void *ws, cudaStream_t st) {
                                            static_cast<const __nv_bfloat16 *>(a.w_dkv),
                                            static_cast<const __nv_bfloat16 *>(a.w_kr), a.T, a.d_model, a.d_c,
                                            a.d_rope, kps, part);
-  const size_t smem = 8 * W * sizeof(float);
-  if (smem > 48 * 1024 && cudaFuncSetAttribute(append_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
-    return MLA_ERR_CUDA;
-  append_finish_kernel<<<(a.T + 7) / 8, 256, smem, st>>>(a, part, nsplit);
+  append_finish_kernel<<<a.T, kFinThreads, 0, st>>>(a, part, nsplit);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
@@ -231,16 +251,20 @@ absorb_mma_kernel(AbsorbArgs a) {
         *reinterpret_cast<__nv_bfloat162 *>(qo + ((int64_t)gr * a.H + s) * W + n0 + nt * 8 + 2 * q) =
             __floats2bfloat162_rn(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
     }
-  if (blockIdx.z != 0) return;
-  const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q_pe);
+  // RoPE of q_pe, spread over the gridDim.z CTAs of this (head, row tile): CTA z takes rows
+  // z, z + gridDim.z, ...; the pair frequencies are computed once per CTA.
+  __shared__ double theta[32];
   const int half = a.d_rope / 2;
+  if (tid < half) theta[tid] = rope_theta(tid, a.d_rope, a.rope_base);
+  __syncthreads();
+  const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q_pe);
   for (int e = tid; e < kBM * half; e += kPT) {
-    const int r = e / half, i = e % half, gr = m0 + r;
-    if (gr >= R) continue;
+    const int r = blockIdx.z + gridDim.z * (e / half), i = e % half, gr = m0 + r;
+    if (r >= kBM || gr >= R) continue;
     const int b = gr / a.n_q, j = gr % a.n_q;
     const int p = a.seqlens[b] - a.n_q + j;
     float cs, sn;
-    rope_cos_sin(p < 0 ? 0 : p, i, a.d_rope, a.rope_base, &cs, &sn);
+    rope_cos_sin_theta(p < 0 ? 0 : p, theta[i], &cs, &sn);
     const int64_t src = ((int64_t)gr * a.H + s) * a.d_rope + 2 * i;
     const float x = __bfloat162float(qp[src]), y = __bfloat162float(qp[src + 1]);
     *reinterpret_cast<__nv_bfloat162 *>(qo + ((int64_t)gr * a.H + s) * W + a.d_c + 2 * i) =
@@ -249,7 +273,7 @@ absorb_mma_kernel(AbsorbArgs a) {
 }
 
 bool absorb_mma_supported(const AbsorbArgs &a, bool bf16) {
-  return bf16 && a.d_nope % 16 == 0 && a.d_nope <= 256 && a.d_c % 128 == 0;
+  return bf16 && a.d_nope % 16 == 0 && a.d_nope <= 256 && a.d_c % 128 == 0 && a.d_rope <= 64;
 }
 
 int launch_absorb_mma(const AbsorbArgs &a, cudaStream_t st) {
