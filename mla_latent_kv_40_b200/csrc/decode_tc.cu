@@ -46,25 +46,27 @@ namespace {
 using namespace sm100;
 
 constexpr int kTileKeys = 64;                      // one cache page of keys (a "page tile")
-constexpr int kSuper = 4;                          // page tiles per score tile: N = 256 keys per MMA
+constexpr int kSuper = 2;                          // page tiles per score tile: N = 128 keys per MMA
 constexpr int kDc = 512, kDr = 64, kW = kDc + kDr;
 constexpr int kRows = 128;                         // M of every MMA: query rows per unit
-constexpr int kKStages = 6;                        // score CTA: [256 keys x 64 dims] stages in flight
+constexpr int kKStages = 10;                       // score CTA: [128 keys x 64 dims] stages in flight
 constexpr int kVStages = 4;                        // value CTA: [64 keys x 256 dims] half-page stages in flight
 constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;                   // per thread at launch (65536 / 384, rounded down to 8)
-constexpr int kLowRegs = 56, kHighRegs = 224;
-static_assert(128 * kLowRegs + 256 * kHighRegs == kThreads * kLaunchRegs, "register split must match the launch");
+constexpr int kLaunchRegs = 168;                   // per thread (65536 / 384, rounded down to 8)
 constexpr uint32_t kChunkBytes = kTileKeys * 128;  // one [64 keys x 64 dims] bf16 TMA box, 128B-swizzled
-constexpr uint32_t kKStageBytes = kSuper * kChunkBytes;            // 32768
+constexpr uint32_t kKStageBytes = kSuper * kChunkBytes;            // 16384
 constexpr uint32_t kVStageBytes = 4 * kChunkBytes;                 // 32768
 constexpr uint32_t kPBytes = kRows * kTileKeys * 2;                // 16384
 constexpr int kPSlots = 5;                         // P page tiles in flight from the score CTA to the value CTA
-constexpr uint32_t kPTxBytes = kPBytes + kRows * 4 + 4 * 4;       // P tile + alpha column + 4 warp flags
+constexpr uint32_t kPWriters = 4;                 // softmax warps that write one P page (one per lane quadrant)
+constexpr uint32_t kPaWords = 36;                  // per writer warp: 32 row rescale factors, a flag word, padding
+constexpr uint32_t kStgBytes = 4096 + kPaWords * 4;                // score CTA: one warp's P rows + factors, staged
+constexpr uint32_t kPTxBytes = kPWriters * kStgBytes;              // bytes that fill one P slot
 constexpr uint32_t kQpeOff = 0;                                    // score CTA: Q rope part, [128 x 64] bf16
 constexpr uint32_t kKOff = kRows * 128;                            // score CTA: key stages
 constexpr uint32_t kPOff = kVStages * kVStageBytes;                // value CTA: P slots
-constexpr uint32_t kRegionA = kKOff + kKStages * kKStageBytes;     // 212992
+constexpr uint32_t kStgOff = kKOff + kKStages * kKStageBytes;      // score CTA: 8 warp staging buffers
+constexpr uint32_t kRegionA = (kStgOff + 8 * kStgBytes + 1023) & ~1023u;   // 214016
 static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
 #ifndef MLA_TC_PREFETCH_PAGES
 #define MLA_TC_PREFETCH_PAGES 0
@@ -77,13 +79,13 @@ constexpr int kTimeoutRecInts = 1 + 6 * 16;
 
 // TMEM columns
 constexpr uint32_t kQCol = 0;      // score CTA: latent part of Q, 256 columns (2 bf16 per column)
-constexpr uint32_t kSCol = 256;    // score CTA: S, 256 columns (one score tile)
+constexpr uint32_t kSCol = 256;    // score CTA: S, two buffers of 128 columns (one score tile each)
 // value CTA: O in columns 0..511
 
 // Barrier slots (same indices in both CTAs).
 enum Bar {
-  B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_SFULL = B_KEMPTY + kKStages, B_SEMPTY = B_SFULL + 1,
-  B_QREADY = B_SEMPTY + 1, B_PEMPTY = B_QREADY + 1, B_STATSEMPTY = B_PEMPTY + kPSlots,
+  B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_SFULL = B_KEMPTY + kKStages, B_SEMPTY = B_SFULL + 2,
+  B_QREADY = B_SEMPTY + 2, B_PEMPTY = B_QREADY + 1, B_STATSEMPTY = B_PEMPTY + kPSlots,
   B_VFULL = B_STATSEMPTY + 1, B_VEMPTY = B_VFULL + kVStages, B_PFULL = B_VEMPTY + kVStages,
   B_PVDONE = B_PFULL + kPSlots, B_REQ = B_PVDONE + kPSlots, B_REQDONE = B_REQ + 1, B_STATSFULL = B_REQDONE + 1,
   B_OFREE = B_STATSFULL + 1, B_COUNT = B_OFREE + 1
@@ -96,8 +98,9 @@ struct Req {
 };
 
 struct SmemB {                       // small region after the tiles
-  float alpha[kPSlots][kRows];       // value CTA: per-row rescale factor of each P slot
-  uint32_t flags[kPSlots][4];        // value CTA: per softmax warp, "some row of this tile rescaled"
+  // value CTA, per P slot and writer warp: the rescale factors of its 32 rows, then a flag word
+  // ("some row of this tile rescaled") and padding; filled by the score CTA's bulk copies.
+  float pa[kPSlots][kPWriters][kPaWords];
   float stat_l[kRows], stat_m[kRows];// value CTA: row sum and reference max of a finished unit
   float xmax[2][2][kRows];           // score CTA: the two softmax halves' tile maxima (double-buffered)
   float xl[2][kRows];                // score CTA: the two halves' row sums at the end of a unit
@@ -336,10 +339,10 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   if (threadIdx.x == 0) {
     uint32_t counts[B_COUNT];
     for (int i = 0; i < B_COUNT; ++i) counts[i] = 1;
-    counts[B_SEMPTY] = 8;                             // one per softmax warp
+    counts[B_SEMPTY] = counts[B_SEMPTY + 1] = 8;      // one per softmax warp
     counts[B_QREADY] = 8;
     counts[B_STATSEMPTY] = 4;                         // remote, one per value-CTA epilogue warp
-    // P full: one local arrival (the relay arms the expected bytes); the bytes arrive by st.async.
+    // P full: the relay's arrival, which also arms the bytes the four writer warps' bulk copies bring.
     counts[B_REQDONE] = kRows;
     counts[B_STATSFULL] = kRows;                      // remote, every softmax thread
     counts[B_OFREE] = kRows;
@@ -375,24 +378,18 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   int b, rb, t0, t1, segid, nseg;
   bool first_u;
 
-  // Register split: the launch gives every thread kLaunchRegs (checked on the host before launch);
-  // warpgroup 0 (producer, MMA issuer, relay) gives registers up to warpgroups 1-2 (softmax /
-  // epilogue).  128 * kLowRegs + 256 * kHighRegs == 384 * kLaunchRegs.
-  // Register split (warpgroup-uniform): the launch gives every thread kLaunchRegs (checked on the
-  // host); warpgroup 0 (producers, MMA issuers, relay) hands registers to warpgroups 1-2 (softmax
-  // and epilogue warps).  128 * kLowRegs + 256 * kHighRegs == 384 * kLaunchRegs.
+  // Every role runs with the launch's kLaunchRegs registers.  No setmaxnreg split: a producer or
+  // issuer squeezed into fewer registers spills, and with the shared-memory carve-out at its
+  // maximum, L1 is too small to hold the spills, so they cost L2 round trips per stage.
   if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (rank == 0) {
       if (warp == 0) {
-      // ---- key producer (whole warp: lookups in warp-wide batches, lane 0 issues): a score tile
-      // is up to 4 pages (256 keys), streamed as 9 stages of [256 keys x 64 dims] (8 latent chunks,
-      // then the RoPE key).  Pages further ahead are prefetched into L2 (a page is contiguous in a
-      // tiled pool and in a fused row pool), so the shared-memory stages wait on L2, not DRAM.
+      // ---- key producer (whole warp: page lookups in warp-wide batches; lane 0 issues): a score
+      // tile is up to 2 pages (128 keys), streamed as 9 stages of [128 keys x 64 dims] (8 latent
+      // chunks, then the RoPE key).  Optionally, pages further ahead are prefetched into L2.
       SegIter it = it0;
       PageRows pr;
       uint32_t n = 0;
-      uint32_t uses[kKStages] = {0, 0, 0, 0, 0, 0};
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         int pf = t0 + kSuper;   // next page to prefetch
         for (int T = t0; T < t1; T += kSuper) {
@@ -414,14 +411,22 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             if (p.tiled) prefetch_l2(p.tiled + (prow / kTileKeys) * (9 * kChunkBytes), 9 * kChunkBytes);
             else if (p.rows_contig) prefetch_l2(p.row_pool + prow * (int64_t)kW * 2, kTileKeys * kW * 2);
           }
-          for (int j = 0; j < 9; ++j, ++n) {
-            if (lane == 0) sb.prog[warp] = (int)n;
-            const int s = n % kKStages;
-            if (n >= kKStages && !warp_wait(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) goto prod_done0;
-            if (lane == 0) {
+          // Lane 0 streams the tile's 9 stages: a stage is chunk j of each page (8 KB each).
+          int ok = 1;
+          if (lane == 0) {
+            for (int j = 0; j < 9; ++j, ++n) {
+              sb.prog[warp] = (int)n;
+              const int s = n % kKStages;
+              if (n >= kKStages &&
+                  !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) {
+                ok = 0;
+                break;
+              }
               const uint32_t dst = smem_u32(tiles + kKOff + s * kKStageBytes);
               mbar_expect_tx(bar(B_KFULL + s), npg * kChunkBytes);
-              for (int pg = 0; pg < npg; ++pg) {
+#pragma unroll
+              for (int pg = 0; pg < kSuper; ++pg) {
+                if (pg >= npg) break;
                 if (p.tiled)   // chunk j of a page is 8 KB, already in the order the MMA reads it
                   bulk_load(dst + pg * kChunkBytes, p.tiled + (int64_t)(rows[pg] / kTileKeys) * (9 * kChunkBytes) + j * kChunkBytes,
                             kChunkBytes, bar(B_KFULL + s));
@@ -429,17 +434,21 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
                 else tma_load_2d(dst + pg * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
               }
             }
-            ++uses[s];
           }
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          n = __shfl_sync(0xffffffffu, n, 0);
+          if (!ok) goto prod_done0;
         }
       }
     prod_done0:
       // Drain: the last load issued on each stage must have landed before exit.
       if (lane == 0)
         for (int s = 0; s < kKStages; ++s)
-          if (uses[s]) mbar_wait(bar(B_KFULL + s), (uses[s] - 1) & 1, kWaitNs);
+          if (const uint32_t uses = n / kKStages + (s < (int)(n % kKStages) ? 1u : 0u))
+            mbar_wait(bar(B_KFULL + s), (uses - 1) & 1, kWaitNs);
       } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: S [128 x N] = Q . K^T, N = 64 * pages (256 for a full score tile).
+      // ---- MMA issuer: S [128 x N] = Q . K^T, N = 64 * pages (128 for a full score tile), into
+      // one of two tensor-memory buffers so that the next tile's MMAs overlap this tile's softmax.
       // The latent part of Q is the A operand from tensor memory; the RoPE part is in shared memory.
       SegIter it = it0;
       uint32_t n = 0, ns = 0, uc = 0;
@@ -450,7 +459,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         for (int T = t0; T < t1; T += kSuper, ++ns) {
           const int npg = min(kSuper, t1 - T);
           const uint32_t idesc = idesc_bf16_f32(kRows, kTileKeys * npg, false, false);
-          if (ns > 0 && !wait_or_abort(sb, bar(B_SEMPTY), (ns - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          const uint32_t sbuf = ns & 1, dcol = tbase + kSCol + 128 * sbuf;
+          if (ns >= 2 && !wait_or_abort(sb, bar(B_SEMPTY + sbuf), ((ns >> 1) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
           tc_fence_after();
           for (int j = 0; j < 9; ++j, ++n) {
             sb.prog[warp] = (int)n;
@@ -462,14 +472,14 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = smem_desc_sw128(kt + kk * 32, 16, 1024);
               if (j < 8)
-                mma_ts(tbase + kSCol, tbase + kQCol + 32 * j + 8 * kk, bd, idesc, (j | kk) ? 1u : 0u);
+                mma_ts(dcol, tbase + kQCol + 32 * j + 8 * kk, bd, idesc, (j | kk) ? 1u : 0u);
               else
-                mma_ss(tbase + kSCol, smem_desc_sw128(smem_u32(tiles + kQpeOff) + kk * 32, 16, 1024), bd, idesc, 1u);
+                mma_ss(dcol, smem_desc_sw128(smem_u32(tiles + kQpeOff) + kk * 32, 16, 1024), bd, idesc, 1u);
             }
             tc_commit(bar(B_KEMPTY + s));
           }
           if (!ok) break;
-          tc_commit(bar(B_SFULL));
+          tc_commit(bar(B_SFULL + sbuf));
         }
         ++uc;
       }
@@ -493,7 +503,6 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       SegIter it = it0;
       PageRows pr;
       uint32_t n = 0;
-      uint32_t uses[kVStages] = {0, 0, 0, 0};
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         if (first_u && lane == 0) {
           // This cluster holds the unit's first tile: publish where its partials live.
@@ -517,14 +526,14 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
                 for (int j = 0; j < 4; ++j)
                   tma_load_2d(dst + j * kChunkBytes, &map_c, 64 * (4 * h + j), (int32_t)row, bar(B_VFULL + s));
             }
-            ++uses[s];
           }
         }
       }
     prod_done1:
       if (lane == 0)
         for (int s = 0; s < kVStages; ++s)
-          if (uses[s]) mbar_wait(bar(B_VFULL + s), (uses[s] - 1) & 1, kWaitNs);
+          if (const uint32_t uses = n / kVStages + (s < (int)(n % kVStages) ? 1u : 0u))
+            mbar_wait(bar(B_VFULL + s), (uses - 1) & 1, kWaitNs);
       } else if (warp == 1 && lane == 0) {
       // ---- MMA issuer: O += P . C
       SegIter it = it0;
@@ -544,8 +553,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             break;
           }
           const bool tail = (t + 1) * kTileKeys > S;
-          const uint32_t *fl = sb.flags[pb];
-          const bool resc = t != t0 && (fl[0] | fl[1] | fl[2] | fl[3]) != 0;
+          const bool resc = t != t0 && (__float_as_uint(sb.pa[pb][0][32]) | __float_as_uint(sb.pa[pb][1][32]) |
+                                        __float_as_uint(sb.pa[pb][2][32]) | __float_as_uint(sb.pa[pb][3][32])) != 0;
           bool have_v = false;
           if (tail || resc) {
             // Rare: let the epilogue warps zero the rows past the end and/or rescale O first.
@@ -562,6 +571,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           }
           const uint32_t pt = smem_u32(tiles + kPOff + pb * kPBytes);
           // O[:, 256h .. 256h+255] += P . C[:, 256h ..]: one half-page stage per group of 4 MMAs.
+#pragma unroll
           for (int h = 0; h < 2; ++h) {
             if (!have_v && !wait_or_abort(sb, bar(B_VFULL + sv[h]), pv[h], p.dev_status, false, p.timeout_rec, __LINE__)) {
               ok = false;
@@ -590,8 +600,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       }
       } else if (warp == 2 && lane == 0) {
       // ---- relay: a P slot is free once the MMAs that read it completed
-      // Each slot's P-full phase is armed with the bytes the score CTA will send
-      // before that CTA may send them (initially, then when the slot frees up).
+      // Each slot's next P-full phase is armed with the bytes the score CTA will copy
+      // before that CTA may copy them (at start-up, then whenever the slot frees up).
       SegIter it = it0;
       uint32_t np = 0;
       const uint32_t pempty_remote = mapa(bar(B_PEMPTY), peer);
@@ -611,18 +621,17 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       }
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     if (rank == 0) {
       // ---- softmax: 8 warps; warp (quadrant q, half h) owns rows 32q..32q+31 (its TMEM lanes)
-      // and the score columns 128h..128h+127 of each score tile.
+      // and page h (score columns 64h..64h+63) of each two-page score tile.
       const int q4 = warp & 3, h = (warp - 4) >> 2;
       const int r = q4 * 32 + lane;
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
       SegIter it = it0;
       uint32_t ns = 0, np = 0, uc = 0;
       const uint32_t pbuf_remote = mapa(smem_u32(tiles + kPOff), peer);
-      const uint32_t alpha_remote = mapa(smem_u32(&sb.alpha[0][0]), peer);
-      const uint32_t flags_remote = mapa(smem_u32(&sb.flags[0][0]), peer);
+      const uint32_t pa_remote = mapa(smem_u32(&sb.pa[0][0][0]), peer);
+      unsigned char *stg = tiles + kStgOff + (warp - 4) * kStgBytes;   // this warp's staging buffer
       const uint32_t statl_remote = mapa(smem_u32(&sb.stat_l[0]), peer);
       const uint32_t statm_remote = mapa(smem_u32(&sb.stat_m[0]), peer);
       const uint32_t pfull_remote = mapa(bar(B_PFULL), peer);
@@ -667,26 +676,31 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         for (int T = t0; T < t1; T += kSuper, ++ns) {
           if (lane == 0) sb.prog[warp] = (int)np;
           const int npg = min(kSuper, t1 - T);
-          warp_wait(sb, bar(B_SFULL), ns & 1, p.dev_status, false, p.timeout_rec, __LINE__);
+          const uint32_t sbuf = ns & 1;
+          warp_wait(sb, bar(B_SFULL + sbuf), (ns >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__);
           tc_fence_after();
-          uint32_t sc[128];
+          // My page of the tile is page h: keys 64T + 64h + k, k < 64.  The scores come into
+          // registers and the buffer is released at once for the tile after next.
+          uint32_t sc[64];
+          {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tbase + lane_off + kSCol + 128 * sbuf + 64 * h, v0);
+            tmem_ld32(tbase + lane_off + kSCol + 128 * sbuf + 64 * h + 32, v1);
+            tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tbase + lane_off + kSCol + 128 * h + 32 * c, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sc[32 * c + i] = v[i];
+            for (int i = 0; i < 32; ++i) {
+              sc[i] = v0[i];
+              sc[32 + i] = v1[i];
+            }
           }
-          tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_SEMPTY));
-          // Keys of my columns: 64T + 128h + k; valid while below the row's causal limit and
-          // inside the pages this score tile holds.
-          const int nvalid = min(visible - (T * kTileKeys + 128 * h), npg * kTileKeys - 128 * h);
+          if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
+          // Valid while below the row's causal limit and inside the pages this tile holds.
+          const int nvalid = min(visible - (T + h) * kTileKeys, (npg - h) * kTileKeys);
           float mx = -CUDART_INF_F;
 #pragma unroll
-          for (int k = 0; k < 128; ++k)
+          for (int k = 0; k < 64; ++k)
             if (k < nvalid) mx = fmaxf(mx, __uint_as_float(sc[k]) * p.scale_log2);
           sb.xmax[ns & 1][h][r] = mx;
           asm volatile("bar.sync 1, 256;" ::: "memory");
@@ -698,37 +712,48 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             l *= alpha;
             m_ref = mx;
           }
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int g = 2 * h + i;              // page of this score tile
-            if (g >= npg) break;
-            const uint32_t pn = np + g;
+          if (h < npg) {
+            const uint32_t pn = np + h;
             const int pb = pn % kPSlots;
-            if (pn >= kPSlots) warp_wait(sb, bar(B_PEMPTY + pb), ((pn / kPSlots) - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__);
-            // P rows -> value CTA, K-major 128B-swizzled [128 rows x 64 keys] tile, by asynchronous
-            // remote stores that complete on the value CTA's P-full barrier (armed by its relay),
-            // 8 keys (16 bytes) at a time.  The first page of a score tile also carries the tile's
-            // O rescale factors.
-            const uint32_t pfull = pfull_remote + 8 * pb;
-            const uint32_t rowbase = pbuf_remote + pb * kPBytes + (r >> 3) * 1024 + (r & 7) * 128;
+            // The staging buffer is free once this warp's previous bulk copies have read it.
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+            // My 32 P rows, K-major and 128B-swizzled like the value CTA's [128 x 64] P tile (rows
+            // 32q..32q+31 are its bytes 4096q..4096q+4095), then the rows' rescale factors (the first
+            // page of a score tile carries the tile's factors) and the warp's flag word.
+            unsigned char *prow = stg + (lane >> 3) * 1024 + (lane & 7) * 128;
             float psum = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
               uint32_t pk[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                const int kk = 64 * i + 8 * c + 2 * e;
+                const int kk = 8 * c + 2 * e;
                 const float p0 = (kk < nvalid) ? exp2f(__uint_as_float(sc[kk]) * p.scale_log2 - m_ref) : 0.f;
                 const float p1 = (kk + 1 < nvalid) ? exp2f(__uint_as_float(sc[kk + 1]) * p.scale_log2 - m_ref) : 0.f;
                 pk[e] = pack_bf16x2(p0, p1);
                 psum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
               }
-              st_async_v4(rowbase + ((c ^ (r & 7)) << 4), pk[0], pk[1], pk[2], pk[3], pfull);
+              *reinterpret_cast<uint4 *>(prow + ((c ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             l += psum;
-            st_async_b32(alpha_remote + (pb * kRows + r) * 4, __float_as_uint(g == 0 ? alpha : 1.f), pfull);
-            const unsigned moved = __ballot_sync(0xffffffffu, need && g == 0 && T != t0);
-            if (lane == 0) st_async_b32(flags_remote + (pb * 4 + q4) * 4, moved ? 1u : 0u, pfull);
+            reinterpret_cast<float *>(stg + 4096)[lane] = h == 0 ? alpha : 1.f;
+            const unsigned moved = __ballot_sync(0xffffffffu, need && h == 0 && T != t0);
+            if (lane < 4) reinterpret_cast<uint32_t *>(stg + 4096 + 128)[lane] = (lane == 0 && moved) ? 1u : 0u;
+            fence_proxy_async_smem();
+            __syncwarp();
+            // Into the value CTA's slot once the MMAs that read its previous contents completed: two
+            // bulk copies that complete on the slot's P-full barrier (armed by the relay).
+            if (pn < kPSlots ||
+                warp_wait(sb, bar(B_PEMPTY + pb), ((pn / kPSlots) - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
+              if (lane == 0) {
+                const uint32_t pfull = pfull_remote + 8 * pb;
+                bulk_copy_to_peer(pbuf_remote + pb * kPBytes + 4096 * q4, smem_u32(stg), 4096, pfull);
+                bulk_copy_to_peer(pa_remote + (pb * kPWriters + q4) * (kPaWords * 4), smem_u32(stg + 4096),
+                                  kPaWords * 4, pfull);
+                bulk_commit();
+              }
+            }
           }
           np += npg;
         }
@@ -745,6 +770,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         asm volatile("bar.sync 1, 256;" ::: "memory");   // xl may be reused by the next unit
         ++uc;
       }
+      if (lane == 0) bulk_wait_all();   // the staged copies have landed before this CTA may exit
     } else if (warp < 8) {
       // ---- epilogue warps: tile fix-ups on request, then each unit's epilogue
       const int r = (warp - 4) * 32 + lane;
@@ -772,7 +798,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             }
             if (q.rescale) {
               tc_fence_after();
-              const float a = sb.alpha[q.slot][r];
+              const float a = sb.pa[q.slot][r >> 5][r & 31];
 #pragma unroll 1
               for (int c = 0; c < 16; ++c) {
                 uint32_t v[32];
@@ -1072,9 +1098,9 @@ int clusters_for_device() {
   if (cached[dev]) return cached[dev];
   if (cudaFuncSetAttribute(mla_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes))
     return 0;
-  // The in-kernel register split assumes exactly kLaunchRegs per thread; never launch otherwise.
+  // One CTA of kThreads per SM needs at most kLaunchRegs registers per thread.
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, mla_decode_tc_kernel) != cudaSuccess || fa.numRegs != kLaunchRegs) return 0;
+  if (cudaFuncGetAttributes(&fa, mla_decode_tc_kernel) != cudaSuccess || fa.numRegs > kLaunchRegs) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * kMaxClusters);
   cfg.blockDim = dim3(kThreads);
