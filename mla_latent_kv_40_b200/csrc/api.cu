@@ -104,6 +104,13 @@ int combine_impl(const mla_dims *dims, int B, int n_q, const int32_t *seqlens, i
   return launch_combine(cb, bf16, st);
 }
 
+// Query absorption: tcgen05 where the shape and alignment allow, else warp MMAs, else CUDA cores.
+int absorb_dispatch(const AbsorbArgs &ab, bool bf16, int *dev_status, cudaStream_t st) {
+  if (absorb_tc_supported(ab, bf16)) return launch_absorb_tc(ab, dev_status, st);
+  if (absorb_mma_supported(ab, bf16)) return launch_absorb_mma(ab, st);
+  return launch_absorb(ab, bf16, st);
+}
+
 int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
                 const void *c_kv, const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
                 int num_blocks, const int32_t *seqlens, int max_seqlen, const void *w_uk,
@@ -118,9 +125,7 @@ int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const 
   void *qbuf = ws + L.q_off;
   AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
                 q_nope, q_pe, w_uk, seqlens, qbuf, dims->rope_base};
-  if ((rc = absorb_mma_supported(ab, dims->dtype == MLA_BF16) ? launch_absorb_mma(ab, st)
-                                                               : launch_absorb(ab, dims->dtype == MLA_BF16, st)))
-    return rc;
+  if ((rc = absorb_dispatch(ab, dims->dtype == MLA_BF16, dev_status, st))) return rc;
   if ((rc = attention_impl(dims, B, n_q, qbuf, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
                            max_seqlen, L, ws, dev_status, st)))
     return rc;
@@ -179,9 +184,15 @@ int mla_append_latent(const mla_dims *dims, int T, const void *h, const void *w_
                                    num_seqs, max_blocks_per_seq, num_blocks, dev_status);
   const bool bf16 = dims->dtype == MLA_BF16;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int nsplit = 1, kps = dims->d_model;
   if (workspace && append_mma_supported(a, bf16) && !(reinterpret_cast<uintptr_t>(workspace) & 15) &&
-      ws_bytes >= append_mma_workspace(T, dims->d_model, dims->d_c + dims->d_rope, nullptr, nullptr))
+      ws_bytes >= append_mma_workspace(T, dims->d_model, dims->d_c + dims->d_rope, &nsplit, &kps)) {
+    if (append_tc_supported(a, bf16)) {
+      const int rc = launch_append_tc(a, workspace, nsplit, kps, st);
+      return rc ? rc : launch_append_finish(a, workspace, nsplit, st);
+    }
     return launch_append_mma(a, workspace, st);
+  }
   return launch_append(a, bf16, st);
 }
 
@@ -192,8 +203,7 @@ int mla_absorb_q(const mla_dims *dims, int B, int n_q, const void *q_nope, const
   AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
                 q_nope, q_pe, w_uk, seqlens, q_out, dims->rope_base};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  return absorb_mma_supported(ab, dims->dtype == MLA_BF16) ? launch_absorb_mma(ab, st)
-                                                           : launch_absorb(ab, dims->dtype == MLA_BF16, st);
+  return absorb_dispatch(ab, dims->dtype == MLA_BF16, nullptr, st);
 }
 
 int mla_decode_workspace_size(const mla_dims *dims, int B, int n_q, int max_seqlen, size_t *bytes) {

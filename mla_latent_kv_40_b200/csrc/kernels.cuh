@@ -90,6 +90,13 @@ bool append_mma_supported(const AppendArgs &a, bool bf16);
 int launch_append_mma(const AppendArgs &a, void *ws, cudaStream_t st);
 bool absorb_mma_supported(const AbsorbArgs &a, bool bf16);
 int launch_absorb_mma(const AbsorbArgs &a, cudaStream_t st);
+// tcgen05 versions (TMA-fed, weights on the M side); the append one writes the same partials
+// as launch_append_mma and leaves them to its finish kernel.
+bool absorb_tc_supported(const AbsorbArgs &a, bool bf16);
+int launch_absorb_tc(const AbsorbArgs &a, int *dev_status, cudaStream_t st);
+bool append_tc_supported(const AppendArgs &a, bool bf16);
+int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split, cudaStream_t st);
+int launch_append_finish(const AppendArgs &a, const void *ws, int nsplit, cudaStream_t st);
 int launch_cache_convert(const void *src, void *dst, int64_t num_rows, int W, bool to_tiled, cudaStream_t st);
 
 }  // namespace mla

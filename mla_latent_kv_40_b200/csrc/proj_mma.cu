@@ -194,7 +194,12 @@ int launch_append_mma(const AppendArgs &a, void *ws, cudaStream_t st) {
                                            static_cast<const __nv_bfloat16 *>(a.w_dkv),
                                            static_cast<const __nv_bfloat16 *>(a.w_kr), a.T, a.d_model, a.d_c,
                                            a.d_rope, kps, part);
-  append_finish_kernel<<<a.T, kFinThreads, 0, st>>>(a, part, nsplit);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  return launch_append_finish(a, part, nsplit, st);
+}
+
+int launch_append_finish(const AppendArgs &a, const void *ws, int nsplit, cudaStream_t st) {
+  append_finish_kernel<<<a.T, kFinThreads, 0, st>>>(a, static_cast<const float *>(ws), nsplit);
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 

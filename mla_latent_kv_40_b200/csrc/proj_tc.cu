@@ -1,0 +1,319 @@
+// bf16 projections around the attention kernel on 5th-generation tensor cores.
+//
+//  * query absorption, q_lat^(s) = q_nope^(s) W_UK^(s)T per head, plus the RoPE
+//    of q_pe ("Transformer升级之路：21、MLA好在哪里?（下）", section 双重投影,
+//    decoding column);
+//  * append down-projection [h W_DKV | h W_KR] over a K-split, reduced and
+//    finished (RMSNorm, RoPE, scatter) by the append finish kernel
+//    ("DeepSeek-V3 解读 1: MLA", sections "MLA：高层次的思路" and
+//    "为什么需要解耦 RoPE").
+//
+// Both are weight-streaming GEMMs with few activation rows, so they run
+// transposed: the weight supplies the 128-row M side of a tcgen05 MMA (read
+// once, by TMA), the activation rows are the N side (N = 64 per CTA), and the
+// fp32 accumulator sits in 64 tensor-memory columns.  One elected thread
+// issues the TMA loads and the MMAs; all warps drain tensor memory.
+#include "kernels.cuh"
+#include "sm100.cuh"
+#include "tmap.cuh"
+
+namespace mla {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kTcThreads = 128;
+constexpr int kTcN = 64;                      // activation rows (tokens / query rows) per CTA
+constexpr uint32_t kAChunk = 128 * 128;       // [128 rows x 64 K] bf16, 128B-swizzled: 16 KB
+constexpr uint32_t kBChunk = kTcN * 128;      // [64 rows x 64 K] bf16: 8 KB
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+// Bounded wait: on expiry report a timeout and let the caller skip its work.
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int *dev_status) {
+  if (mbar_wait(bar, parity, kWaitNs)) return true;
+  report(dev_status, MLA_ERR_TIMEOUT);
+  return false;
+}
+
+// ------------------------------------------------------------------ absorb
+// CTA = (head s, 128 latent columns m0.., 64 query rows r0..):
+//   D[m][r] = sum_k W_UK[s][m0 + m][k] q_nope[r0 + r][s][k]   (A and B both K-major)
+// The CTAs with blockIdx.y == 0 .. 3 share the RoPE of their 64 rows.
+__global__ void __launch_bounds__(kTcThreads)
+absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_q, AbsorbArgs a,
+                 int *dev_status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_full, bar_mma;
+  __shared__ uint32_t tmem_slot;
+  const int nkc = a.d_nope / 64;
+  unsigned char *As = sm;                                  // [nkc][128 x 128 B]
+  unsigned char *Bs = As + nkc * kAChunk;                  // [nkc][64 x 128 B]
+  __nv_bfloat16 *Os = reinterpret_cast<__nv_bfloat16 *>(Bs + nkc * kBChunk);   // [64][128 + 8]
+  constexpr int ldo = 128 + 8;
+  const int s = blockIdx.x, m0 = blockIdx.y * 128, r0 = blockIdx.z * kTcN;
+  const int R = a.B * a.n_q, W = a.d_c + a.d_rope;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    mbar_init(smem_u32(&bar_full), 1);
+    mbar_init(smem_u32(&bar_mma), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), kTcN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (tid == 0) {
+    tma_prefetch_desc(&map_w);
+    tma_prefetch_desc(&map_q);
+    mbar_expect_tx(smem_u32(&bar_full), nkc * (kAChunk + kBChunk));
+    for (int kc = 0; kc < nkc; ++kc) {
+      tma_load_2d(smem_u32(As + kc * kAChunk), &map_w, 64 * kc, s * a.d_c + m0, smem_u32(&bar_full));
+      tma_load_2d(smem_u32(Bs + kc * kBChunk), &map_q, s * a.d_nope + 64 * kc, r0, smem_u32(&bar_full));
+    }
+  }
+
+  // RoPE of q_pe by warps 1-3 while the tiles stream in (thread 0 goes straight on to the MMAs):
+  // rows r0 + y, y + gridDim.y, ... of this CTA; a warp takes whole rows, a lane one (x, y) pair,
+  // and every row's loads are issued before any of its arithmetic.
+  if (warp > 0) {
+    __shared__ double theta[32];                           // pair frequencies, once per CTA
+    const __nv_bfloat16 *qp = static_cast<const __nv_bfloat16 *>(a.q_pe);
+    __nv_bfloat16 *qo = static_cast<__nv_bfloat16 *>(a.q_out);
+    const int half = a.d_rope / 2;
+    if (tid - 32 < half) theta[tid - 32] = rope_theta(tid - 32, a.d_rope, a.rope_base);
+    asm volatile("bar.sync 1, 96;" ::: "memory");       // warps 1-3 only
+    constexpr int kRowsPerWarp = 8;
+    const int nr = (kTcN - (int)blockIdx.y + (int)gridDim.y - 1) / (int)gridDim.y;
+    for (int w0 = (warp - 1) * kRowsPerWarp; w0 < nr; w0 += 3 * kRowsPerWarp) {
+      int pos[kRowsPerWarp];
+      __nv_bfloat162 xy[kRowsPerWarp];
+#pragma unroll
+      for (int k = 0; k < kRowsPerWarp; ++k) {
+        const int gr = r0 + blockIdx.y + gridDim.y * (w0 + k);
+        const bool live = w0 + k < nr && gr < R && lane < half;
+        pos[k] = live ? max(0, a.seqlens[gr / a.n_q] - a.n_q + gr % a.n_q) : -1;   // -1: nothing to do
+        xy[k] = live ? *reinterpret_cast<const __nv_bfloat162 *>(qp + ((int64_t)gr * a.H + s) * a.d_rope + 2 * lane)
+                     : __floats2bfloat162_rn(0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < kRowsPerWarp; ++k) {
+        if (pos[k] < 0) continue;
+        const int gr = r0 + blockIdx.y + gridDim.y * (w0 + k);
+        float cs, sn;
+        rope_cos_sin_theta(pos[k], theta[lane], &cs, &sn);
+        const float x = __low2float(xy[k]), y = __high2float(xy[k]);
+        *reinterpret_cast<__nv_bfloat162 *>(qo + ((int64_t)gr * a.H + s) * W + a.d_c + 2 * lane) =
+            __floats2bfloat162_rn(x * cs - y * sn, x * sn + y * cs);
+      }
+    }
+  }
+
+  int ok = 1;
+  if (tid == 0) {
+    ok = wait_bar(smem_u32(&bar_full), 0, dev_status) ? 1 : 0;
+    if (ok) {
+      tc_fence_after();
+      const uint32_t idesc = idesc_bf16_f32(128, kTcN, false, false);
+      for (int kc = 0; kc < nkc; ++kc)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem, smem_desc_sw128(smem_u32(As + kc * kAChunk) + kk * 32, 16, 1024),
+                 smem_desc_sw128(smem_u32(Bs + kc * kBChunk) + kk * 32, 16, 1024), idesc, (kc | kk) ? 1u : 0u);
+      tc_commit(smem_u32(&bar_mma));
+    }
+  }
+  ok = __syncthreads_and(ok);
+  if (ok && lane == 0) ok = wait_bar(smem_u32(&bar_mma), 0, dev_status) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_wait(smem_u32(&bar_mma), 0, kWaitNs);
+  tc_fence_after();
+  // Warp w drains latent rows 32w..32w+31 (its lane quadrant): thread = one latent column m,
+  // 64 query rows -> the staging tile, transposed to [query row][m].
+  {
+    uint32_t v[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * h, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Os[(32 * h + i) * ldo + warp * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (ok) {
+    __nv_bfloat16 *qo = static_cast<__nv_bfloat16 *>(a.q_out);
+    for (int c = tid; c < kTcN * 16; c += kTcThreads) {
+      const int r = c >> 4, q8 = c & 15, gr = r0 + r;
+      if (gr < R)
+        *reinterpret_cast<uint4 *>(qo + ((int64_t)gr * a.H + s) * W + m0 + q8 * 8) =
+            *reinterpret_cast<const uint4 *>(Os + r * ldo + q8 * 8);
+    }
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTcN);
+  }
+}
+
+// ------------------------------------------------------------------ append projection
+// CTA = (128 output columns m0.. of [W_DKV | W_KR], K-split ks, 64 tokens t0..):
+//   D[m][t] = sum_{k in split} W[k][m0 + m] h[t0 + t][k]     (A = W^T is M-major, B = h is K-major)
+// Stages of 64 K rows stream through a ring; the partial goes to part[ks][t][m] (fp32).
+constexpr int kApStages = 4;
+constexpr uint32_t kApStageBytes = kAChunk + kBChunk;      // A: 2 M-chunks of [64 K x 128 B]; B: [64 x 128 B]
+
+__global__ void __launch_bounds__(kTcThreads)
+append_tc_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_constant__ CUtensorMap map_wr,
+                 const __grid_constant__ CUtensorMap map_h, int T, int d_c, int d_rope, int k_per_split, int D,
+                 float *part, int *dev_status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bar_full[kApStages], bar_empty[kApStages], bar_mma;
+  __shared__ uint32_t tmem_slot;
+  const int W = d_c + d_rope;
+  const int m0 = blockIdx.x * 128, ks = blockIdx.y, t0 = blockIdx.z * kTcN;
+  const int kbeg = ks * k_per_split, kend = min(D, kbeg + k_per_split);
+  const int nst = (kend - kbeg + 63) / 64;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool rope_tile = m0 >= d_c;
+
+  if (tid == 0) {
+    for (int i = 0; i < kApStages; ++i) {
+      mbar_init(smem_u32(&bar_full[i]), 1);
+      mbar_init(smem_u32(&bar_empty[i]), 1);
+    }
+    mbar_init(smem_u32(&bar_mma), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), kTcN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  int ok = 1;
+  if (tid == 0) {
+    // Producer: stage i = K rows kbeg + 64i ..; the weight chunk c holds output columns m0 + 64c ..
+    // (the RoPE tile reads W_KR, whose second chunk lies outside it and arrives as zeros).
+    const CUtensorMap *mw = rope_tile ? &map_wr : &map_wd;
+    const int mx = rope_tile ? m0 - d_c : m0;
+    tma_prefetch_desc(mw);
+    tma_prefetch_desc(&map_h);
+    for (int i = 0; i < nst; ++i) {
+      const int st = i % kApStages;
+      if (i >= kApStages && !wait_bar(smem_u32(&bar_empty[st]), ((i / kApStages) - 1) & 1, dev_status)) { ok = 0; break; }
+      unsigned char *base = sm + st * kApStageBytes;
+      const int k0 = kbeg + 64 * i;
+      mbar_expect_tx(smem_u32(&bar_full[st]), kApStageBytes);
+      tma_load_2d(smem_u32(base), mw, mx, k0, smem_u32(&bar_full[st]));
+      tma_load_2d(smem_u32(base + kAChunk / 2), mw, mx + 64, k0, smem_u32(&bar_full[st]));
+      tma_load_2d(smem_u32(base + kAChunk), &map_h, k0, t0, smem_u32(&bar_full[st]));
+    }
+  } else if (tid == 32) {
+    // MMA issuer.
+    const uint32_t idesc = idesc_bf16_f32(128, kTcN, true, false);
+    for (int i = 0; i < nst; ++i) {
+      const int st = i % kApStages;
+      if (!wait_bar(smem_u32(&bar_full[st]), (i / kApStages) & 1, dev_status)) { ok = 0; break; }
+      tc_fence_after();
+      const uint32_t a = smem_u32(sm + st * kApStageBytes), b = a + kAChunk;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem, smem_desc_sw128(a + kk * 2048, kAChunk / 2, 1024), smem_desc_sw128(b + kk * 32, 16, 1024), idesc,
+               (i | kk) ? 1u : 0u);
+      tc_commit(smem_u32(&bar_empty[st]));
+    }
+    tc_commit(smem_u32(&bar_mma));
+  }
+  ok = __syncthreads_and(ok);
+  if (ok && lane == 0) ok = wait_bar(smem_u32(&bar_mma), 0, dev_status) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_wait(smem_u32(&bar_mma), 0, kWaitNs);
+  tc_fence_after();
+  // Thread = output column m0 + 32w + lane; for each token its value goes to part[ks][t][m]:
+  // consecutive lanes write consecutive columns.
+  {
+    const int m = m0 + warp * 32 + lane;
+    float *dst = part + ((int64_t)ks * T) * W + m;
+    uint32_t v[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 32 * h, v);
+      tmem_wait_ld();
+      if (ok && m < W)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int t = t0 + 32 * h + i;
+          if (t < T) dst[(int64_t)t * W] = __uint_as_float(v[i]);
+        }
+    }
+  }
+  // Every issued load has landed (the MMA consumed it) before the CTA may leave.
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTcN);
+  }
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host side
+bool absorb_tc_supported(const AbsorbArgs &a, bool bf16) {
+  return bf16 && a.d_nope % 64 == 0 && a.d_nope <= 256 && a.d_c % 128 == 0 && a.d_rope <= 64 && a.d_rope % 2 == 0 &&
+         !(reinterpret_cast<uintptr_t>(a.q_nope) & 15) && !(reinterpret_cast<uintptr_t>(a.w_uk) & 15) &&
+         !(reinterpret_cast<uintptr_t>(a.q_pe) & 3) && !(reinterpret_cast<uintptr_t>(a.q_out) & 15) &&
+         ((a.d_c + a.d_rope) % 8) == 0;
+}
+
+int launch_absorb_tc(const AbsorbArgs &a, int *dev_status, cudaStream_t st) {
+  const int R = a.B * a.n_q;
+  CUtensorMap mw, mq;
+  if (!make_tmap_bf16(&mw, a.w_uk, a.d_nope, (uint64_t)a.H * a.d_c, (uint64_t)a.d_nope * 2, 128) ||
+      !make_tmap_bf16(&mq, a.q_nope, (uint64_t)a.H * a.d_nope, R, (uint64_t)a.H * a.d_nope * 2, kTcN))
+    return MLA_ERR_CUDA;
+  const int nkc = a.d_nope / 64;
+  const size_t smem = 1024 + nkc * (kAChunk + kBChunk) + sizeof(__nv_bfloat16) * kTcN * (128 + 8);
+  if (cudaFuncSetAttribute(absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+    return MLA_ERR_CUDA;
+  const dim3 grid(a.H, a.d_c / 128, (R + kTcN - 1) / kTcN);
+  absorb_tc_kernel<<<grid, kTcThreads, smem, st>>>(mw, mq, a, dev_status);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+bool append_tc_supported(const AppendArgs &a, bool bf16) {
+  return bf16 && a.d_model % 64 == 0 && a.d_c % 128 == 0 && a.d_rope <= 128 && a.d_rope % 8 == 0 &&
+         !(reinterpret_cast<uintptr_t>(a.h) & 15) && !(reinterpret_cast<uintptr_t>(a.w_dkv) & 15) &&
+         !(reinterpret_cast<uintptr_t>(a.w_kr) & 15);
+}
+
+int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split, cudaStream_t st) {
+  const int W = a.d_c + a.d_rope;
+  CUtensorMap mwd, mwr, mh;
+  if (!make_tmap_bf16(&mwd, a.w_dkv, a.d_c, a.d_model, (uint64_t)a.d_c * 2, 64) ||
+      !make_tmap_bf16(&mwr, a.w_kr, a.d_rope, a.d_model, (uint64_t)a.d_rope * 2, 64) ||
+      !make_tmap_bf16(&mh, a.h, a.d_model, a.T, (uint64_t)a.d_model * 2, kTcN))
+    return MLA_ERR_CUDA;
+  const size_t smem = 1024 + kApStages * kApStageBytes;
+  if (cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+    return MLA_ERR_CUDA;
+  const dim3 grid((W + 127) / 128, nsplit, (a.T + kTcN - 1) / kTcN);
+  append_tc_kernel<<<grid, kTcThreads, smem, st>>>(mwd, mwr, mh, a.T, a.d_c, a.d_rope, k_per_split, a.d_model,
+                                                   static_cast<float *>(ws), a.dev_status);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+}  // namespace mla
