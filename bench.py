@@ -112,21 +112,28 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def _traffic_for(kernel_file):
-    """dram bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+# Sources an attention kernel's DRAM traffic depends on; a recorded figure holds only while they are unchanged.
+_TRAFFIC_SOURCES = {"decode_tc.cu": ("decode_tc.cu", "decode_tc.cuh", "sm100.cuh", "common.cuh", "kernels.cuh"),
+                    "attn_simt.cu": ("attn_simt.cu", "common.cuh", "kernels.cuh")}
+
+
+def traffic_source_hash(kernel_file):
     import hashlib
+    h = hashlib.sha256()
+    for f in _TRAFFIC_SOURCES[kernel_file]:
+        h.update(open(os.path.join(ROOT, "mla_latent_kv_40_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_for(kernel_file):
+    """dram bytes per launch from the committed ncu summary, if the kernel's sources are unchanged since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    j = json.load(open(path))
-    ent = j.get(os.path.basename(kernel_file))
-    if not ent:
+    ent = json.load(open(path)).get(kernel_file)
+    if not ent or ent.get("source_sha256_16") != traffic_source_hash(kernel_file):
         return None
-    src = os.path.join(ROOT, "mla_latent_kv_40_b200", "csrc", os.path.basename(kernel_file))
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    if h != ent.get("source_sha256_16"):
-        return None
-    return ent.get("dram_bytes_per_full_launch")
+    return ent.get("dram_bytes_per_launch")
 
 
 def cpu_baseline(case, target_s=12.0, inp=None):
@@ -159,8 +166,29 @@ def cpu_baseline(case, target_s=12.0, inp=None):
                       f"form, FLOPs counted as absorbed-form work; {el:.1f} s"}
 
 
+def rank_info():
+    """(rank, world size, local rank) of this process, as torchrun sets them (1 process by default)."""
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks_of(x, world, device):
+    """The largest x over all ranks (one all-reduce); x itself on a single process."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(step_flops_per_rank, world, ms_max):
+    """Whole-job TFLOP/s: every rank does one step of the same work; the slowest rank sets the time."""
+    return step_flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    rank, _, _ = rank_info()
     if rank != 0:
         return
     from workloads import DECODE_CASES, make_decode_inputs
@@ -186,9 +214,7 @@ def run_reference(args):
 def run_mla(args):
     import torch
     import torch.distributed as dist
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_info()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -227,14 +253,22 @@ def run_mla(args):
     app_ws_bytes = mla.mla_append_workspace_size(dims, T)
     app_ws = mla.alloc_workspace(app_ws_bytes) if app_ws_bytes else None
 
+    # The append (cache write of the new tokens) and the query absorption are independent: the
+    # append runs on a side stream, and the attention, which reads the new tokens, waits for it.
+    side = torch.cuda.Stream()
+    appended = torch.cuda.Event()
+
     def append():
+        side.wait_stream(stream)   # after everything already queued (the previous step's readers)
         mla.mla_append_latent(dims, dev["h_new"], dev["w_dkv"], dev["w_kr"], dev["gamma"], dev["seq_idx"],
                               dev["pos"], c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status,
-                              workspace=app_ws)
+                              workspace=app_ws, stream=side)
+        appended.record(side)
 
     def step(ev=None):
         append()
         mla.mla_absorb_q(dims, dev["q_nope"], dev["q_pe"], dev["w_uk"], dev["seqlens"], q_abs)
+        stream.wait_event(appended)
         if ev is not None:
             ev[0].record(stream)
         mla.mla_decode_attention(dims, q_abs, c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
@@ -254,11 +288,7 @@ def run_mla(args):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(x, world, "cuda")
 
     att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -287,9 +317,11 @@ def run_mla(args):
             for k, t in host_in.items():
                 dev[k].copy_(t, non_blocking=True)
             append()
-            mla.mla_decode(dims, dev["q_nope"], dev["q_pe"], c_kv, k_pe, bt, inp["max_blocks_per_seq"],
-                           inp["num_blocks"], dev["seqlens"], max_seqlen, dev["w_uk"], dev["w_uv"], out, lse, ws,
-                           status)
+            mla.mla_absorb_q(dims, dev["q_nope"], dev["q_pe"], dev["w_uk"], dev["seqlens"], q_abs)
+            stream.wait_event(appended)
+            mla.mla_decode_attention(dims, q_abs, c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
+                                     dev["seqlens"], max_seqlen, ws, status)
+            mla.mla_decode_combine(dims, B, n_q, dev["seqlens"], max_seqlen, dev["w_uv"], out, lse, ws)
             host_out.copy_(out, non_blocking=True)
 
         for _ in range(3):
@@ -313,7 +345,7 @@ def run_mla(args):
     step_flops = fl["total"] + append_flops(d, T)
     lat_bytes = latent_bytes(d, inp["seqlens"].tolist())
     peaks = _peaks()
-    value = step_flops * world / (ms * 1e-3) / 1e12
+    value = weak_scaling_value(step_flops, world, ms)
     att_gbs = lat_bytes / (att_ms * 1e-3) / 1e9
     # append (projection + finish with a workspace, one fused kernel without), then absorb + attention + combine
     launches_per_step = (2 if app_ws is not None else 1) + mla.mla_decode_launches(dims, n_q)

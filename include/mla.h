@@ -284,6 +284,21 @@ MLA_API int mla_cache_pack(const mla_dims *dims, const void *rows, void *tiled, 
 MLA_API int mla_cache_unpack(const mla_dims *dims, const void *tiled, void *rows, int64_t num_rows,
                              mla_stream_t stream);
 
+/*
+ * mla_wait_selftest — exercise the bounded device wait used by every
+ *   tensor-core kernel of this library.  One thread waits on a barrier that
+ *   nothing completes; after limit_ns nanoseconds of device time
+ *   (globaltimer) it gives up, writes MLA_ERR_TIMEOUT into *dev_status (if it
+ *   still holds MLA_OK) and exits normally.  It causes no fault and leaves
+ *   the context usable.  This is a diagnostic with no counterpart on the
+ *   pages.
+ *   limit_ns: 1 .. 10^10.  dev_status: device int, required.
+ *   Returns MLA_ERR_INVALID_ARG for a bad limit or a NULL status, MLA_ERR_CUDA
+ *   if the launch fails, else MLA_OK (asynchronous; read *dev_status after a
+ *   synchronisation).
+ */
+MLA_API int mla_wait_selftest(long long limit_ns, int *dev_status, mla_stream_t stream);
+
 /* Human-readable text of an mla_status value (static storage). */
 MLA_API const char *mla_status_string(int status);
 

@@ -69,6 +69,7 @@ _sigs = {
     "mla_cache_unpack": [_D, _P, _P, ctypes.c_int64, _P],
     "mla_decode_noalloc": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P],
     "mla_prefill": [_D, _I, _P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P, _P],
+    "mla_wait_selftest": [ctypes.c_longlong, _P, _P],
 }
 for _n, _a in _sigs.items():
     getattr(_lib, _n).argtypes = _a
@@ -284,6 +285,12 @@ def mla_cache_unpack(dims, tiled, rows, stream=None):
     _check("mla_cache_unpack", _lib.mla_cache_unpack(ctypes.byref(dims), _ptr(tiled, torch.bfloat16, "tiled"),
                                                      _ptr(rows, torch.bfloat16, "rows"), int(rows.shape[0]),
                                                      _stream(stream)))
+
+
+def mla_wait_selftest(limit_ns, dev_status, stream=None):
+    """Bounded device wait on a barrier nothing completes: *dev_status becomes MLA_ERR_TIMEOUT."""
+    _check("mla_wait_selftest", _lib.mla_wait_selftest(int(limit_ns), _ptr(dev_status, torch.int32, "dev_status"),
+                                                       _stream(stream)))
 
 
 def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
