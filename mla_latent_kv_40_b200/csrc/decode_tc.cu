@@ -333,8 +333,10 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   auto bar = [&](int i) { return smem_u32(&sb.bars[i]); };
   const uint32_t peer = rank ^ 1u;
 
-  if (threadIdx.x == 0 && cid == 0 && rank == 0)
-    for (int i = 0; i < kTimeoutRecInts; ++i) p.timeout_rec[i] = 0;
+  // The next kernel on the stream may start its prologue now.  Roles that read what an earlier
+  // kernel of this library writes (queries, pool pages) or that write global memory call
+  // grid_dep_wait() first; the prologue below touches inputs only.
+  grid_dep_launch();
   if (threadIdx.x < 8) sb.prog[threadIdx.x] = 0;
   if (threadIdx.x == 0) {
     uint32_t counts[B_COUNT];
@@ -387,6 +389,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       // ---- key producer (whole warp: page lookups in warp-wide batches; lane 0 issues): a score
       // tile is up to 2 pages (128 keys), streamed as 9 stages of [128 keys x 64 dims] (8 latent
       // chunks, then the RoPE key).  Optionally, pages further ahead are prefetched into L2.
+      grid_dep_wait();
       SegIter it = it0;
       PageRows pr;
       uint32_t n = 0;
@@ -488,7 +491,9 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       if (warp == 0) {
       // ---- latent producer (whole warp: lookups in warp-wide batches, lane 0 issues): each page's
       // c_KV part is streamed as two half-page stages [64 keys x 256 dims], one per PV MMA group.
+      grid_dep_wait();
       if (cid == 0) {
+        for (int i = lane; i < kTimeoutRecInts; i += 32) p.timeout_rec[i] = 0;
         // Units with no tiles get an empty segment list (their rows combine to zero).
         for (int u = lane; u < p.U; u += 32)
           if (unit_tiles(p, u) == 0) {
@@ -627,6 +632,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       const int q4 = warp & 3, h = (warp - 4) >> 2;
       const int r = q4 * 32 + lane;
       const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+      grid_dep_wait();
       SegIter it = it0;
       uint32_t ns = 0, np = 0, uc = 0;
       const uint32_t pbuf_remote = mapa(smem_u32(tiles + kPOff), peer);
@@ -775,6 +781,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       // ---- epilogue warps: tile fix-ups on request, then each unit's epilogue
       const int r = (warp - 4) * 32 + lane;
       const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+      grid_dep_wait();
       SegIter it = it0;
       uint32_t nreq = 0, uc = 0;
       const uint32_t statsempty_remote = mapa(bar(B_STATSEMPTY), peer);
@@ -882,8 +889,9 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
   const int g0 = blockIdx.y * kCombRows;
   const int rows = B * n_q;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  sm100::grid_dep_launch();
 
-  // W_UV slices stream in while the partials are merged.
+  // W_UV slices stream in while the partials are merged (an input: no need to wait for them).
   const __nv_bfloat16 *w = w_uv ? w_uv + (int64_t)s * kDc * d_v : nullptr;
   auto load_w = [&](int buf, int k0) {
     for (int c = tid; c < 64 * 16; c += kCombThreads) {       // 64 rows x 128 cols = 1024 chunks of 16 B
@@ -894,6 +902,7 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
   };
   if (w)
     for (int i = 0; i < kWSlices - 1; ++i) load_w(i, 64 * i);
+  sm100::grid_dep_wait();   // the partials and the segment table come from the attention kernel
 
   // Merge weights: four threads per row, so every row's segment info and log-sum-exps are
   // fetched at once rather than one row after another.
@@ -1187,6 +1196,11 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, mla_decode_tc_kernel, mc, mpe, p) != cudaSuccess) return MLA_ERR_CUDA;
   return MLA_OK;
 }
@@ -1204,11 +1218,13 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid(d.n_heads, (B * n_q + kCombRows - 1) / kCombRows);
-  tc_combine_kernel<<<grid, kCombThreads, smem, st>>>(
-      B, n_q, d.n_heads, n_rb, B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
-      reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part), reinterpret_cast<const float *>(w + L.lse_part),
-      static_cast<const __nv_bfloat16 *>(w_uv), d.d_v, static_cast<__nv_bfloat16 *>(out), lse);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, B, n_q, d.n_heads, n_rb,
+                    B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
+                    reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part),
+                    reinterpret_cast<const float *>(w + L.lse_part), static_cast<const __nv_bfloat16 *>(w_uv),
+                    d.d_v, static_cast<__nv_bfloat16 *>(out), lse) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 }  // namespace mla

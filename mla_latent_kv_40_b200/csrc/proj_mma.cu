@@ -11,6 +11,7 @@
 // staged by cp.async into padded shared tiles and read with ldmatrix.
 #include "kernels.cuh"
 #include "mma_tile.cuh"
+#include "sm100.cuh"
 
 namespace mla {
 
@@ -107,6 +108,8 @@ append_finish_kernel(AppendArgs a, const float *part, int nsplit) {
   const int W = a.d_c + a.d_rope, npair = W / 2;
   const int tok = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  sm100::grid_dep_launch();
+  sm100::grid_dep_wait();   // the partials come from the projection kernel just before
   const int64_t split_stride = (int64_t)a.T * W / 2;   // in float2
   const float2 *pp = reinterpret_cast<const float2 *>(part) + (int64_t)tok * npair;
   constexpr int kMaxPairsPerThr = 2;
@@ -199,8 +202,10 @@ int launch_append_mma(const AppendArgs &a, void *ws, cudaStream_t st) {
 }
 
 int launch_append_finish(const AppendArgs &a, const void *ws, int nsplit, cudaStream_t st) {
-  append_finish_kernel<<<a.T, kFinThreads, 0, st>>>(a, static_cast<const float *>(ws), nsplit);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_pdl(append_finish_kernel, dim3(a.T), dim3(kFinThreads), 0, st, a, static_cast<const float *>(ws),
+                    nsplit) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 // ------------------------------------------------------------ query absorption

@@ -55,6 +55,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
   const int s = blockIdx.x, m0 = blockIdx.y * 128, r0 = blockIdx.z * kTcN;
   const int R = a.B * a.n_q, W = a.d_c + a.d_rope;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dep_launch();   // reads below touch inputs only; q_out is written after grid_dep_wait()
 
   if (tid == 0) {
     mbar_init(smem_u32(&bar_full), 1);
@@ -90,6 +91,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
     const int half = a.d_rope / 2;
     if (tid - 32 < half) theta[tid - 32] = rope_theta(tid - 32, a.d_rope, a.rope_base);
     asm volatile("bar.sync 1, 96;" ::: "memory");       // warps 1-3 only
+    grid_dep_wait();                                       // q_out may still be read by an earlier kernel
     constexpr int kRowsPerWarp = 8;
     const int nr = (kTcN - (int)blockIdx.y + (int)gridDim.y - 1) / (int)gridDim.y;
     for (int w0 = (warp - 1) * kRowsPerWarp; w0 < nr; w0 += 3 * kRowsPerWarp) {
@@ -149,6 +151,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
   }
   tc_fence_before();
   __syncthreads();
+  grid_dep_wait();
   if (ok) {
     __nv_bfloat16 *qo = static_cast<__nv_bfloat16 *>(a.q_out);
     for (int c = tid; c < kTcN * 16; c += kTcThreads) {
@@ -185,6 +188,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_consta
   const int nst = (kend - kbeg + 63) / 64;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool rope_tile = m0 >= d_c;
+  grid_dep_launch();   // h and the weights are inputs; the partials are written after grid_dep_wait()
 
   if (tid == 0) {
     for (int i = 0; i < kApStages; ++i) {
@@ -242,6 +246,7 @@ append_tc_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_consta
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (ok) mbar_wait(smem_u32(&bar_mma), 0, kWaitNs);
   tc_fence_after();
+  grid_dep_wait();
   // Thread = output column m0 + 32w + lane; for each token its value goes to part[ks][t][m]:
   // consecutive lanes write consecutive columns.
   {
@@ -290,8 +295,9 @@ int launch_absorb_tc(const AbsorbArgs &a, int *dev_status, cudaStream_t st) {
   if (cudaFuncSetAttribute(absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid(a.H, a.d_c / 128, (R + kTcN - 1) / kTcN);
-  absorb_tc_kernel<<<grid, kTcThreads, smem, st>>>(mw, mq, a, dev_status);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_pdl(absorb_tc_kernel, grid, dim3(kTcThreads), smem, st, mw, mq, a, dev_status) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 bool append_tc_supported(const AppendArgs &a, bool bf16) {
@@ -311,9 +317,10 @@ int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split,
   if (cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid((W + 127) / 128, nsplit, (a.T + kTcN - 1) / kTcN);
-  append_tc_kernel<<<grid, kTcThreads, smem, st>>>(mwd, mwr, mh, a.T, a.d_c, a.d_rope, k_per_split, a.d_model,
-                                                   static_cast<float *>(ws), a.dev_status);
-  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+  return launch_pdl(append_tc_kernel, grid, dim3(kTcThreads), smem, st, mwd, mwr, mh, a.T, a.d_c, a.d_rope,
+                    k_per_split, a.d_model, static_cast<float *>(ws), a.dev_status) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 }  // namespace mla
