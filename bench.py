@@ -305,34 +305,74 @@ def run_mla(args):
     att_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in att_ev))
     clocks = clk.summary()
 
-    # End to end through the public call: pinned host inputs in, result out, copies inside the timed region.
+    # End to end through the public calls: pinned host inputs in, result out, every step's copies inside the
+    # timed region.  The inputs of step i+1 are copied (copy stream) while step i computes, into the other of
+    # two device buffer sets, and step i's result goes back (a second copy stream) while step i+1 computes.
     e2e = None
     if not args.no_e2e:
-        host_in = {k: inp[k].pin_memory() for k in ("h_new", "q_nope", "q_pe", "seqlens", "seq_idx", "pos")}
-        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        in_keys = ("h_new", "q_nope", "q_pe", "seqlens", "seq_idx", "pos")
+        host_in = {k: inp[k].pin_memory() for k in in_keys}
+        host_out = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-        d2h = host_out.numel() * host_out.element_size()
+        d2h = host_out[0].numel() * host_out[0].element_size()
+        bufs = [{k: torch.empty_like(dev[k]) for k in in_keys} for _ in range(2)]
+        outs = [torch.empty_like(out) for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        in_free = [torch.cuda.Event() for _ in range(2)]
+        out_ready = [torch.cuda.Event() for _ in range(2)]
+        out_read = [torch.cuda.Event() for _ in range(2)]
+        for e in in_free + out_read:
+            e.record(stream)
 
-        def e2e_step():
-            for k, t in host_in.items():
-                dev[k].copy_(t, non_blocking=True)
-            append()
-            mla.mla_absorb_q(dims, dev["q_nope"], dev["q_pe"], dev["w_uk"], dev["seqlens"], q_abs)
+        def h2d_copy(i):
+            j = i % 2
+            h2d_s.wait_event(in_free[j])              # step i-2 no longer reads buffer set j
+            with torch.cuda.stream(h2d_s):
+                for k in in_keys:
+                    bufs[j][k].copy_(host_in[k], non_blocking=True)
+            in_ready[j].record(h2d_s)
+
+        def e2e_step(i, last):
+            j = i % 2
+            if not last:
+                h2d_copy(i + 1)
+            x = bufs[j]
+            stream.wait_event(in_ready[j])
+            stream.wait_event(out_read[j])            # step i-2's result has left outs[j]
+            side.wait_stream(stream)
+            mla.mla_append_latent(dims, x["h_new"], dev["w_dkv"], dev["w_kr"], dev["gamma"], x["seq_idx"], x["pos"],
+                                  c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status,
+                                  workspace=app_ws, stream=side)
+            appended.record(side)
+            mla.mla_absorb_q(dims, x["q_nope"], x["q_pe"], dev["w_uk"], x["seqlens"], q_abs)
             stream.wait_event(appended)
             mla.mla_decode_attention(dims, q_abs, c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
-                                     dev["seqlens"], max_seqlen, ws, status)
-            mla.mla_decode_combine(dims, B, n_q, dev["seqlens"], max_seqlen, dev["w_uv"], out, lse, ws)
-            host_out.copy_(out, non_blocking=True)
+                                     x["seqlens"], max_seqlen, ws, status)
+            mla.mla_decode_combine(dims, B, n_q, x["seqlens"], max_seqlen, dev["w_uv"], outs[j], lse, ws)
+            in_free[j].record(stream)
+            out_ready[j].record(stream)
+            d2h_s.wait_event(out_ready[j])
+            with torch.cuda.stream(d2h_s):
+                host_out[j].copy_(outs[j], non_blocking=True)
+            out_read[j].record(d2h_s)
 
-        for _ in range(3):
-            e2e_step()
+        def e2e_run(n):
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            h2d_s.wait_event(f0)
+            h2d_copy(0)
+            for i in range(n):
+                e2e_step(i, i == n - 1)
+            stream.wait_stream(d2h_s)                  # the last result is back on the host
+            f1.record(stream)
+            return f0, f1
+
+        e2e_run(3)
         torch.cuda.synchronize()
         barrier()
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        f1.record(stream)
+        f0, f1 = e2e_run(args.steps)
         torch.cuda.synchronize()
         barrier()
         e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps)

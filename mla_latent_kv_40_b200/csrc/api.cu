@@ -95,9 +95,10 @@ int attention_impl(const mla_dims *dims, int B, int n_q, const void *q_abs, cons
 }
 
 int combine_impl(const mla_dims *dims, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
-                 void *out, float *lse, const DecodeLayout &L, char *ws, cudaStream_t st) {
+                 void *out, float *lse, const DecodeLayout &L, char *ws, int *dev_status, cudaStream_t st) {
   const bool bf16 = dims->dtype == MLA_BF16;
-  if (L.use_tc) return launch_tc_combine(*dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, ws + L.tc_off, st);
+  if (L.use_tc)
+    return launch_tc_combine(*dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, ws + L.tc_off, dev_status, st);
   CombineArgs cb{B, n_q, dims->n_heads, dims->d_c, dims->d_v, seqlens, kSimtChunk, L.max_chunks,
                  reinterpret_cast<const float *>(ws + L.o_off), reinterpret_cast<const float *>(ws + L.lse_off),
                  w_uv, out, lse};
@@ -129,7 +130,7 @@ int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const 
   if ((rc = attention_impl(dims, B, n_q, qbuf, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
                            max_seqlen, L, ws, dev_status, st)))
     return rc;
-  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, ws, st);
+  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, ws, dev_status, st);
 }
 
 }  // namespace
@@ -256,7 +257,7 @@ int mla_decode_combine(const mla_dims *dims, int B, int n_q, const int32_t *seql
   const DecodeLayout L = decode_layout(dims, B, n_q, max_seqlen);
   int rc = check_ws(L, workspace, ws_bytes);
   if (rc) return rc;
-  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, static_cast<char *>(workspace),
+  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, static_cast<char *>(workspace), nullptr,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 

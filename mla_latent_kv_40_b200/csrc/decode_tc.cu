@@ -867,41 +867,57 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
 
 // ------------------------------------------------------------ combine (+ W_UV)
 // CTA = (head s, 64 query rows (b, j)).  The split partials of each row are
-// merged by their log-sum-exps into a bf16 [64 x 512] tile in shared memory,
-// which is then multiplied by W_UV[s] ([512 x d_v], streamed in 64-row
-// slices) on warp-level tensor cores: out^(s) = o_lat W_UV^(s).
+// merged by their log-sum-exps into a bf16 [64 x 512] tile o_lat, which is then
+// multiplied by W_UV[s] ([512 x d_v]) on the tensor cores, transposed so that
+// W_UV supplies the 128-row M side: out^T [d_v x 64] = W_UV^(s)T . o_lat^T
+// (A = W_UV^T, M-major; B = o_lat, K-major; fp32 accumulator in 64 tensor-memory
+// columns).  All of W_UV[s] (128 KB) is requested at the start, straight into
+// the MMA's 128-byte-swizzled operand layout, so its transfer overlaps the merge.
 constexpr int kCombRows = 64;
 constexpr int kCombThreads = 256;
 constexpr int kMaxSegPerUnit = kMaxClusters + 1;
-constexpr int kOlLd = kDc + 8;             // padded bf16 row of the merged tile
-constexpr int kWLd = 128 + 8;              // padded bf16 row of a W_UV slice
-constexpr int kWSlices = 4;                // W_UV slices of 64 rows in flight
+constexpr int kDv = 128;                                   // the W_UV tile width this kernel takes
+constexpr uint32_t kOlBytes = kCombRows * kDc * 2;         // o_lat: [8 K-chunks][64 rows][128 B]
+constexpr uint32_t kWuvBytes = kDc * kDv * 2;              // W_UV^T: [8 K-chunks][2 M-chunks][64 K rows][128 B]
 
 __global__ void __launch_bounds__(kCombThreads)
 tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part,
-                  const float *lse_part, const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out) {
-  extern __shared__ __align__(16) unsigned char csm[];
-  __nv_bfloat16 *ol = reinterpret_cast<__nv_bfloat16 *>(csm);                     // [64][kOlLd]
-  __nv_bfloat16 *wsl = ol + kCombRows * kOlLd;                                     // [kWSlices][64][kWLd]
-  float *wgt = reinterpret_cast<float *>(wsl + kWSlices * 64 * kWLd);              // [64][kMaxSegPerUnit]
+                  const float *lse_part, const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out,
+                  int *dev_status) {
+  extern __shared__ unsigned char csm_raw[];
+  unsigned char *csm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char *ol = csm;                                                          // o_lat, K-major, swizzled
+  unsigned char *wa = csm + kOlBytes;                                               // W_UV^T, M-major, swizzled
+  float *wgt = reinterpret_cast<float *>(wa + kWuvBytes);                           // [64][kMaxSegPerUnit]
   int *sinfo = reinterpret_cast<int *>(wgt + kCombRows * kMaxSegPerUnit);          // [64][3]
+  __shared__ __align__(8) uint64_t bar_mma;
+  __shared__ uint32_t tmem_slot;
   const int s = blockIdx.x;
   const int g0 = blockIdx.y * kCombRows;
   const int rows = B * n_q;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  (void)d_v;
   sm100::grid_dep_launch();
+  const __nv_bfloat16 *w = w_uv ? w_uv + (int64_t)s * kDc * kDv : nullptr;
 
-  // W_UV slices stream in while the partials are merged (an input: no need to wait for them).
-  const __nv_bfloat16 *w = w_uv ? w_uv + (int64_t)s * kDc * d_v : nullptr;
-  auto load_w = [&](int buf, int k0) {
-    for (int c = tid; c < 64 * 16; c += kCombThreads) {       // 64 rows x 128 cols = 1024 chunks of 16 B
-      const int r = c >> 4, q = c & 15;
-      mma::cp16(wsl + (buf * 64 + r) * kWLd + q * 8, w + (int64_t)(k0 + r) * d_v + q * 8, true);
+  if (w) {
+    if (tid == 0) {
+      mbar_init(smem_u32(&bar_mma), 1);
+      fence_mbar_init();
+    }
+    if (warp == 0) {
+      tmem_alloc(smem_u32(&tmem_slot), kCombRows);
+      tmem_relinquish();
+    }
+    // W_UV[s] (an input: no need to wait): row k, 16-byte group q (8 output columns) ->
+    // K-chunk k/64, M-chunk q/8, row k%64, group (q%8) XOR (k%8).
+    for (int c = tid; c < kDc * (kDv / 8); c += kCombThreads) {
+      const int k = c >> 4, q = c & 15;
+      const int kc = k >> 6, kr = k & 63, mc = q >> 3, qq = q & 7;
+      mma::cp16(wa + ((kc * 2 + mc) * 64 + kr) * 128 + ((qq ^ (kr & 7)) << 4), w + (int64_t)k * kDv + q * 8, true);
     }
     mma::cp_commit();
-  };
-  if (w)
-    for (int i = 0; i < kWSlices - 1; ++i) load_w(i, 64 * i);
+  }
   sm100::grid_dep_wait();   // the partials and the segment table come from the attention kernel
 
   // Merge weights: four threads per row, so every row's segment info and log-sum-exps are
@@ -954,16 +970,14 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
     constexpr int kRowStep = kCombThreads / kGroups;         // 4
     constexpr int kItems = 8;
     constexpr int kPasses = kCombRows / (kRowStep * kItems); // 2
-    const int c8 = (tid % kGroups) * 8, rr0 = tid / kGroups;
+    const int c8 = tid % kGroups, rr0 = tid / kGroups;
 #pragma unroll 1
     for (int pass = 0; pass < kPasses; ++pass) {
       float v[kItems][8];
-      int nsr[kItems];
       int maxns = 0;
 #pragma unroll
       for (int i = 0; i < kItems; ++i) {
-        nsr[i] = sinfo[3 * (rr0 + kRowStep * (i + kItems * pass)) + 1];
-        maxns = max(maxns, nsr[i]);
+        maxns = max(maxns, sinfo[3 * (rr0 + kRowStep * (i + kItems * pass)) + 1]);
 #pragma unroll
         for (int k = 0; k < 8; ++k) v[i][k] = 0.f;
       }
@@ -972,14 +986,14 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
 #pragma unroll
         for (int i = 0; i < kItems; ++i) {
           const int rr = rr0 + kRowStep * (i + kItems * pass);
-          x[i] = k < nsr[i] ? *reinterpret_cast<const uint4 *>(
-                                  o_part + ((int64_t)(sinfo[3 * rr] + k) * kRows + sinfo[3 * rr + 2]) * kDc + c8)
-                            : make_uint4(0, 0, 0, 0);
+          x[i] = k < sinfo[3 * rr + 1] ? *reinterpret_cast<const uint4 *>(
+                                             o_part + ((int64_t)(sinfo[3 * rr] + k) * kRows + sinfo[3 * rr + 2]) * kDc + c8 * 8)
+                                       : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int i = 0; i < kItems; ++i) {
           const int rr = rr0 + kRowStep * (i + kItems * pass);
-          const float wk = k < nsr[i] ? wgt[rr * kMaxSegPerUnit + k] : 0.f;
+          const float wk = k < sinfo[3 * rr + 1] ? wgt[rr * kMaxSegPerUnit + k] : 0.f;
           const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[i]);
 #pragma unroll
           for (int e2 = 0; e2 < 4; ++e2) {
@@ -989,6 +1003,7 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
           }
         }
       }
+      // Row rr, latent group c8 -> K-chunk c8/8, group (c8%8) XOR (rr%8) of the row's 128 bytes.
 #pragma unroll
       for (int i = 0; i < kItems; ++i) {
         const int rr = rr0 + kRowStep * (i + kItems * pass);
@@ -996,56 +1011,70 @@ tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_
         __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
 #pragma unroll
         for (int e2 = 0; e2 < 4; ++e2) ph[e2] = __floats2bfloat162_rn(v[i][2 * e2], v[i][2 * e2 + 1]);
-        *reinterpret_cast<uint4 *>(ol + rr * kOlLd + c8) = packed;
+        *reinterpret_cast<uint4 *>(ol + (c8 >> 3) * 8192 + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4)) = packed;
       }
     }
   }
-  __syncthreads();
   if (!w) {   // latent output: o_lat itself
+    __syncthreads();
     for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
-      const int rr = e / (kDc / 8), c8 = (e % (kDc / 8)) * 8, g = g0 + rr;
-      if (g < rows) *reinterpret_cast<uint4 *>(out + ((int64_t)g * H + s) * kDc + c8) = *reinterpret_cast<const uint4 *>(ol + rr * kOlLd + c8);
+      const int rr = e / (kDc / 8), c8 = e % (kDc / 8), g = g0 + rr;
+      if (g < rows)
+        *reinterpret_cast<uint4 *>(out + ((int64_t)g * H + s) * kDc + c8 * 8) =
+            *reinterpret_cast<const uint4 *>(ol + (c8 >> 3) * 8192 + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4));
     }
     return;
   }
-  // out [64 x 128] = ol [64 x 512] . W_UV[s] [512 x 128]; warp (wr, wc) owns rows 16wr.. and columns 64wc..
-  const int wr = warp & 3, wc = warp >> 2;
-  float acc[8][4];
+  // Both operands written by this CTA's threads (generic proxy) -> visible to the tensor cores.
+  mma::cp_wait<0>();
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+  if (tid == 0) {
+    const uint32_t idesc = idesc_bf16_f32(128, kCombRows, true, false);
+    for (int kc = 0; kc < kDc / 64; ++kc)
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) acc[i][k] = 0.f;
-  for (int it = 0; it < kDc / 64; ++it) {
-    const int buf = it % kWSlices;
-    // Keep kWSlices - 1 slices in flight: issue slice it + 3 (or an empty group), then wait for slice it.
-    if (it + kWSlices - 1 < kDc / 64) load_w((it + kWSlices - 1) % kWSlices, 64 * (it + kWSlices - 1));
-    else mma::cp_commit();
-    mma::cp_wait<kWSlices - 1>();
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 64; kk += 16) {
-      uint32_t a[4];
-      mma::load_a(ol, kOlLd, wr * 16, 64 * it + kk, a);
-#pragma unroll
-      for (int nt = 0; nt < 8; nt += 2) {
-        uint32_t bb[4];
-        mma::load_b2(wsl + buf * 64 * kWLd, kWLd, kk, wc * 64 + nt * 8, true, bb);
-        mma::mma16816(acc[nt], a, bb[0], bb[1]);
-        mma::mma16816(acc[nt + 1], a, bb[2], bb[3]);
-      }
-    }
-    __syncthreads();
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tmem, smem_desc_sw128(smem_u32(wa + kc * 16384) + kk * 2048, 8192, 1024),
+               smem_desc_sw128(smem_u32(ol + kc * 8192) + kk * 32, 16, 1024), idesc, (kc | kk) ? 1u : 0u);
+    tc_commit(smem_u32(&bar_mma));
   }
-  const int gq = lane >> 2, q = lane & 3;
+  int ok = 1;
+  if (lane == 0 && !mbar_wait(smem_u32(&bar_mma), 0, kWaitNs)) {
+    report(dev_status, MLA_ERR_TIMEOUT);
+    ok = 0;
+  }
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_wait(smem_u32(&bar_mma), 0, kWaitNs);
+  tc_fence_after();
+  // Warp w drains output columns 32(w%4).. (its lane quadrant) for query rows 32(w/4)..: each thread
+  // holds one output column of 32 rows -> a [64 rows x 128] bf16 staging tile over o_lat's space.
+  __nv_bfloat16 *stg = reinterpret_cast<__nv_bfloat16 *>(ol);
+  constexpr int lds = kDv + 8;
+  {
+    uint32_t v[32];
+    tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 32 * (warp >> 2), v);
+    tmem_wait_ld();
+    __syncthreads();   // every thread is past its reads of o_lat (the MMAs completed before the loads)
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int g = g0 + wr * 16 + gq + 8 * hf;
+    for (int i = 0; i < 32; ++i)
+      stg[(32 * (warp >> 2) + i) * lds + (warp & 3) * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (ok)
+    for (int c = tid; c < kCombRows * (kDv / 8); c += kCombThreads) {
+      const int rr = c >> 4, q8 = c & 15, g = g0 + rr;
       if (g < rows)
-        *reinterpret_cast<__nv_bfloat162 *>(out + ((int64_t)g * H + s) * d_v + wc * 64 + nt * 8 + 2 * q) =
-            __floats2bfloat162_rn(acc[nt][2 * hf], acc[nt][2 * hf + 1]);
+        *reinterpret_cast<uint4 *>(out + ((int64_t)g * H + s) * kDv + q8 * 8) =
+            *reinterpret_cast<const uint4 *>(stg + rr * lds + q8 * 8);
     }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCombRows);
+  }
 }
 
 // ------------------------------------------------------------ host side
@@ -1206,15 +1235,15 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
 }
 
 int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
-                      void *out, float *lse, void *ws, cudaStream_t st) {
+                      void *out, float *lse, void *ws, int *dev_status, cudaStream_t st) {
   (void)seqlens;
   (void)max_seqlen;
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
   const WsLayout L = ws_layout(B, n_rb);
   char *w = static_cast<char *>(ws);
-  const size_t smem = sizeof(__nv_bfloat16) * (kCombRows * kOlLd + kWSlices * 64 * kWLd) +
-                      sizeof(float) * kCombRows * kMaxSegPerUnit + sizeof(int) * 3 * kCombRows;
-  if (w_uv && d.d_v != 128) return MLA_ERR_UNSUPPORTED;
+  const size_t smem = 1024 + kOlBytes + kWuvBytes + sizeof(float) * kCombRows * kMaxSegPerUnit +
+                      sizeof(int) * 3 * kCombRows;
+  if (w_uv && (d.d_v != kDv || (reinterpret_cast<uintptr_t>(w_uv) & 15))) return MLA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid(d.n_heads, (B * n_q + kCombRows - 1) / kCombRows);
@@ -1222,7 +1251,7 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
                     B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
                     reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part),
                     reinterpret_cast<const float *>(w + L.lse_part), static_cast<const __nv_bfloat16 *>(w_uv),
-                    d.d_v, static_cast<__nv_bfloat16 *>(out), lse) == cudaSuccess
+                    d.d_v, static_cast<__nv_bfloat16 *>(out), lse, dev_status) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
 }

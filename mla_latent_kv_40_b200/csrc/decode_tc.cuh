@@ -16,6 +16,6 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
                         const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st);
 // Merge of the partials (+ W_UV when w_uv != NULL).
 int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
-                      void *out, float *lse, void *ws, cudaStream_t st);
+                      void *out, float *lse, void *ws, int *dev_status, cudaStream_t st);
 
 }  // namespace mla
