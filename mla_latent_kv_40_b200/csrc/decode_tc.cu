@@ -65,8 +65,8 @@ constexpr uint32_t kPTxBytes = kPWriters * kStgBytes;              // bytes that
 constexpr uint32_t kQpeOff = 0;                                    // score CTA: Q rope part, [128 x 64] bf16
 constexpr uint32_t kKOff = kRows * 128;                            // score CTA: key stages
 constexpr uint32_t kPOff = kVStages * kVStageBytes;                // value CTA: P slots
-constexpr uint32_t kStgOff = kKOff + kKStages * kKStageBytes;      // score CTA: 8 warp staging buffers
-constexpr uint32_t kRegionA = (kStgOff + 8 * kStgBytes + 1023) & ~1023u;   // 214016
+constexpr uint32_t kStgOff = kKOff + kKStages * kKStageBytes;      // score CTA: P pages of both halves, factors
+constexpr uint32_t kRegionA = (kStgOff + 2 * kPTxBytes + 1023) & ~1023u;   // 214016
 static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
 #ifndef MLA_TC_PREFETCH_PAGES
 #define MLA_TC_PREFETCH_PAGES 0
@@ -637,7 +637,9 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       uint32_t ns = 0, np = 0, uc = 0;
       const uint32_t pbuf_remote = mapa(smem_u32(tiles + kPOff), peer);
       const uint32_t pa_remote = mapa(smem_u32(&sb.pa[0][0][0]), peer);
-      unsigned char *stg = tiles + kStgOff + (warp - 4) * kStgBytes;   // this warp's staging buffer
+      // Staging of this half's P page (all four lane quadrants) and of its rescale factors.
+      unsigned char *stgp = tiles + kStgOff + h * kPBytes;
+      unsigned char *stga = tiles + kStgOff + 2 * kPBytes + h * (kPWriters * kPaWords * 4);
       const uint32_t statl_remote = mapa(smem_u32(&sb.stat_l[0]), peer);
       const uint32_t statm_remote = mapa(smem_u32(&sb.stat_m[0]), peer);
       const uint32_t pfull_remote = mapa(bar(B_PFULL), peer);
@@ -721,13 +723,14 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           if (h < npg) {
             const uint32_t pn = np + h;
             const int pb = pn % kPSlots;
-            // The staging buffer is free once this warp's previous bulk copies have read it.
-            if (lane == 0) bulk_wait_read_all();
-            __syncwarp();
+            const bool issuer = q4 == 0 && lane == 0;   // sends the half's page for all four warps
+            // The page's staging buffer is free once the previous copies out of it have read it.
+            if (issuer) bulk_wait_read_all();
+            asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
             // My 32 P rows, K-major and 128B-swizzled like the value CTA's [128 x 64] P tile (rows
             // 32q..32q+31 are its bytes 4096q..4096q+4095), then the rows' rescale factors (the first
             // page of a score tile carries the tile's factors) and the warp's flag word.
-            unsigned char *prow = stg + (lane >> 3) * 1024 + (lane & 7) * 128;
+            unsigned char *prow = stgp + 4096 * q4 + (lane >> 3) * 1024 + (lane & 7) * 128;
             float psum = 0.f;
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
@@ -743,22 +746,21 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
               *reinterpret_cast<uint4 *>(prow + ((c ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             l += psum;
-            reinterpret_cast<float *>(stg + 4096)[lane] = h == 0 ? alpha : 1.f;
+            float *pa = reinterpret_cast<float *>(stga) + q4 * kPaWords;
+            pa[lane] = h == 0 ? alpha : 1.f;
             const unsigned moved = __ballot_sync(0xffffffffu, need && h == 0 && T != t0);
-            if (lane < 4) reinterpret_cast<uint32_t *>(stg + 4096 + 128)[lane] = (lane == 0 && moved) ? 1u : 0u;
+            if (lane < 4) reinterpret_cast<uint32_t *>(pa + 32)[lane] = (lane == 0 && moved) ? 1u : 0u;
             fence_proxy_async_smem();
-            __syncwarp();
+            asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
             // Into the value CTA's slot once the MMAs that read its previous contents completed: two
-            // bulk copies that complete on the slot's P-full barrier (armed by the relay).
-            if (pn < kPSlots ||
-                warp_wait(sb, bar(B_PEMPTY + pb), ((pn / kPSlots) - 1) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
-              if (lane == 0) {
-                const uint32_t pfull = pfull_remote + 8 * pb;
-                bulk_copy_to_peer(pbuf_remote + pb * kPBytes + 4096 * q4, smem_u32(stg), 4096, pfull);
-                bulk_copy_to_peer(pa_remote + (pb * kPWriters + q4) * (kPaWords * 4), smem_u32(stg + 4096),
-                                  kPaWords * 4, pfull);
-                bulk_commit();
-              }
+            // bulk copies (the page, its factors) that complete on the slot's P-full barrier.
+            if (issuer && (pn < kPSlots || wait_or_abort(sb, bar(B_PEMPTY + pb), ((pn / kPSlots) - 1) & 1, p.dev_status,
+                                                         true, p.timeout_rec, __LINE__))) {
+              const uint32_t pfull = pfull_remote + 8 * pb;
+              bulk_copy_to_peer(pbuf_remote + pb * kPBytes, smem_u32(stgp), kPBytes, pfull);
+              bulk_copy_to_peer(pa_remote + pb * (kPWriters * kPaWords * 4), smem_u32(stga), kPWriters * kPaWords * 4,
+                                pfull);
+              bulk_commit();
             }
           }
           np += npg;
