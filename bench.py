@@ -118,10 +118,14 @@ _TRAFFIC_SOURCES = {"decode_tc.cu": ("decode_tc.cu", "decode_tc.cuh", "sm100.cuh
 
 
 def traffic_source_hash(kernel_file):
+    """Hash of the kernel's sources with // comments and blank lines removed (comment edits keep the figure)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in _TRAFFIC_SOURCES[kernel_file]:
-        h.update(open(os.path.join(ROOT, "mla_latent_kv_40_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "mla_latent_kv_40_b200", "csrc", f), encoding="utf-8").read()
+        code = [re.sub(r"\s*//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in code if ln).encode())
     return h.hexdigest()[:16]
 
 

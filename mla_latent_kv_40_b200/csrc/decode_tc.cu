@@ -10,13 +10,16 @@
 // Resources decide the shape of the kernel.  O is 128 x 512 fp32 = 256 KB, the
 // whole tensor memory of one SM, and Q is 147 KB of bf16.  So each work unit
 // runs on a cluster of two CTAs on two SMs:
-//   * the score CTA (rank 0) keeps Q in its tensor memory (A operand of a
-//     TS-form MMA), streams full 576-wide key tiles with TMA, computes S into
-//     tensor memory, runs the online softmax in registers and writes P (bf16)
-//     straight into the value CTA's shared memory (distributed shared memory);
+//   * the score CTA (rank 0) keeps the latent part of Q in its tensor memory
+//     (A operand of TS-form MMAs) and the RoPE part in shared memory, streams
+//     the unit's pages as stages of [128 keys x 64 dims] (contiguous 8 KB
+//     chunks of the tiled pool), computes S for two pages at a time into one
+//     of two tensor-memory buffers, runs the online softmax in registers, and
+//     sends each page of P (bf16, staged in shared memory) to the value CTA
+//     with one shared-to-peer bulk copy (distributed shared memory);
 //   * the value CTA (rank 1) streams the 512-wide latent part of the same
-//     tiles with TMA and accumulates O = P . C in all 512 tensor-memory
-//     columns, then normalises and writes the unit's partial output.
+//     pages and accumulates O = P . C in all 512 tensor-memory columns, then
+//     normalises and writes the unit's partial output.
 // The score CTA does 53% of the MMA work and the value CTA 47%.
 //
 // Online softmax uses a lazy reference maximum (kept in log2 units): P is
