@@ -69,7 +69,8 @@ constexpr uint32_t kQpeOff = 0;                                    // score CTA:
 constexpr uint32_t kKOff = kRows * 128;                            // score CTA: key stages
 constexpr uint32_t kPOff = kVStages * kVStageBytes;                // value CTA: P slots
 constexpr uint32_t kStgOff = kKOff + kKStages * kKStageBytes;      // score CTA: P pages of both halves, factors
-constexpr uint32_t kRegionA = (kStgOff + 2 * kPTxBytes + 1023) & ~1023u;   // 214016
+constexpr uint32_t kScoreEnd = kStgOff + 2 * kPTxBytes, kValueEnd = kPOff + kPSlots * kPBytes;
+constexpr uint32_t kRegionA = ((kScoreEnd > kValueEnd ? kScoreEnd : kValueEnd) + 1023) & ~1023u;   // 214016
 static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
 #ifndef MLA_TC_PREFETCH_PAGES
 #define MLA_TC_PREFETCH_PAGES 0

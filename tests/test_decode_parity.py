@@ -15,7 +15,7 @@ from helpers import check_close, gpu_decode
 pytestmark = pytest.mark.gpu
 
 SMALL = ["small_f32", "small_f32_nq2", "tiny_fp32", "small_v3_bf16", "small_v3_nq2_bf16", "small_v2lite_bf16",
-         "small_v3_contig_bf16"]
+         "small_v3_contig_bf16", "small_v3_b128_bf16", "small_v3_many_bf16"]
 
 
 def _oracle(inp, picks=None, latent=False):

@@ -110,6 +110,12 @@ DECODE_CASES = {
     "small_v3_nq2_bf16": DecodeCase("small_v3_nq2_bf16", Dims(**V3), 4, 2, ("list", (2, 64, 129, 1000)), 64, True, 2004),
     "small_v2lite_bf16": DecodeCase("small_v2lite_bf16", Dims(**V2_LITE), 5, 1, ("list", (63, 64, 65, 511, 2048)), 64, True, 2005),
     "small_v3_contig_bf16": DecodeCase("small_v3_contig_bf16", Dims(**V3), 2, 1, ("list", (300, 1024)), 64, False, 2006),
+    # 128-token blocks (two 64-token pages per block in the tiled pool).
+    "small_v3_b128_bf16": DecodeCase("small_v3_b128_bf16", Dims(**V3), 3, 1, ("list", (100, 128, 513)), 128, True, 2007),
+    # Many short units: clusters cross unit boundaries, page boundaries at every offset class.
+    "small_v3_many_bf16": DecodeCase("small_v3_many_bf16", Dims(**V3), 24, 1,
+                                     ("list", (1, 5, 64, 65, 127, 128, 129, 200, 255, 256, 257, 300, 383, 384, 385,
+                                               448, 511, 512, 513, 600, 640, 700, 768, 1000)), 64, True, 2008),
 }
 
 PREFILL_CASES = {
