@@ -102,6 +102,9 @@ int launch_absorb(const AbsorbArgs &a, bool bf16, cudaStream_t st);
 int launch_attn_simt(const AttnArgs &a, bool bf16, cudaStream_t st);
 int launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st);
 int launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st);
+// Step (3) of the prefill, causal attention over the decompressed rows, on tcgen05.
+bool prefill_tc_supported(const PrefillArgs &a, bool bf16);
+int launch_prefill_tc_attention(const PrefillArgs &a, cudaStream_t st);
 // bf16 tensor-core (mma.sync) projections.
 size_t append_mma_workspace(int T, int d_model, int W, int *nsplit, int *k_per_split);
 bool append_mma_supported(const AppendArgs &a, bool bf16);

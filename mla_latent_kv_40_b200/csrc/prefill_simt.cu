@@ -237,6 +237,9 @@ static int launch_prefill_t(const PrefillArgs &a, cudaStream_t st) {
   if (cudaFuncSetAttribute(prefill_decompress_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dec))
     return MLA_ERR_CUDA;
   prefill_decompress_kernel<T><<<dim3(a.H, (a.total + kDecRows - 1) / kDecRows), kPfThreads, smem_dec, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+  // Step (3) on the tensor cores where the shape allows it (bf16, 192-wide keys, 128-wide values).
+  if (prefill_tc_supported(a, sizeof(T) == 2)) return launch_prefill_tc_attention(a, st);
   const size_t smem_att = sizeof(float) * (kPfRows * dqk + kPfKeys * (dqk + 1) + kPfKeys * (a.d_v + 1) +
                                            kPfRows * kPfKeys + 3 * kPfRows);
   if (cudaFuncSetAttribute(prefill_attn_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_att))
