@@ -104,6 +104,9 @@ int launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st);
 int launch_prefill_simt(const PrefillArgs &a, bool bf16, cudaStream_t st);
 // Step (3) of the prefill, causal attention over the decompressed rows, on tcgen05.
 bool prefill_tc_supported(const PrefillArgs &a, bool bf16);
+// Step (2) of the prefill, per-head decompression of K and V, on tcgen05 (row pools).
+bool decompress_tc_supported(const PrefillArgs &a, bool bf16);
+int launch_decompress_tc(const PrefillArgs &a, cudaStream_t st);
 int launch_prefill_tc_attention(const PrefillArgs &a, cudaStream_t st);
 // bf16 tensor-core (mma.sync) projections.
 size_t append_mma_workspace(int T, int d_model, int W, int *nsplit, int *k_per_split);

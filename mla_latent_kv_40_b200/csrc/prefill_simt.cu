@@ -236,7 +236,11 @@ static int launch_prefill_t(const PrefillArgs &a, cudaStream_t st) {
   const size_t smem_dec = sizeof(float) * kDecRows * a.d_c;
   if (cudaFuncSetAttribute(prefill_decompress_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dec))
     return MLA_ERR_CUDA;
-  prefill_decompress_kernel<T><<<dim3(a.H, (a.total + kDecRows - 1) / kDecRows), kPfThreads, smem_dec, st>>>(a);
+  if (decompress_tc_supported(a, sizeof(T) == 2)) {
+    if (const int rc = launch_decompress_tc(a, st)) return rc;
+  } else {
+    prefill_decompress_kernel<T><<<dim3(a.H, (a.total + kDecRows - 1) / kDecRows), kPfThreads, smem_dec, st>>>(a);
+  }
   if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
   // Step (3) on the tensor cores where the shape allows it (bf16, 192-wide keys, 128-wide values).
   if (prefill_tc_supported(a, sizeof(T) == 2)) return launch_prefill_tc_attention(a, st);

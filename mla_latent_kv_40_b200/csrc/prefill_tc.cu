@@ -293,12 +293,202 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   }
 }
 
+// ------------------------------------------------------------ decompression
+// CTA = (sequence b, head s, 128 tokens p0.. of the sequence):
+//   D [128 tokens x 256] = C [128 x d_c] . [W_UK^(s) | W_UV^(s)] [d_c x 256]
+// A = the tokens' latent rows (K-major, two 64-token pages per K chunk, TMA boxes from the
+// row pool through the block table), B = the two weights side by side (N-major: output
+// columns contiguous, 64-column chunks), streamed over d_c in stages of 64.
+// Columns 0..127 are k_nope -> kbuf[t][s][0..127], columns 128..255 are v -> vbuf[t][s][..];
+// the token's RoPE key is copied to kbuf[t][s][128..191].
+constexpr int kDcTok = 128;                    // tokens per CTA
+constexpr int kDcStages = 4;
+constexpr uint32_t kDcA = kDcTok * 128;        // [128 tokens x 64 dims]: 16 KB
+constexpr uint32_t kDcB = 4 * kKChunk;         // [64 dims x 256 outputs]: 4 chunks of [64 x 64]
+constexpr uint32_t kDcStage = kDcA + kDcB;     // 48 KB
+constexpr size_t kDcSmem = 1024 + kDcStages * kDcStage + 64;
+
+struct DcParams {
+  int H, d_c, block_size, max_blocks_per_seq, num_blocks, total;
+  const int32_t *cu_seqlens, *block_table;
+  const __nv_bfloat16 *k_pe;
+  int64_t kpe_stride;
+  __nv_bfloat16 *kbuf, *vbuf;
+  int *dev_status;
+};
+
+__device__ __forceinline__ int64_t dc_row(const DcParams &p, int b, int pos) {
+  const int lb = pos / p.block_size;
+  if (lb >= p.max_blocks_per_seq) return -1;
+  const int blk = p.block_table ? p.block_table[(int64_t)b * p.max_blocks_per_seq + lb] : b * p.max_blocks_per_seq + lb;
+  if (blk < 0 || blk >= p.num_blocks) return -1;
+  return (int64_t)blk * p.block_size + pos % p.block_size;
+}
+
+__global__ void __launch_bounds__(128, 1)
+decompress_tc_kernel(const __grid_constant__ CUtensorMap mc, const __grid_constant__ CUtensorMap mwk,
+                     const __grid_constant__ CUtensorMap mwv, const DcParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *tiles = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kDcStages], empty[kDcStages], done;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int page_row[2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.z, s = blockIdx.y;
+  const int start = p.cu_seqlens[b], L = p.cu_seqlens[b + 1] - start;
+  const int p0 = blockIdx.x * kDcTok;
+  if (start < 0 || L < 0 || start + L > p.total) {
+    if (threadIdx.x == 0 && s == 0 && blockIdx.x == 0) report(p.dev_status, MLA_ERR_BAD_INDEX);
+    return;
+  }
+  if (p0 >= L) return;                                          // CTA-uniform
+  const int nkc = p.d_c / 64;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kDcStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    mbar_init(smem_u32(&done), 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 2) {
+    // first pool row of each 64-token page of the tile (-1: past the end or a bad block id)
+    const int pos = p0 + 64 * threadIdx.x;
+    page_row[threadIdx.x] = pos < L ? (int)dc_row(p, b, pos) : -1;
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(&tmem_slot), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+  grid_dep_launch();
+  int ok = 1;
+  if (warp == 0 && lane == 0) {
+    grid_dep_wait();
+    for (int kc = 0; kc < nkc; ++kc) {
+      const int st = kc % kDcStages;
+      if (kc >= kDcStages && !mbar_wait(smem_u32(&empty[st]), ((kc / kDcStages) - 1) & 1, kWait)) {
+        report(p.dev_status, MLA_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      unsigned char *stg = tiles + st * kDcStage;
+      mbar_expect_tx(smem_u32(&full[st]), kDcStage);
+      for (int pg = 0; pg < 2; ++pg)   // a page past the end (or invalid) reads row 0: masked on output
+        tma_load_2d(smem_u32(stg + pg * (64 * 128)), &mc, 64 * kc, max(page_row[pg], 0), smem_u32(&full[st]));
+      for (int c = 0; c < 2; ++c) {
+        tma_load_2d(smem_u32(stg + kDcA + c * kKChunk), &mwk, 64 * c, s * p.d_c + 64 * kc, smem_u32(&full[st]));
+        tma_load_2d(smem_u32(stg + kDcA + (2 + c) * kKChunk), &mwv, 64 * c, s * p.d_c + 64 * kc, smem_u32(&full[st]));
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = idesc_bf16_f32(128, 256, false, true);
+    for (int kc = 0; kc < nkc; ++kc) {
+      const int st = kc % kDcStages;
+      if (!mbar_wait(smem_u32(&full[st]), (kc / kDcStages) & 1, kWait)) {
+        report(p.dev_status, MLA_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a = smem_u32(tiles + st * kDcStage), bb = a + kDcA;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ss(tbase, smem_desc_sw128(a + kk * 32, 16, 1024), smem_desc_sw128(bb + kk * 2048, kKChunk, 1024), idesc,
+               (kc | kk) ? 1u : 0u);
+      tc_commit(smem_u32(&empty[st]));
+    }
+    tc_commit(smem_u32(&done));
+  }
+  ok = __syncthreads_and(ok);
+  int ok2 = 0;
+  if (lane == 0 && ok) ok2 = mbar_wait(smem_u32(&done), 0, kWait) ? 1 : 0;
+  ok2 = __shfl_sync(0xffffffffu, ok2, 0);
+  if (ok2) mbar_wait(smem_u32(&done), 0, kWait);
+  tc_fence_after();
+  grid_dep_wait();
+  // Thread = token p0 + 32w + lane (its tensor-memory lane): 256 outputs -> kbuf / vbuf rows.
+  const int tok = 32 * warp + lane, pos = p0 + tok;
+  const bool real = ok2 && pos < L && page_row[tok >> 6] >= 0;
+  const int64_t t = start + pos;
+#pragma unroll 1
+  for (int c = 0; c < 8; ++c) {
+    uint32_t v[32];
+    tmem_ld32(tbase + ((uint32_t)(32 * warp) << 16) + 32 * c, v);
+    tmem_wait_ld();
+    if (real) {
+      __nv_bfloat16 *dst = c < 4 ? p.kbuf + (t * p.H + s) * kDqk + 32 * c : p.vbuf + (t * p.H + s) * kDvp + 32 * (c - 4);
+#pragma unroll
+      for (int i = 0; i < 32; i += 8)
+        *reinterpret_cast<uint4 *>(dst + i) =
+            make_uint4(pack_bf16x2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                       pack_bf16x2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
+                       pack_bf16x2(__uint_as_float(v[i + 4]), __uint_as_float(v[i + 5])),
+                       pack_bf16x2(__uint_as_float(v[i + 6]), __uint_as_float(v[i + 7])));
+    }
+  }
+  if (real) {   // the shared RoPE key, already rotated in the cache
+    const int64_t row = (int64_t)page_row[tok >> 6] + (tok & 63);
+    const uint4 *src = reinterpret_cast<const uint4 *>(p.k_pe + row * p.kpe_stride);
+    uint4 *dst = reinterpret_cast<uint4 *>(p.kbuf + (t * p.H + s) * kDqk + 128);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = src[i];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
 }  // namespace
 
 bool prefill_tc_supported(const PrefillArgs &a, bool bf16) {
   return bf16 && a.d_nope + a.d_rope == kDqk && a.d_v == kDvp && a.cache.d_c > 0 &&
          !(reinterpret_cast<uintptr_t>(a.qbuf) & 15) && !(reinterpret_cast<uintptr_t>(a.kbuf) & 15) &&
          !(reinterpret_cast<uintptr_t>(a.vbuf) & 15) && !(reinterpret_cast<uintptr_t>(a.out) & 15);
+}
+
+bool decompress_tc_supported(const PrefillArgs &a, bool bf16) {
+  const CacheView &c = a.cache;
+  return bf16 && a.d_nope == 128 && a.d_v == kDvp && a.d_rope == 64 && a.d_c % 64 == 0 && c.layout == MLA_CACHE_ROWS &&
+         c.block_size % 64 == 0 && !(reinterpret_cast<uintptr_t>(c.c_kv) & 15) &&
+         !(reinterpret_cast<uintptr_t>(c.k_pe) & 15) && (c.ckv_stride * 2) % 16 == 0 && (c.kpe_stride * 2) % 16 == 0 &&
+         !(reinterpret_cast<uintptr_t>(a.w_uk) & 15) && !(reinterpret_cast<uintptr_t>(a.w_uv) & 15) &&
+         !(reinterpret_cast<uintptr_t>(a.kbuf) & 15) && !(reinterpret_cast<uintptr_t>(a.vbuf) & 15);
+}
+
+int launch_decompress_tc(const PrefillArgs &a, cudaStream_t st) {
+  const CacheView &c = a.cache;
+  CUtensorMap mc, mwk, mwv;
+  const uint64_t pool_rows = (uint64_t)c.num_blocks * c.block_size;
+  if (!make_tmap_bf16(&mc, c.c_kv, a.d_c, pool_rows, (uint64_t)c.ckv_stride * 2, 64) ||
+      !make_tmap_bf16(&mwk, a.w_uk, a.d_nope, (uint64_t)a.H * a.d_c, (uint64_t)a.d_nope * 2, 64) ||
+      !make_tmap_bf16(&mwv, a.w_uv, a.d_v, (uint64_t)a.H * a.d_c, (uint64_t)a.d_v * 2, 64))
+    return MLA_ERR_CUDA;
+  if (cudaFuncSetAttribute(decompress_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDcSmem))
+    return MLA_ERR_CUDA;
+  DcParams p;
+  p.H = a.H;
+  p.d_c = a.d_c;
+  p.block_size = c.block_size;
+  p.max_blocks_per_seq = c.max_blocks_per_seq;
+  p.num_blocks = c.num_blocks;
+  p.total = a.total;
+  p.cu_seqlens = a.cu_seqlens;
+  p.block_table = c.block_table;
+  p.k_pe = static_cast<const __nv_bfloat16 *>(c.k_pe);
+  p.kpe_stride = c.kpe_stride;
+  p.kbuf = static_cast<__nv_bfloat16 *>(a.kbuf);
+  p.vbuf = static_cast<__nv_bfloat16 *>(a.vbuf);
+  p.dev_status = a.dev_status;
+  const dim3 grid((a.max_seqlen + kDcTok - 1) / kDcTok, a.H, a.B);
+  return launch_pdl(decompress_tc_kernel, grid, dim3(128), kDcSmem, st, mc, mwk, mwv, p) == cudaSuccess ? MLA_OK
+                                                                                                    : MLA_ERR_CUDA;
 }
 
 int launch_prefill_tc_attention(const PrefillArgs &a, cudaStream_t st) {
