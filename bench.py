@@ -39,6 +39,7 @@ def _args():
     p.add_argument("--config", default="v3_bf16")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement (single-GPU runs only)")
     return p.parse_args()
 
 
@@ -213,6 +214,57 @@ def run_reference(args):
                              "sample": "each step: " + last["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def measure_prefill(mla, torch, peaks):
+    """The causal prefill (the secondary path row) on its workload: V3 shapes, 2 sequences x 8192 tokens,
+    128 heads, 64-token pages.  Device-side seeded inputs; 1 warm-up and 2 timed calls of mla_prefill."""
+    from workloads import PREFILL_CASES, prefill_flops
+    case = PREFILL_CASES["v3_prefill_bf16"]
+    d = case.dims
+    B, T = len(case.seqlens), sum(case.seqlens)
+    g = torch.Generator(device="cuda").manual_seed(case.seed)
+    dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype)
+    cu = torch.zeros(B + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(case.seqlens, dtype=torch.int32), 0)
+    mbps = max((s_ + case.block_size - 1) // case.block_size for s_ in case.seqlens)
+    num_blocks = B * mbps
+    bt = torch.randperm(num_blocks, generator=torch.Generator().manual_seed(case.seed)).to(torch.int32).view(B, mbps)
+    pool = torch.randn(num_blocks * case.block_size, d.d_c + d.d_rope, generator=g, device="cuda").to(torch.bfloat16)
+    q_nope = torch.randn(T, d.n_heads, d.d_nope, generator=g, device="cuda").to(torch.bfloat16)
+    q_pe = torch.randn(T, d.n_heads, d.d_rope, generator=g, device="cuda").to(torch.bfloat16)
+    w_uk = (torch.randn(d.n_heads, d.d_c, d.d_nope, generator=g, device="cuda") / d.d_c ** 0.5).to(torch.bfloat16)
+    w_uv = (torch.randn(d.n_heads, d.d_c, d.d_v, generator=g, device="cuda") / d.d_c ** 0.5).to(torch.bfloat16)
+    out = torch.empty(T, d.n_heads, d.d_v, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(T, d.n_heads, dtype=torch.float32, device="cuda")
+    ms_ = max(case.seqlens)
+    ws = mla.alloc_workspace(mla.mla_prefill_workspace_size(dims, B, T, ms_))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cu_d, bt_d = cu.cuda(), bt.cuda()
+
+    def run():
+        mla.mla_prefill(dims, cu_d, ms_, q_nope, q_pe, pool, pool[:, d.d_c:], bt_d, mbps, num_blocks, w_uk, w_uv,
+                        out, lse, ws, st)
+
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(2):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the prefill")
+    ms = e0.elapsed_time(e1) / 2
+    fl = prefill_flops(d, list(case.seqlens))
+    t_roof = fl["total"] / (peaks["bf16_tflops"] * 1e12)
+    del q_nope, q_pe, ws, out
+    torch.cuda.empty_cache()
+    return {"workload": "v3_prefill_bf16: causal prefill, 2 x 8192 tokens, 128 heads, keys 192, values 128",
+            "ms": ms, "tflops": fl["total"] / (ms * 1e-3) / 1e12, "flops": fl["total"],
+            "roofline": {"bound": "tensor", "t_us": t_roof * 1e6, "frac": t_roof / (ms * 1e-3),
+                         "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"]}}
 
 
 def run_mla(args):
@@ -420,6 +472,8 @@ def run_mla(args):
         line["e2e"] = {"value": step_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": UNIT,
                        "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                        "ms_per_step": e2e["ms_per_step"]}
+    if world == 1 and rank == 0 and not args.no_prefill:
+        line["prefill"] = measure_prefill(mla, torch, peaks)
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if rank == 0:
