@@ -37,6 +37,48 @@ def test_status_strings():
     assert "unknown" in mla.mla_status_string(-99)
 
 
+def _prototypes():
+    """name -> list of parameter type strings, parsed from include/mla.h."""
+    src = open(os.path.join(ROOT, "include", "mla.h")).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"MLA_API\s+(?:const\s+char\s*\*|int)\s*(mla_\w+)\s*\(([^)]*)\)", src):
+        params = [" ".join(p.split()) for p in m.group(2).split(",")]
+        types = []
+        for p in params:
+            p = re.sub(r"\b\w+$", "", p).strip()         # drop the parameter name
+            types.append(p.replace(" *", "*").replace("* ", "*"))
+        out[m.group(1)] = types
+    return out
+
+
+def _ctype_of(c):
+    """The ctypes class a C parameter type must be marshalled as (width matters on the stack)."""
+    if c.endswith("*") or c == "mla_stream_t":
+        return "ptr"
+    return {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "int64_t": ctypes.c_int64,
+            "long long": ctypes.c_longlong}[c]
+
+
+def test_binding_argtypes_match_header_prototypes():
+    """Every entry point is called with declared argument types of the right count and width
+    (an undeclared 64-bit argument passed on the stack arrives with a garbage upper half)."""
+    import mla_latent_kv_40_b200 as mla
+    protos = _prototypes()
+    assert set(protos) == set(_declared())
+    for name, ctypes_list in protos.items():
+        fn = getattr(mla._lib, name)
+        assert fn.argtypes is not None, name
+        assert len(fn.argtypes) == len(ctypes_list), (name, len(fn.argtypes), len(ctypes_list))
+        for i, (c, got) in enumerate(zip(ctypes_list, fn.argtypes)):
+            want = _ctype_of(c)
+            if want == "ptr":
+                assert got is ctypes.c_void_p or issubclass(got, ctypes._Pointer), (name, i, c, got)
+            else:
+                assert issubclass(got, ctypes._SimpleCType) and ctypes.sizeof(got) == ctypes.sizeof(want), \
+                    (name, i, c, got)
+
+
 def test_dims_struct_matches_header_layout():
     import mla_latent_kv_40_b200 as mla
     assert ctypes.sizeof(mla.mla_dims) == 14 * 4
