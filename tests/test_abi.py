@@ -75,7 +75,7 @@ def test_binding_argtypes_match_header_prototypes():
             if want == "ptr":
                 assert got is ctypes.c_void_p or issubclass(got, ctypes._Pointer), (name, i, c, got)
             else:
-                assert issubclass(got, ctypes._SimpleCType) and ctypes.sizeof(got) == ctypes.sizeof(want), \
+                assert issubclass(got, ctypes._SimpleCData) and ctypes.sizeof(got) == ctypes.sizeof(want), \
                     (name, i, c, got)
 
 
