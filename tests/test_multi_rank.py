@@ -64,6 +64,28 @@ def test_single_process_needs_no_process_group():
     assert abs(bench.weak_scaling_value(1e12, 1, 1.0) - 1000.0) < 1e-9   # 1 TFLOP in 1 ms
 
 
+def test_reference_arm_line_on_rank_zero():
+    """Rank 0 of `bench.py --impl reference` prints one JSON line with the contract's keys; the oracle
+    is the reference arm, so its e2e moves no bytes and its cpu_baseline describes the same run."""
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                          "small_v3_bf16", "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, out.stdout
+    line = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["config"]["workload"].startswith("small_v3_bf16")
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": line["unit"], "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
+
+
 def test_reference_arm_runs_on_rank_zero_only():
     """A non-zero rank of `bench.py --impl reference` exits 0 at once and prints nothing."""
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
