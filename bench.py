@@ -40,6 +40,14 @@ def _args():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-prefill", action="store_true", help="skip the prefill measurement (single-GPU runs only)")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other decode workloads (V2-Lite, V3 ragged, V3 long; single-GPU runs only)")
+    p.add_argument("--repeats", type=int, default=10,
+                   help="extra blocks of --steps steps timed after the headline block, for the spread")
+    p.add_argument("--only", default="all", choices=["all", "decode", "prefill", "configs"],
+                   help="run one part alone (for profiler captures of a single kernel family)")
+    p.add_argument("--prefill-seqlens", default=None,
+                   help="comma-separated prefill sequence lengths instead of the workload's 8192,8192 (profiling)")
     return p.parse_args()
 
 
@@ -216,11 +224,15 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def measure_prefill(mla, torch, peaks):
+def measure_prefill(mla, torch, peaks, seqlens=None, calls=10):
     """The causal prefill (the secondary path row) on its workload: V3 shapes, 2 sequences x 8192 tokens,
-    128 heads, 64-token pages.  Device-side seeded inputs; 1 warm-up and 2 timed calls of mla_prefill."""
+    128 heads, 64-token pages.  Device-side seeded inputs; 2 warm-up calls, then `calls` timed calls of
+    mla_prefill, each bracketed by CUDA events (median and spread reported)."""
+    import dataclasses
     from workloads import PREFILL_CASES, prefill_flops
     case = PREFILL_CASES["v3_prefill_bf16"]
+    if seqlens:
+        case = dataclasses.replace(case, seqlens=tuple(seqlens))
     d = case.dims
     B, T = len(case.seqlens), sum(case.seqlens)
     g = torch.Generator(device="cuda").manual_seed(case.seed)
@@ -246,25 +258,89 @@ def measure_prefill(mla, torch, peaks):
         mla.mla_prefill(dims, cu_d, ms_, q_nope, q_pe, pool, pool[:, d.d_c:], bt_d, mbps, num_blocks, w_uk, w_uv,
                         out, lse, ws, st)
 
-    run()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
     for _ in range(2):
         run()
-    e1.record()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(calls)]
+    for a, b in evs:
+        a.record()
+        run()
+        b.record()
     torch.cuda.synchronize()
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} in the prefill")
-    ms = e0.elapsed_time(e1) / 2
+    times = sorted(a.elapsed_time(b) for a, b in evs)
+    ms = statistics.median(times)
     fl = prefill_flops(d, list(case.seqlens))
     t_roof = fl["total"] / (peaks["bf16_tflops"] * 1e12)
     del q_nope, q_pe, ws, out
     torch.cuda.empty_cache()
-    return {"workload": "v3_prefill_bf16: causal prefill, 2 x 8192 tokens, 128 heads, keys 192, values 128",
-            "ms": ms, "tflops": fl["total"] / (ms * 1e-3) / 1e12, "flops": fl["total"],
+    return {"workload": f"v3_prefill_bf16: causal prefill, {B} x {max(case.seqlens)} tokens, 128 heads, keys 192, "
+                        "values 128",
+            "ms": ms, "ms_min": times[0], "ms_max": times[-1], "calls": calls,
+            "tflops": fl["total"] / (ms * 1e-3) / 1e12, "flops": fl["total"],
             "roofline": {"bound": "tensor", "t_us": t_roof * 1e6, "frac": t_roof / (ms * 1e-3),
                          "peak_tflops": peaks["bf16_tflops"], "peak_source": peaks["source"]}}
+
+
+def measure_decode_configs(mla, torch, peaks, steps, names=("v2lite_bf16", "v3_ragged_bf16", "v3_long_bf16")):
+    """The other decode workloads at full size, each timed through one public call per step
+    (mla_decode: absorb + split-KV attention + combine/W_UV), inputs resident on the device.
+    Reported per workload: TFLOP/s, latent-KV GB/s, decode tokens/s and the fraction of the roofline
+    max(latent bytes / HBM peak, decode FLOPs / bf16 peak)."""
+    from workloads import DECODE_CASES, decode_flops, latent_bytes, make_decode_inputs_device
+    res = {}
+    for name in names:
+        case = DECODE_CASES[name]
+        d = case.dims
+        inp = make_decode_inputs_device(case)
+        tiled = d.dtype == "bf16" and case.block_size % 64 == 0 and (d.d_c + d.d_rope) % 64 == 0
+        dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                             rope_base=d.rope_base, rms_eps=d.rms_eps, cache_layout=1 if tiled else 0)
+        pool = inp["pool"]
+        if tiled:
+            packed = torch.empty_like(pool)
+            mla.mla_cache_pack(dims, pool, packed)
+            torch.cuda.synchronize()
+            del pool
+            inp["pool"] = pool = packed
+        c_kv, k_pe = (pool, pool) if tiled else (pool, pool[:, d.d_c:])
+        B, n_q, H = case.batch, case.n_q, d.n_heads
+        sl = inp["seqlens"]
+        max_seqlen = int(sl.max())
+        bt = inp["block_table"].cuda() if case.paged else None
+        sl_d = sl.cuda()
+        ws = mla.alloc_workspace(mla.mla_decode_workspace_size(dims, B, n_q, max_seqlen))
+        out = torch.empty((B, n_q, H, d.d_v), dtype=d.torch_dtype, device="cuda")
+        lse = torch.empty((B, n_q, H), dtype=torch.float32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+        def run():
+            mla.mla_decode(dims, inp["q_nope"], inp["q_pe"], c_kv, k_pe, bt, inp["max_blocks_per_seq"],
+                           inp["num_blocks"], sl_d, max_seqlen, inp["w_uk"], inp["w_uv"], out, lse, ws, st)
+
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"device status {int(st.item())} in {name}")
+        ms = e0.elapsed_time(e1) / steps
+        fl = decode_flops(d, sl.tolist(), n_q)["total"]
+        lb = latent_bytes(d, sl.tolist())
+        t_roof = max(lb / (peaks["hbm_gbs"] * 1e9), fl / (peaks["bf16_tflops"] * 1e12))
+        res[name] = {"ms": ms, "tflops": fl / (ms * 1e-3) / 1e12, "latent_kv_gbs": lb / (ms * 1e-3) / 1e9,
+                     "decode_tokens_per_s": B * n_q / (ms * 1e-3), "roofline_us": t_roof * 1e6,
+                     "roofline_frac": t_roof / (ms * 1e-3), "batch": B, "n_q": n_q,
+                     "seqlens": list(case.seqlens), "latent_bytes": lb, "flops": fl, "call": "mla_decode"}
+        del inp, pool, c_kv, k_pe, ws, out
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_mla(args):
@@ -277,6 +353,15 @@ def run_mla(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
     import mla_latent_kv_40_b200 as mla
     from workloads import DECODE_CASES, append_flops, decode_flops, latent_bytes, make_decode_step_inputs
+
+    if args.only in ("prefill", "configs"):   # profiling helpers: one kernel family alone, no JSON contract
+        peaks = _peaks()
+        if args.only == "prefill":
+            sl = [int(x) for x in args.prefill_seqlens.split(",")] if args.prefill_seqlens else None
+            print(json.dumps({"prefill": measure_prefill(mla, torch, peaks, sl, calls=max(args.steps, 1))}), flush=True)
+        else:
+            print(json.dumps({"configs": measure_decode_configs(mla, torch, peaks, max(args.steps, 1))}), flush=True)
+        return
 
     case = DECODE_CASES[args.config]
     d = case.dims
@@ -346,20 +431,55 @@ def run_mla(args):
     def max_over_ranks(x):
         return max_over_ranks_of(x, world, "cuda")
 
-    att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    def timed_block():
+        """Exactly --steps steps between a barrier + synchronize on each side: (ms per step, attention ms
+        per launch), each the max over ranks."""
+        att_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
         e0.record(stream)
         for i in range(args.steps):
             step(att_ev[i])
         e1.record(stream)
         torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    att_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in att_ev))
+        barrier()
+        return (max_over_ranks(e0.elapsed_time(e1) / args.steps),
+                max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in att_ev)))
+
+    # The headline block, then --repeats more blocks of the same steps for the spread; the clocks are
+    # sampled across all of them.
+    with ClockSampler(local) as clk:
+        ms, att_ms = timed_block()
+        reps = [timed_block() for _ in range(args.repeats)]
     clocks = clk.summary()
+    all_ms = sorted([ms] + [r[0] for r in reps])
+    all_att = sorted([att_ms] + [r[1] for r in reps])
+
+    # The same step through the single public decode call: append, then mla_decode (absorb + attention +
+    # combine/W_UV in one call) on one stream.
+    dec_ws = mla.alloc_workspace(mla.mla_decode_workspace_size(dims, B, n_q, max_seqlen))
+
+    def api_step():
+        mla.mla_append_latent(dims, dev["h_new"], dev["w_dkv"], dev["w_kr"], dev["gamma"], dev["seq_idx"],
+                              dev["pos"], c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status,
+                              workspace=app_ws)
+        mla.mla_decode(dims, dev["q_nope"], dev["q_pe"], c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
+                       dev["seqlens"], max_seqlen, dev["w_uk"], dev["w_uv"], out, lse, dec_ws, status)
+
+    for _ in range(3):
+        api_step()
+    torch.cuda.synchronize()
+    barrier()
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    for _ in range(args.steps):
+        api_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    api_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
 
     # End to end through the public calls: pinned host inputs in, result out, every step's copies inside the
     # timed region.  The inputs of step i+1 are copied (copy stream) while step i computes, into the other of
@@ -461,19 +581,32 @@ def run_mla(args):
                                   "peaks, over the whole step time"},
         "roofline": {"kernel": "split-KV attention (mla_decode_attention)", "bound": "hbm",
                      "achieved": att_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": att_gbs / peaks["hbm_gbs"],
-                     "traffic": _traffic_for("decode_tc.cu" if mla.mla_decode_launches(dims, n_q) != 3 else
-                                             "attn_simt.cu"),
+                     "traffic": _traffic_for("decode_tc.cu" if mla.mla_decode_path(dims, n_q) == mla.PATH_TCGEN05
+                                             else "attn_simt.cu"),
                      "peak_source": peaks["source"], "kernel_ms": att_ms,
                      "algorithmic_bytes_per_launch": lat_bytes},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "spread": {"blocks": len(all_ms), "steps_per_block": args.steps,
+                   "ms_per_step_median": statistics.median(all_ms), "ms_per_step_min": all_ms[0],
+                   "ms_per_step_max": all_ms[-1], "attention_ms_median": statistics.median(all_att),
+                   "attention_ms_min": all_att[0], "attention_ms_max": all_att[-1],
+                   "attention_frac_median": lat_bytes / (statistics.median(all_att) * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+        "api_step": {"calls": "mla_append_latent + mla_decode, one stream", "ms_per_step": api_ms,
+                     "tflops": step_flops * world / (api_ms * 1e-3) / 1e12,
+                     "roofline_frac": max(t_hbm, t_flop) / (api_ms * 1e-3)},
     }
     if e2e:
         line["e2e"] = {"value": step_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": UNIT,
                        "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                        "ms_per_step": e2e["ms_per_step"]}
-    if world == 1 and rank == 0 and not args.no_prefill:
+    del dec_ws
+    if world == 1 and rank == 0 and not args.no_prefill and args.only == "all":
         line["prefill"] = measure_prefill(mla, torch, peaks)
+    if world == 1 and rank == 0 and not args.no_configs and args.only == "all":
+        del dev, pool, c_kv, k_pe, ws
+        torch.cuda.empty_cache()
+        line["configs"] = measure_decode_configs(mla, torch, peaks, max(args.steps, 5))
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if rank == 0:

@@ -25,8 +25,14 @@
  *    bounded wait that timed out) are written to *dev_status (if non-NULL) with
  *    an atomic compare-and-swap from 0, so the first error wins; the caller
  *    zeroes it beforehand and reads it after synchronising.
- *  - The library keeps no mutable global state; concurrent calls on different
- *    streams with disjoint outputs and workspaces are safe.
+ *  - Concurrent calls on different streams with disjoint outputs and
+ *    workspaces are safe, with one exception: mla_decode_noalloc, whose calls
+ *    share one library-owned scratch buffer per GPU (see there).  Besides that
+ *    buffer, the library's only global state is per-device host-side caches
+ *    filled on first use and read-only afterwards: the number of attention
+ *    clusters that fit on the device, the driver's tensor-map encoder, and the
+ *    device address of the no-allocation scratch buffer.  Each is guarded, so
+ *    first calls from several host threads are safe.
  *  - There is no CPU fallback: a shape the CUDA kernels do not handle returns
  *    MLA_ERR_UNSUPPORTED.
  *
@@ -270,6 +276,17 @@ MLA_API int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, 
  *   profilers and benchmarks.  Writes *count; no device work.
  */
 MLA_API int mla_decode_launches(const mla_dims *dims, int n_q, int *count);
+
+/*
+ * mla_decode_path — which kernels mla_decode / mla_decode_attention run for
+ *   this shape: MLA_PATH_TCGEN05 (the tensor-core split-KV kernel and its
+ *   combine: bf16, d_c 512, d_R 64, d_v 128, 64-token-multiple pages,
+ *   n_q * H <= 256) or MLA_PATH_CUDA_CORES (fp32 and every other shape).
+ *   Host-side logic only; no device work.  Writes *path.
+ */
+#define MLA_PATH_CUDA_CORES 0
+#define MLA_PATH_TCGEN05 1
+MLA_API int mla_decode_path(const mla_dims *dims, int n_q, int *path);
 
 /*
  * mla_cache_pack / mla_cache_unpack — convert a latent pool between the row

@@ -65,6 +65,7 @@ _sigs = {
     "mla_decode_combine": [_D, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_prefill_workspace_size": [_D, _I, _I, _I, _SZ],
     "mla_decode_launches": [_D, _I, ctypes.POINTER(ctypes.c_int)],
+    "mla_decode_path": [_D, _I, ctypes.POINTER(ctypes.c_int)],
     "mla_cache_pack": [_D, _P, _P, ctypes.c_int64, _P],
     "mla_cache_unpack": [_D, _P, _P, ctypes.c_int64, _P],
     "mla_decode_noalloc": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P],
@@ -241,6 +242,16 @@ def mla_decode_combine(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, worksp
 def mla_decode_launches(dims, n_q) -> int:
     n = ctypes.c_int(0)
     _check("mla_decode_launches", _lib.mla_decode_launches(ctypes.byref(dims), int(n_q), ctypes.byref(n)))
+    return int(n.value)
+
+
+PATH_CUDA_CORES, PATH_TCGEN05 = 0, 1   # MLA_PATH_* in include/mla.h
+
+
+def mla_decode_path(dims, n_q) -> int:
+    """PATH_TCGEN05 when mla_decode runs the tensor-core kernels for this shape, else PATH_CUDA_CORES."""
+    n = ctypes.c_int(-1)
+    _check("mla_decode_path", _lib.mla_decode_path(ctypes.byref(dims), int(n_q), ctypes.byref(n)))
     return int(n.value)
 
 

@@ -267,6 +267,12 @@ int mla_decode_launches(const mla_dims *dims, int n_q, int *count) {
   return MLA_OK;
 }
 
+int mla_decode_path(const mla_dims *dims, int n_q, int *path) {
+  if (!dims_ok(dims) || n_q <= 0 || !path) return MLA_ERR_INVALID_ARG;
+  *path = tc_decode_supported(*dims, n_q) ? MLA_PATH_TCGEN05 : MLA_PATH_CUDA_CORES;
+  return MLA_OK;
+}
+
 int mla_prefill_workspace_size(const mla_dims *dims, int B, int total_tokens, int max_seqlen,
                                size_t *bytes) {
   if (!dims_ok(dims) || B <= 0 || total_tokens <= 0 || max_seqlen <= 0 || !bytes)

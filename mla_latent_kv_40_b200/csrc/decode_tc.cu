@@ -36,6 +36,7 @@
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -1130,16 +1131,21 @@ WsLayout ws_layout(int B, int n_rb) {
   return L;
 }
 
-// Clusters of two CTAs that fit on the current device at once (0 without a device).
+// Clusters of two CTAs that fit on the current device at once (0 without a device).  The
+// answer is cached per device; the first query on a device computes it under a mutex, so
+// concurrent first calls from several host threads are safe.
 int clusters_for_device() {
-  static int cached[128] = {0};
+  static std::atomic<int> cached[128];
+  static std::mutex mu;
   int dev = 0, ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev <= 0) {
     cudaGetLastError();
     return 0;
   }
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 0;
-  if (cached[dev]) return cached[dev];
+  if (const int c = cached[dev].load(std::memory_order_acquire)) return c;
+  std::lock_guard<std::mutex> lock(mu);
+  if (const int c = cached[dev].load(std::memory_order_acquire)) return c;
   if (cudaFuncSetAttribute(mla_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes))
     return 0;
   // One CTA of kThreads per SM needs at most kLaunchRegs registers per thread.
@@ -1164,7 +1170,7 @@ int clusters_for_device() {
     n = sms / 2;
   }
   if (n > kMaxClusters) n = kMaxClusters;
-  cached[dev] = n;
+  cached[dev].store(n, std::memory_order_release);
   return n;
 }
 

@@ -154,3 +154,38 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_decode_path_query():
+    """mla_decode_path is host logic: the V3 and V2-Lite bf16 shapes take the tensor-core kernels,
+    the fp32 shapes the CUDA-core kernels (no GPU needed)."""
+    import mla_latent_kv_40_b200 as mla
+    from workloads import DECODE_CASES
+    for name, want in (("v3_bf16", mla.PATH_TCGEN05), ("v2lite_bf16", mla.PATH_TCGEN05),
+                       ("v3_ragged_bf16", mla.PATH_TCGEN05), ("tiny_fp32", mla.PATH_CUDA_CORES),
+                       ("small_f32_nq2", mla.PATH_CUDA_CORES)):
+        case = DECODE_CASES[name]
+        d = case.dims
+        for layout in ((0, 1) if d.dtype == "bf16" else (0,)):
+            dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                                 cache_layout=layout)
+            assert mla.mla_decode_path(dims, case.n_q) == want, (name, layout)
+    with pytest.raises(mla.MlaError):
+        mla.mla_decode_path(mla.make_dims(8, 64, 16, 32, 32, 256, 0, "f32"), 1)   # block_size 0
+
+
+def test_bench_picks_the_traffic_entry_of_the_kernel_that_runs():
+    """The bench's DRAM-traffic figure for the V3 batch-64 step is keyed by the tensor-core attention
+    kernel's source file, which is what mla_decode_path reports for that shape."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import mla_latent_kv_40_b200 as mla
+    from workloads import DECODE_CASES
+    case = DECODE_CASES["v3_bf16"]
+    d = case.dims
+    dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                         cache_layout=1)
+    key = "decode_tc.cu" if mla.mla_decode_path(dims, case.n_q) == mla.PATH_TCGEN05 else "attn_simt.cu"
+    assert key == "decode_tc.cu"
+    assert key in bench._TRAFFIC_SOURCES

@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from workloads import DECODE_CASES, make_decode_inputs
 from helpers import check_close, dims_of, gpu_decode
 
@@ -37,12 +38,17 @@ def test_noalloc_matches_workspace_entry_point_twice(lib, name):
     inp = make_decode_inputs(DECODE_CASES[name])
     ref, ref_lse, st = gpu_decode(lib, inp)
     assert st == 0
+    # The fp64 oracle on the same inputs, so the no-allocation path is held to the same bar as mla_decode.
+    o_ref, o_lse = oracle.decode(inp["dims"], inp["q_nope"], inp["q_pe"], inp["pool"], inp["block_table"],
+                                 inp["block_size"], inp["seqlens"], inp["w_uk"], inp["w_uv"])
+    tol = 1e-4 if inp["dims"].dtype == "f32" else 3e-2
     for _ in range(2):            # the second call reuses the scratch the first one left behind
         out, lse, st = _noalloc(lib, inp)
         assert st == 0
-        check_close(out, ref, inp["dims"].dtype, name + " noalloc")
-        tol = 1e-4 if inp["dims"].dtype == "f32" else 3e-2
+        check_close(out, ref, inp["dims"].dtype, name + " noalloc vs mla_decode")
         assert np.max(np.abs(lse - ref_lse)) <= tol
+        check_close(out, o_ref, inp["dims"].dtype, name + " noalloc vs oracle")
+        assert np.max(np.abs(lse - o_lse)) <= tol
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(lib):

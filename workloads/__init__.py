@@ -23,6 +23,7 @@ __all__ = [
     "Dims", "DecodeCase", "PrefillCase", "DECODE_CASES", "PREFILL_CASES",
     "make_decode_inputs", "make_prefill_inputs", "make_append_inputs",
     "cache_row_of", "latent_bytes", "decode_flops", "prefill_flops", "make_decode_step_inputs", "append_flops",
+    "make_decode_inputs_device",
 ]
 
 
@@ -330,3 +331,31 @@ def make_decode_step_inputs(case: DecodeCase, fill: str = "random") -> dict:
 def append_flops(dims: Dims, T: int) -> int:
     """FLOPs of appending T tokens: the [T, D] x [D, d_c + d_R] projection."""
     return 2 * T * dims.d_model * (dims.d_c + dims.d_rope)
+
+
+def make_decode_inputs_device(case: DecodeCase, device="cuda") -> dict:
+    """The inputs of ``make_decode_inputs`` for timing runs at full size, drawn on the device.
+
+    Sequence lengths and the block table come from the same CPU generator and
+    seed as ``make_decode_inputs`` (the same structure); the values (cache rows,
+    queries, weights) come from a device generator seeded with the case seed, so
+    they are not the CPU draws' bits but follow the same distributions.  Unused
+    pool rows hold NaN.
+    """
+    d = case.dims
+    gen = torch.Generator().manual_seed(case.seed)
+    seqlens = case.draw_seqlens(gen)
+    bt, num_blocks, mbps = _block_table(gen, seqlens, case.block_size, case.paged, spare_blocks=2 if case.paged else 0)
+    W = d.latent_width
+    dt = d.torch_dtype
+    g = torch.Generator(device=device).manual_seed(case.seed)
+    pool = torch.full((num_blocks * case.block_size, W), float("nan"), dtype=dt, device=device)
+    rows = torch.cat([_rows_of(bt, case.block_size, b, int(seqlens[b])) for b in range(case.batch)]).to(device)
+    pool[rows] = torch.randn(rows.numel(), W, generator=g, device=device).to(dt)
+    q_nope = torch.randn(case.batch, case.n_q, d.n_heads, d.d_nope, generator=g, device=device).to(dt)
+    q_pe = torch.randn(case.batch, case.n_q, d.n_heads, d.d_rope, generator=g, device=device).to(dt)
+    w_uk = (torch.randn(d.n_heads, d.d_c, d.d_nope, generator=g, device=device) / math.sqrt(d.d_c)).to(dt)
+    w_uv = (torch.randn(d.n_heads, d.d_c, d.d_v, generator=g, device=device) / math.sqrt(d.d_c)).to(dt)
+    return dict(case=case, dims=d, seqlens=seqlens, block_table=bt, num_blocks=num_blocks,
+                max_blocks_per_seq=mbps, block_size=case.block_size, pool=pool,
+                q_nope=q_nope, q_pe=q_pe, w_uk=w_uk, w_uv=w_uv)
