@@ -209,6 +209,56 @@ def decode(dims, q_nope, q_pe, pool, block_table, block_size: int, seqlens, w_uk
     return out, lse
 
 
+# ---------------------------------------------------------------- sparse decode over selected tokens
+
+def decode_sparse(dims, q_nope, q_pe, pool, block_table, block_size: int, seqlens, topk_idx, w_uk, w_uv,
+                  picks=None):
+    """Decode step in unabsorbed form over a selected subset of each query token's cached tokens.
+
+    The MQA-mode MLA of V3.2 (developer.cloud.tencent.com search results for
+    "MLA", the snippet "MHA版MLA VS MQA版MLA": every head attends to the one
+    shared latent key/value) restricted, for query token j of sequence b, to
+    the cached tokens listed in topk_idx[b, j, :].  Entries equal to -1 are
+    padding; every other entry is a token index in 0 .. S_b - n_q + j (the
+    causal limit of that query token).  The listed tokens are attended to as
+    listed: z_i = scale * q . k_i over the list, softmax over the list,
+    output sum_i p_i v_i, per head, with keys and values decompressed from the
+    cache exactly as in ``decode``.
+
+    topk_idx [B, n_q, k] (int).  Returns (out [B, n_q, H, d_v], lse [B, n_q, H])
+    as float64; with ``picks`` = list of (b, j, s) only those entries are computed.
+    """
+    q_nope = _f64(q_nope)
+    q_pe = _f64(q_pe)
+    w_uk = _f64(w_uk)
+    w_uv = _f64(w_uv)
+    sl = _i64(seqlens)
+    idx = _i64(topk_idx)
+    bt = _i64(block_table)
+    B, n_q, H, _ = q_nope.shape
+    out = np.full((B, n_q, H, dims.d_v), np.nan)
+    lse = np.full((B, n_q, H), np.nan)
+    if picks is None:
+        picks = [(b, j, s) for b in range(B) for s in range(H) for j in range(n_q)]
+    scale = 1.0 / math.sqrt(dims.d_nope + dims.d_rope)
+    for (b, j, s) in picks:
+        p_j = int(sl[b]) - n_q + j
+        listed = [int(i) for i in idx[b, j] if int(i) != -1]
+        if not listed or min(listed) < 0 or max(listed) > p_j:
+            raise ValueError(f"selection of ({b}, {j}) must be non-empty and within 0..{p_j}")
+        tok = np.asarray(listed, dtype=np.int64)
+        rows = bt[b, tok // block_size] * block_size + tok % block_size
+        if hasattr(pool, "detach"):
+            import torch
+            sel = _f64(pool[torch.from_numpy(rows)])
+        else:
+            sel = _f64(np.asarray(pool)[rows])
+        K, V = decompress_head(sel[:, :dims.d_c], sel[:, dims.d_c:dims.d_c + dims.d_rope], w_uk[s], w_uv[s])
+        q = np.concatenate([q_nope[b, j, s], rope_rotate(q_pe[b, j, s], p_j, dims.rope_base)])
+        out[b, j, s], lse[b, j, s], _ = attend(q, K, V, len(listed), scale)
+    return out, lse
+
+
 # ---------------------------------------------------------------- prefill (decompressed MHA form)
 
 def prefill(dims, q_nope, q_pe, pool, block_table, block_size: int, cu_seqlens, w_uk, w_uv,

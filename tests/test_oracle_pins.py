@@ -391,3 +391,129 @@ def test_planted_wrong_scale_is_caught(monkeypatch):
     def wrong(q, K, V, n_visible, scale):
         return orig(q, K, V, n_visible, scale * 2.0)
     _assert_some_pin_fails(monkeypatch, "attend", wrong, [test_decode_brute_force_tiny])
+
+
+# ------------------------------------------------------------------ sparse decode over selected tokens
+
+def _sparse_tiny_inputs(seed):
+    r = _rng(seed)
+    d = TINY
+    S, n_q = 6, 2
+    pool = r.standard_normal((8, d.d_c + d.d_rope))
+    bt = np.array([[3, 1, 2]])       # block size 2: tokens 0,1 -> rows 6,7; 2,3 -> rows 2,3; 4,5 -> rows 4,5
+    q_nope = r.standard_normal((1, n_q, d.n_heads, d.d_nope))
+    q_pe = r.standard_normal((1, n_q, d.n_heads, d.d_rope))
+    w_uk = r.standard_normal((d.n_heads, d.d_c, d.d_nope))
+    w_uv = r.standard_normal((d.n_heads, d.d_c, d.d_v))
+    return d, S, n_q, pool, bt, q_nope, q_pe, w_uk, w_uv
+
+
+def test_sparse_decode_brute_force_tiny():
+    """Two query tokens at positions 4 and 5, each with its own selection (padding included):
+    pure-Python loops over the listed tokens only, RoPE at the query's own position."""
+    d, S, n_q, pool, bt, q_nope, q_pe, w_uk, w_uv = _sparse_tiny_inputs(21)
+    sel = np.array([[[4, -1, 0, 2], [5, 1, -1, 3]]])
+    out, lse = O.decode_sparse(d, q_nope, q_pe, pool, bt, 2, np.array([S]), sel, w_uk, w_uv)
+    row_of = {0: 6, 1: 7, 2: 2, 3: 3, 4: 4, 5: 5}
+    for j in range(n_q):
+        p = S - n_q + j
+        toks = [t for t in sel[0, j] if t != -1]
+        for s in range(d.n_heads):
+            qr = [q_pe[0, j, s, 0] * math.cos(p) - q_pe[0, j, s, 1] * math.sin(p),
+                  q_pe[0, j, s, 0] * math.sin(p) + q_pe[0, j, s, 1] * math.cos(p)]
+            zs, vs = [], []
+            for t in toks:
+                row = pool[row_of[t]]
+                c = row[:4]
+                kn = [sum(c[x] * w_uk[s][x][y] for x in range(4)) for y in range(3)]
+                z = sum(q_nope[0, j, s, y] * kn[y] for y in range(3)) + qr[0] * row[4] + qr[1] * row[5]
+                zs.append(z / math.sqrt(5))
+                vs.append([sum(c[x] * w_uv[s][x][y] for x in range(4)) for y in range(3)])
+            den = sum(math.exp(z) for z in zs)
+            for y in range(3):
+                want = sum(math.exp(zs[i]) * vs[i][y] for i in range(len(toks))) / den
+                assert abs(out[0, j, s, y] - want) < 1e-12
+            assert abs(lse[0, j, s] - math.log(den)) < 1e-12
+
+
+def test_sparse_decode_full_selection_is_dense_decode():
+    """Selecting every token up to each query's causal limit, in order, is the dense decode."""
+    inp = make_decode_inputs(DECODE_CASES["small_f32_nq2"])
+    B, n_q, H = inp["q_nope"].shape[:3]
+    sl = inp["seqlens"].numpy()
+    k = int(sl.max())
+    sel = np.full((B, n_q, k), -1, dtype=np.int64)
+    for b in range(B):
+        for j in range(n_q):
+            p = int(sl[b]) - n_q + j
+            sel[b, j, :p + 1] = np.arange(p + 1)
+    args = (inp["dims"], inp["q_nope"], inp["q_pe"], inp["pool"], inp["block_table"], inp["block_size"], inp["seqlens"])
+    o1, l1 = oracle.decode_sparse(*args, sel, inp["w_uk"], inp["w_uv"])
+    o2, l2 = oracle.decode(*args, inp["w_uk"], inp["w_uv"])
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=1e-12)
+
+
+def test_sparse_decode_is_a_set_function_and_ignores_padding():
+    """Softmax over a set: shuffling the listed tokens and moving the padding changes nothing."""
+    d, S, n_q, pool, bt, q_nope, q_pe, w_uk, w_uv = _sparse_tiny_inputs(22)
+    a = np.array([[[0, 2, 4, -1, -1], [1, 3, 5, 0, -1]]])
+    b = np.array([[[-1, 4, -1, 0, 2], [-1, 5, 0, 3, 1]]])
+    o1, l1 = oracle.decode_sparse(d, q_nope, q_pe, pool, bt, 2, np.array([S]), a, w_uk, w_uv)
+    o2, l2 = oracle.decode_sparse(d, q_nope, q_pe, pool, bt, 2, np.array([S]), b, w_uk, w_uv)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, rtol=1e-13)
+
+
+def test_sparse_decode_single_token_returns_its_value_row():
+    """One listed token: its softmax weight is exactly 1, so the output is that token's
+    value c W_UV and the lse is its scaled logit."""
+    d, S, n_q, pool, bt, q_nope, q_pe, w_uk, w_uv = _sparse_tiny_inputs(23)
+    sel = np.array([[[3], [2]]])
+    out, lse = oracle.decode_sparse(d, q_nope, q_pe, pool, bt, 2, np.array([S]), sel, w_uk, w_uv)
+    row_of = {2: 2, 3: 3}
+    for j, t in ((0, 3), (1, 2)):
+        c = pool[row_of[t]][:4]
+        for s in range(d.n_heads):
+            np.testing.assert_allclose(out[0, j, s], c @ w_uv[s], rtol=1e-13, atol=1e-14)
+
+
+def test_sparse_decode_rejects_tokens_past_the_causal_limit():
+    d, S, n_q, pool, bt, q_nope, q_pe, w_uk, w_uv = _sparse_tiny_inputs(24)
+    with pytest.raises(ValueError):
+        oracle.decode_sparse(d, q_nope, q_pe, pool, bt, 2, np.array([S]), np.array([[[5], [5]]]), w_uk, w_uv)
+    with pytest.raises(ValueError):
+        oracle.decode_sparse(d, q_nope, q_pe, pool, bt, 2, np.array([S]), np.array([[[-1], [1]]]), w_uk, w_uv)
+
+
+def _sparse_variant(mistake):
+    """decode_sparse rewritten with one planted mistake: "position" rotates the query by the list
+    length instead of its position; "prefix" attends to the first tokens instead of the listed ones."""
+    def run(dims, q_nope, q_pe, pool, block_table, block_size, seqlens, topk_idx, w_uk, w_uv, picks=None):
+        q_nope, q_pe, pool = np.asarray(q_nope, float), np.asarray(q_pe, float), np.asarray(pool, float)
+        B, n_q, H, _ = q_nope.shape
+        out = np.full((B, n_q, H, dims.d_v), np.nan)
+        lse = np.full((B, n_q, H), np.nan)
+        for b in range(B):
+            for j in range(n_q):
+                listed = [int(i) for i in topk_idx[b, j] if int(i) != -1]
+                p = int(seqlens[b]) - n_q + j
+                if mistake == "prefix":
+                    listed = list(range(len(listed)))
+                if mistake == "position":
+                    p = len(listed) - 1
+                tok = np.asarray(listed)
+                rows = np.asarray(block_table)[b, tok // block_size] * block_size + tok % block_size
+                for s in range(H):
+                    K, V = O.decompress_head(pool[rows, :dims.d_c], pool[rows, dims.d_c:], w_uk[s], w_uv[s])
+                    q = np.concatenate([q_nope[b, j, s], O.rope_rotate(q_pe[b, j, s], p, dims.rope_base)])
+                    out[b, j, s], lse[b, j, s], _ = O.attend(q, K, V, len(listed),
+                                                             1 / math.sqrt(dims.d_nope + dims.d_rope))
+        return out, lse
+    return run
+
+
+@pytest.mark.parametrize("mistake", ["position", "prefix"])
+def test_planted_sparse_mistakes_are_caught(monkeypatch, mistake):
+    _assert_some_pin_fails(monkeypatch, "decode_sparse", _sparse_variant(mistake),
+                           [test_sparse_decode_brute_force_tiny])
