@@ -247,6 +247,36 @@ MLA_API int mla_decode_noalloc(const mla_dims *dims, int B, int n_q, const void 
                                mla_stream_t stream);
 
 /*
+ * mla_decode_sparse_workspace_size — scratch bytes of mla_decode_sparse for B
+ *   sequences of n_q query tokens with lists of topk entries.
+ */
+MLA_API int mla_decode_sparse_workspace_size(const mla_dims *dims, int B, int n_q, int topk, size_t *bytes);
+
+/*
+ * mla_decode_sparse — the decode of mla_decode restricted, per query token, to a
+ *   selected subset of its sequence's cached tokens.
+ *   The MQA-mode MLA that V3.2 moved to (developer.cloud.tencent.com search
+ *   results for "MLA", the snippet "MHA版MLA VS MQA版MLA": every head attends to
+ *   the one shared latent key/value), with the attended tokens chosen per query
+ *   token by the caller (the selection itself is not computed here).
+ *   topk_idx [B, n_q, topk] (int32, device): the token indices query token j of
+ *   sequence b attends to.  -1 is padding.  Every other entry must lie in
+ *   0 .. seqlens[b] - n_q + j (the query's causal limit) and its block id in
+ *   [0, num_blocks); entries that do not are reported as MLA_ERR_BAD_INDEX and
+ *   skipped.  The valid entries are attended to as listed (softmax over the
+ *   list, no deduplication); a query token with none reports MLA_ERR_BAD_INDEX
+ *   and gets zeros.  The query's RoPE position is its own, seqlens[b] - n_q + j.
+ *   Other arguments and outputs as mla_decode.  workspace: >=
+ *   mla_decode_sparse_workspace_size bytes, 256-byte aligned; it holds the
+ *   gathered rows (topk rows per query token, rounded up to 64).
+ */
+MLA_API int mla_decode_sparse(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                              const void *c_kv, const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
+                              int num_blocks, const int32_t *seqlens, int max_seqlen, const int32_t *topk_idx,
+                              int topk, const void *w_uk, const void *w_uv, void *out, float *lse, void *workspace,
+                              size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
  * mla_prefill_workspace_size — scratch bytes of mla_prefill for total_tokens
  *   query tokens in B sequences of at most max_seqlen tokens.
  */

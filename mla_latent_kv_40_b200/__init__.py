@@ -64,6 +64,9 @@ _sigs = {
     "mla_decode_attention": [_D, _I, _I, _P, _P, _P, _P, _I, _I, _P, _I, _P, ctypes.c_size_t, _P, _P],
     "mla_decode_combine": [_D, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_prefill_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode_sparse_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode_sparse": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P, _P,
+                          ctypes.c_size_t, _P, _P],
     "mla_decode_launches": [_D, _I, ctypes.POINTER(ctypes.c_int)],
     "mla_decode_path": [_D, _I, ctypes.POINTER(ctypes.c_int)],
     "mla_cache_pack": [_D, _P, _P, ctypes.c_int64, _P],
@@ -205,6 +208,35 @@ def mla_decode_noalloc(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_p
                                  _ptr(lse, torch.float32, "lse", True), _ptr(dev_status, torch.int32, "dev_status", True),
                                  _stream(stream))
     _check("mla_decode_noalloc", rc)
+
+
+def mla_decode_sparse_workspace_size(dims, B, n_q, topk) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_decode_sparse_workspace_size",
+           _lib.mla_decode_sparse_workspace_size(ctypes.byref(dims), int(B), int(n_q), int(topk), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_sparse(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                      max_seqlen, topk_idx, w_uk, w_uv, out, lse, workspace, dev_status=None, stream=None):
+    """topk_idx [B, n_q, topk] int32: the token indices each query token attends to (-1 = padding)."""
+    et = _elem_dtype(dims)
+    B, n_q = q_nope.shape[0], q_nope.shape[1]
+    for n, t in (("q_nope", q_nope), ("q_pe", q_pe), ("block_table", block_table), ("seqlens", seqlens),
+                 ("topk_idx", topk_idx), ("w_uk", w_uk), ("w_uv", w_uv), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    if topk_idx.dim() != 3 or tuple(topk_idx.shape[:2]) != (B, n_q):
+        raise ValueError("topk_idx must be [B, n_q, topk]")
+    rc = _lib.mla_decode_sparse(ctypes.byref(dims), B, n_q, _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"),
+                                _ptr(c_kv, et, "c_kv"), _ptr(k_pe, et, "k_pe"),
+                                _ptr(block_table, torch.int32, "block_table", True), int(max_blocks_per_seq),
+                                int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"), int(max_seqlen),
+                                _ptr(topk_idx, torch.int32, "topk_idx"), int(topk_idx.shape[2]),
+                                _ptr(w_uk, et, "w_uk"), _ptr(w_uv, et, "w_uv"), _ptr(out, et, "out"),
+                                _ptr(lse, torch.float32, "lse", True), _ptr(workspace, None, "workspace"),
+                                ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_decode_sparse", rc)
 
 
 def mla_decode_latent(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,

@@ -133,9 +133,85 @@ int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const 
   return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, ws, dev_status, st);
 }
 
+// Sparse decode: the gathered pool holds B * n_q short "sequences" (one per query token) of
+// 64-token pages, in the tiled layout where the tensor-core path takes the shape, else fused rows.
+struct SparseLayout {
+  mla_dims inner;               // dims of the gathered pool and of the attention over it
+  int units, pages;             // B * n_q query tokens, pages per token
+  size_t counts_off, pool_off, dec_off, total;
+  DecodeLayout dec;             // decode workspace of the inner call (B * n_q sequences, one query each)
+};
+
+SparseLayout sparse_layout(const mla_dims *d, int B, int n_q, int topk) {
+  SparseLayout L{};
+  L.inner = *d;
+  L.inner.block_size = 64;
+  const int W = d->d_c + d->d_rope;
+  const bool tiled = d->dtype == MLA_BF16 && W % 64 == 0;
+  L.inner.cache_layout = tiled ? MLA_CACHE_TILED : MLA_CACHE_ROWS;
+  L.inner.ckv_stride = L.inner.kpe_stride = W;
+  L.units = B * n_q;
+  L.pages = (topk + 63) / 64;
+  L.counts_off = 0;
+  L.pool_off = align256((size_t)L.units * sizeof(int32_t));
+  L.dec_off = L.pool_off + align256((size_t)L.units * L.pages * 64 * W * elem(d));
+  L.dec = decode_layout(&L.inner, L.units, 1, L.pages * 64);
+  L.total = L.dec_off + L.dec.total;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mla_decode_sparse_workspace_size(const mla_dims *dims, int B, int n_q, int topk, size_t *bytes) {
+  if (!dims_ok(dims) || B <= 0 || n_q <= 0 || topk <= 0 || !bytes) return MLA_ERR_INVALID_ARG;
+  if (dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  *bytes = sparse_layout(dims, B, n_q, topk).total;
+  return MLA_OK;
+}
+
+int mla_decode_sparse(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe, const void *c_kv,
+                      const void *k_pe, const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                      const int32_t *seqlens, int max_seqlen, const int32_t *topk_idx, int topk, const void *w_uk,
+                      const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes, int *dev_status,
+                      mla_stream_t stream) {
+  if (!dims_ok(dims) || B <= 0 || n_q <= 0 || topk <= 0 || max_seqlen < n_q || max_blocks_per_seq <= 0 ||
+      num_blocks <= 0)
+    return MLA_ERR_INVALID_ARG;
+  if (!q_nope || (!q_pe && dims->d_rope) || !c_kv || (!k_pe && dims->d_rope && dims->cache_layout == MLA_CACHE_ROWS) ||
+      !seqlens || !topk_idx || !w_uk || !w_uv || !out)
+    return MLA_ERR_INVALID_ARG;
+  if ((int64_t)max_blocks_per_seq * dims->block_size < max_seqlen) return MLA_ERR_INVALID_ARG;
+  if (dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  const SparseLayout L = sparse_layout(dims, B, n_q, topk);
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts_off);
+  char *pool = ws + L.pool_off;
+  char *dws = ws + L.dec_off;
+  // (1) Query absorption at each token's own position (the real sequence lengths).
+  void *qbuf = dws + L.dec.q_off;
+  AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
+                q_nope, q_pe, w_uk, seqlens, qbuf, dims->rope_base};
+  int rc = absorb_dispatch(ab, dims->dtype == MLA_BF16, dev_status, st);
+  if (rc) return rc;
+  // (2) The listed rows of every query token into its own pages of the gathered pool.
+  CacheView src{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq, num_blocks,
+                dims->block_size, dims->cache_layout, dims->d_c, dims->d_c + dims->d_rope};
+  if ((rc = launch_sparse_gather(B, n_q, topk, topk_idx, seqlens, max_seqlen, src, pool,
+                                 L.inner.cache_layout == MLA_CACHE_TILED, (int)elem(dims), counts, dev_status, st)))
+    return rc;
+  // (3) + (4) Attention over the gathered pool (every listed key visible to its own query) and combine.
+  const mla_dims *in = &L.inner;
+  const int W = dims->d_c + dims->d_rope;
+  if ((rc = attention_impl(in, L.units, 1, qbuf, pool, pool + (size_t)dims->d_c * elem(dims), nullptr, L.pages,
+                           L.units * L.pages, counts, L.pages * 64, L.dec, dws, dev_status, st)))
+    return rc;
+  (void)W;
+  return combine_impl(in, L.units, 1, counts, L.pages * 64, w_uv, out, lse, L.dec, dws, dev_status, st);
+}
 
 const char *mla_status_string(int s) {
   switch (s) {

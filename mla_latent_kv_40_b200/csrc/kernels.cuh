@@ -122,5 +122,9 @@ bool append_tc_supported(const AppendArgs &a, bool bf16);
 int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split, cudaStream_t st);
 int launch_append_finish(const AppendArgs &a, const void *ws, int nsplit, cudaStream_t st);
 int launch_cache_convert(const void *src, void *dst, int64_t num_rows, int W, bool to_tiled, cudaStream_t st);
+// Sparse decode: compact each query token's listed cache rows into its own run of 64-token pages.
+int launch_sparse_gather(int B, int n_q, int topk, const int32_t *idx, const int32_t *seqlens, int max_seqlen,
+                         const CacheView &src, void *pool, bool dst_tiled, int elem, int32_t *counts,
+                         int *dev_status, cudaStream_t st);
 
 }  // namespace mla

@@ -189,3 +189,18 @@ def test_bench_picks_the_traffic_entry_of_the_kernel_that_runs():
     key = "decode_tc.cu" if mla.mla_decode_path(dims, case.n_q) == mla.PATH_TCGEN05 else "attn_simt.cu"
     assert key == "decode_tc.cu"
     assert key in bench._TRAFFIC_SOURCES
+
+
+def test_sparse_decode_host_validation():
+    """mla_decode_sparse rejects a missing selection and a non-positive topk before launching."""
+    import mla_latent_kv_40_b200 as mla
+    dims = mla.make_dims(128, 512, 64, 128, 128, 7168, 64, "bf16", cache_layout=1)
+    n = ctypes.c_size_t(0)
+    assert mla._lib.mla_decode_sparse_workspace_size(ctypes.byref(dims), 64, 1, 0, ctypes.byref(n)) == -1
+    assert mla._lib.mla_decode_sparse_workspace_size(ctypes.byref(dims), 64, 1, 2048, ctypes.byref(n)) == 0
+    # the gathered rows alone: 64 tokens x 2048 rows x 1152 bytes
+    assert n.value >= 64 * 2048 * 1152
+    fake = ctypes.c_void_p(256)
+    rc = mla._lib.mla_decode_sparse(ctypes.byref(dims), 64, 1, fake, fake, fake, fake, None, 64, 4096, fake, 4096,
+                                    None, 2048, fake, fake, fake, None, fake, n.value, None, None)
+    assert rc == -1
