@@ -247,6 +247,46 @@ MLA_API int mla_decode_noalloc(const mla_dims *dims, int B, int n_q, const void 
                                mla_stream_t stream);
 
 /*
+ * mla_decode_partial — one device's share of a decode whose keys are split
+ *   between devices: mla_decode_latent restricted to the cached keys in
+ *   [kv_begin, kv_end) of every sequence (each query token still sees only
+ *   keys up to its own position seqlens[b] - n_q + j).
+ *   "现代 LLM 的 Memory-Compute Trade-off：从 MHA 到 MLA", section "MHA 与 KV
+ *   Cache": the cache of one long sequence grows linearly with its length, so
+ *   a 128k-token sequence may be spread over several GPUs; and "Transformer
+ *   升级之路：21", section 总而言之: MQA-form decoding cannot be split by head,
+ *   so the split is by key range.  Each device's partial is merged exactly by
+ *   mla_merge_partials.
+ *   kv_begin: a multiple of 64, >= 0; kv_end > kv_begin.  seqlens are the full
+ *   sequence lengths (they fix the query positions).
+ *   Writes o_lat [B, n_q, H, d_c] (dims->dtype): the softmax-weighted latent
+ *   over the range's visible keys, normalised by their own sum; and lse
+ *   [B, n_q, H] (float, required): their log-sum-exp, -inf (with o_lat 0)
+ *   where none is visible.  Workspace as mla_decode_workspace_size.
+ */
+MLA_API int mla_decode_partial(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,
+                               const void *c_kv, const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
+                               int num_blocks, const int32_t *seqlens, int max_seqlen, int kv_begin, int kv_end,
+                               const void *w_uk, void *o_lat, float *lse, void *workspace, size_t ws_bytes,
+                               int *dev_status, mla_stream_t stream);
+
+/*
+ * mla_merge_workspace_size / mla_merge_partials — the exact merge of n_parts
+ *   partials of one decode (e.g. gathered from n_parts devices):
+ *   LSE = ln sum_r exp(lse_r), o_lat = sum_r exp(lse_r - LSE) o_lat_r, then
+ *   out^(s) = o_lat^(s) W_UV^(s) ("Transformer升级之路：21", section 双重投影,
+ *   decoding column); with w_uv == NULL it writes o_lat [B, n_q, H, d_c].
+ *   o_lat_parts [n_parts, B, n_q, H, d_c] (dims->dtype), lse_parts
+ *   [n_parts, B, n_q, H] (float), both device memory (the caller gathers them,
+ *   e.g. with an all-gather over NCCL).  Writes out [B, n_q, H, d_v] and, if
+ *   non-NULL, lse [B, n_q, H].  Runs on CUDA cores (the merge is small).
+ */
+MLA_API int mla_merge_workspace_size(const mla_dims *dims, int B, int n_q, int n_parts, size_t *bytes);
+MLA_API int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts, const void *o_lat_parts,
+                               const float *lse_parts, const void *w_uv, void *out, float *lse, void *workspace,
+                               size_t ws_bytes, mla_stream_t stream);
+
+/*
  * mla_decode_sparse_workspace_size — scratch bytes of mla_decode_sparse for B
  *   sequences of n_q query tokens with lists of topk entries.
  */

@@ -65,6 +65,10 @@ _sigs = {
     "mla_decode_combine": [_D, _I, _I, _P, _I, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_prefill_workspace_size": [_D, _I, _I, _I, _SZ],
     "mla_decode_sparse_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode_partial": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, ctypes.c_size_t,
+                           _P, _P],
+    "mla_merge_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_merge_partials": [_D, _I, _I, _I, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_decode_sparse": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P, _P,
                           ctypes.c_size_t, _P, _P],
     "mla_decode_launches": [_D, _I, ctypes.POINTER(ctypes.c_int)],
@@ -208,6 +212,47 @@ def mla_decode_noalloc(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_p
                                  _ptr(lse, torch.float32, "lse", True), _ptr(dev_status, torch.int32, "dev_status", True),
                                  _stream(stream))
     _check("mla_decode_noalloc", rc)
+
+
+def mla_decode_partial(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                       max_seqlen, kv_begin, kv_end, w_uk, o_lat, lse, workspace, dev_status=None, stream=None):
+    """This device's share of a decode split by key range: o_lat [B, n_q, H, d_c] and lse [B, n_q, H]
+    over the keys in [kv_begin, kv_end) (kv_begin a multiple of 64)."""
+    et = _elem_dtype(dims)
+    B, n_q = q_nope.shape[0], q_nope.shape[1]
+    for n, t in (("q_nope", q_nope), ("q_pe", q_pe), ("block_table", block_table), ("seqlens", seqlens),
+                 ("w_uk", w_uk), ("o_lat", o_lat), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_decode_partial(ctypes.byref(dims), B, n_q, _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"),
+                                 _ptr(c_kv, et, "c_kv"), _ptr(k_pe, et, "k_pe"),
+                                 _ptr(block_table, torch.int32, "block_table", True), int(max_blocks_per_seq),
+                                 int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"), int(max_seqlen),
+                                 int(kv_begin), int(kv_end), _ptr(w_uk, et, "w_uk"), _ptr(o_lat, et, "o_lat"),
+                                 _ptr(lse, torch.float32, "lse"), _ptr(workspace, None, "workspace"),
+                                 ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                 _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_decode_partial", rc)
+
+
+def mla_merge_workspace_size(dims, B, n_q, n_parts) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_merge_workspace_size",
+           _lib.mla_merge_workspace_size(ctypes.byref(dims), int(B), int(n_q), int(n_parts), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_merge_partials(dims, o_lat_parts, lse_parts, w_uv, out, lse, workspace, stream=None):
+    """o_lat_parts [N, B, n_q, H, d_c], lse_parts [N, B, n_q, H] -> out [B, n_q, H, d_v] (o_lat when w_uv is None)."""
+    et = _elem_dtype(dims)
+    N, B, n_q = o_lat_parts.shape[0], o_lat_parts.shape[1], o_lat_parts.shape[2]
+    for n, t in (("o_lat_parts", o_lat_parts), ("lse_parts", lse_parts), ("w_uv", w_uv), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_merge_partials(ctypes.byref(dims), int(B), int(n_q), int(N), _ptr(o_lat_parts, et, "o_lat_parts"),
+                                 _ptr(lse_parts, torch.float32, "lse_parts"), _ptr(w_uv, et, "w_uv", True),
+                                 _ptr(out, et, "out"), _ptr(lse, torch.float32, "lse", True),
+                                 _ptr(workspace, None, "workspace"),
+                                 ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
+    _check("mla_merge_partials", rc)
 
 
 def mla_decode_sparse_workspace_size(dims, B, n_q, topk) -> int:

@@ -80,17 +80,21 @@ int check_ws(const DecodeLayout &L, const void *workspace, size_t ws_bytes) {
   return MLA_OK;
 }
 
+constexpr int kAllKeys = 0x7fffffff;   // kv_end of a decode over every cached key
+
 int attention_impl(const mla_dims *dims, int B, int n_q, const void *q_abs, const void *c_kv, const void *k_pe,
                    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, const int32_t *seqlens,
-                   int max_seqlen, const DecodeLayout &L, char *ws, int *dev_status, cudaStream_t st) {
+                   int max_seqlen, const DecodeLayout &L, char *ws, int *dev_status, cudaStream_t st,
+                   int kv_begin = 0, int kv_end = kAllKeys) {
   const bool bf16 = dims->dtype == MLA_BF16;
   CacheView cv{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq,
                num_blocks, dims->block_size, dims->cache_layout, dims->d_c, dims->d_c + dims->d_rope};
   if (L.use_tc)
-    return launch_tc_attention(*dims, B, n_q, q_abs, cv, seqlens, max_seqlen, ws + L.tc_off, dev_status, st);
+    return launch_tc_attention(*dims, B, n_q, q_abs, cv, seqlens, max_seqlen, ws + L.tc_off, dev_status, st,
+                               kv_begin, kv_end);
   AttnArgs at{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, q_abs, cv, seqlens, default_scale(*dims),
               kSimtChunk, L.max_chunks, reinterpret_cast<float *>(ws + L.o_off),
-              reinterpret_cast<float *>(ws + L.lse_off), dev_status};
+              reinterpret_cast<float *>(ws + L.lse_off), dev_status, kv_begin, kv_end};
   return launch_attn_simt(at, bf16, st);
 }
 
@@ -116,7 +120,7 @@ int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const 
                 const void *c_kv, const void *k_pe, const int32_t *block_table, int max_blocks_per_seq,
                 int num_blocks, const int32_t *seqlens, int max_seqlen, const void *w_uk,
                 const void *w_uv, void *out, float *lse, void *workspace, size_t ws_bytes,
-                int *dev_status, cudaStream_t st) {
+                int *dev_status, cudaStream_t st, int kv_begin = 0, int kv_end = kAllKeys) {
   int rc = check_decode_args(dims, B, n_q, c_kv, k_pe, max_blocks_per_seq, num_blocks, seqlens, max_seqlen);
   if (rc) return rc;
   if (!q_nope || (!q_pe && dims->d_rope) || !w_uk || !out) return MLA_ERR_INVALID_ARG;
@@ -128,7 +132,7 @@ int decode_impl(const mla_dims *dims, int B, int n_q, const void *q_nope, const 
                 q_nope, q_pe, w_uk, seqlens, qbuf, dims->rope_base};
   if ((rc = absorb_dispatch(ab, dims->dtype == MLA_BF16, dev_status, st))) return rc;
   if ((rc = attention_impl(dims, B, n_q, qbuf, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
-                           max_seqlen, L, ws, dev_status, st)))
+                           max_seqlen, L, ws, dev_status, st, kv_begin, kv_end)))
     return rc;
   return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L, ws, dev_status, st);
 }
@@ -347,6 +351,45 @@ int mla_decode_path(const mla_dims *dims, int n_q, int *path) {
   if (!dims_ok(dims) || n_q <= 0 || !path) return MLA_ERR_INVALID_ARG;
   *path = tc_decode_supported(*dims, n_q) ? MLA_PATH_TCGEN05 : MLA_PATH_CUDA_CORES;
   return MLA_OK;
+}
+
+int mla_decode_partial(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe, const void *c_kv,
+                       const void *k_pe, const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                       const int32_t *seqlens, int max_seqlen, int kv_begin, int kv_end, const void *w_uk,
+                       void *o_lat, float *lse, void *workspace, size_t ws_bytes, int *dev_status,
+                       mla_stream_t stream) {
+  if (kv_begin < 0 || kv_begin % 64 || kv_end <= kv_begin || !lse) return MLA_ERR_INVALID_ARG;
+  return decode_impl(dims, B, n_q, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                     max_seqlen, w_uk, nullptr, o_lat, lse, workspace, ws_bytes, dev_status,
+                     reinterpret_cast<cudaStream_t>(stream), kv_begin, kv_end);
+}
+
+int mla_merge_workspace_size(const mla_dims *dims, int B, int n_q, int n_parts, size_t *bytes) {
+  if (!dims_ok(dims) || B <= 0 || n_q <= 0 || n_parts <= 0 || !bytes) return MLA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)B * n_parts * n_q * dims->n_heads;
+  *bytes = align256(rows * dims->d_c * sizeof(float)) + align256(rows * sizeof(float));
+  return MLA_OK;
+}
+
+int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts, const void *o_lat_parts,
+                       const float *lse_parts, const void *w_uv, void *out, float *lse, void *workspace,
+                       size_t ws_bytes, mla_stream_t stream) {
+  size_t need = 0;
+  int rc = mla_merge_workspace_size(dims, B, n_q, n_parts, &need);
+  if (rc) return rc;
+  if (!o_lat_parts || !lse_parts || !out) return MLA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
+  if ((size_t)16 * (dims->d_c + n_parts) * sizeof(float) > 220 * 1024) return MLA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t rows = (size_t)B * n_parts * n_q * dims->n_heads;
+  float *o_part = static_cast<float *>(workspace);
+  float *lse_part = reinterpret_cast<float *>(static_cast<char *>(workspace) + align256(rows * dims->d_c * sizeof(float)));
+  const bool bf16 = dims->dtype == MLA_BF16;
+  if ((rc = launch_partials_to_splits(n_parts, B, n_q, dims->n_heads, dims->d_c, o_lat_parts, lse_parts, bf16, o_part,
+                                      lse_part, st)))
+    return rc;
+  CombineArgs cb{B, n_q, dims->n_heads, dims->d_c, dims->d_v, nullptr, 1, n_parts, o_part, lse_part, w_uv, out, lse};
+  return launch_combine(cb, bf16, st);
 }
 
 int mla_prefill_workspace_size(const mla_dims *dims, int B, int total_tokens, int max_seqlen,

@@ -50,8 +50,8 @@ attn_simt_kernel(AttnArgs a) {
     }
     return;
   }
-  const int k_begin = split * a.chunk;
-  const int k_end = min(S, k_begin + a.chunk);
+  const int k_begin = max(split * a.chunk, a.kv_begin);
+  const int k_end = min(min(S, split * a.chunk + a.chunk), a.kv_end);
 
   const T *q = static_cast<const T *>(a.q);
   for (int e = tid; e < kRowGrp * W; e += kAttnThreads) {

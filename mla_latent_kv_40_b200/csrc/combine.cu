@@ -39,9 +39,11 @@ combine_kernel(CombineArgs a) {
       continue;
     }
     const int b = g / a.n_q, j = g % a.n_q;
-    const int S = a.seqlens[b];
-    int nsplit = (S + a.chunk - 1) / a.chunk;
-    nsplit = max(0, min(nsplit, a.max_chunks));
+    int nsplit = a.max_chunks;
+    if (a.seqlens) {
+      const int S = a.seqlens[b];
+      nsplit = max(0, min((S + a.chunk - 1) / a.chunk, a.max_chunks));
+    }
     const int64_t base = (int64_t)b * a.max_chunks * R + (int64_t)j * a.H + s;
     float m = -CUDART_INF_F;
     for (int k = lane; k < nsplit; k += 32) m = fmaxf(m, a.lse_part[base + (int64_t)k * R]);
@@ -101,6 +103,37 @@ combine_kernel(CombineArgs a) {
       if (g < rows) out[((int64_t)g * a.H + s) * a.d_v + v] = from_f32<T>(acc[r]);
     }
   }
+}
+
+// Partials of N devices (each normalised over its own key range, with its lse) laid out as the N
+// splits of every query row, in fp32.
+template <typename T>
+__global__ void partials_to_splits_kernel(int N, int B, int R, int d_c, const T *o_parts, const float *lse_parts,
+                                          float *o_part, float *lse_part) {
+  const int64_t per = (int64_t)B * R;                 // query rows of one device's partial
+  const int64_t n = (int64_t)N * per * d_c;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+    const int c = (int)(e % d_c);
+    const int64_t row = e / d_c;                      // r * per + b * R + q
+    const int r = (int)(row / per);
+    const int64_t rem = row % per;
+    const int b = (int)(rem / R), q = (int)(rem % R);
+    const int64_t dst = ((int64_t)b * N + r) * R + q;
+    o_part[dst * d_c + c] = to_f32(o_parts[e]);
+    if (c == 0) lse_part[dst] = lse_parts[row];
+  }
+}
+
+int launch_partials_to_splits(int N, int B, int n_q, int H, int d_c, const void *o_parts, const float *lse_parts,
+                              bool bf16, float *o_part, float *lse_part, cudaStream_t st) {
+  const int R = n_q * H;
+  if (bf16)
+    partials_to_splits_kernel<<<1184, 256, 0, st>>>(N, B, R, d_c, static_cast<const __nv_bfloat16 *>(o_parts),
+                                                   lse_parts, o_part, lse_part);
+  else
+    partials_to_splits_kernel<<<1184, 256, 0, st>>>(N, B, R, d_c, static_cast<const float *>(o_parts), lse_parts,
+                                                   o_part, lse_part);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
 int launch_combine(const CombineArgs &a, bool bf16, cudaStream_t st) {

@@ -12,8 +12,8 @@
 // runs on a cluster of two CTAs on two SMs:
 //   * the score CTA (rank 0) keeps the latent part of Q in its tensor memory
 //     (A operand of TS-form MMAs) and the RoPE part in shared memory, streams
-//     the unit's pages as stages of [128 keys x 64 dims] (contiguous 8 KB
-//     chunks of the tiled pool), computes S for two pages at a time into one
+//     the unit's pages as half-page stages (one 32-40 KB contiguous bulk copy
+//     each from the tiled pool), computes S for two pages at a time into one
 //     of two tensor-memory buffers, runs the online softmax in registers, and
 //     sends each page of P (bf16, staged in shared memory) to the value CTA
 //     with one shared-to-peer bulk copy (distributed shared memory);
@@ -53,12 +53,17 @@ constexpr int kTileKeys = 64;                      // one cache page of keys (a 
 constexpr int kSuper = 2;                          // page tiles per score tile: N = 128 keys per MMA
 constexpr int kDc = 512, kDr = 64, kW = kDc + kDr;
 constexpr int kRows = 128;                         // M of every MMA: query rows per unit
-constexpr int kKStages = 10;                       // score CTA: [128 keys x 64 dims] stages in flight
+constexpr int kKStages = 4;                        // score CTA: half-page stages in flight (two pages)
 constexpr int kVStages = 4;                        // value CTA: [64 keys x 256 dims] half-page stages in flight
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;                   // per thread (65536 / 384, rounded down to 8)
 constexpr uint32_t kChunkBytes = kTileKeys * 128;  // one [64 keys x 64 dims] bf16 TMA box, 128B-swizzled
-constexpr uint32_t kKStageBytes = kSuper * kChunkBytes;            // 16384
+// A score-CTA stage is half a page, brought in by ONE contiguous bulk copy: chunks 0-3 (the
+// first 256 latent dims, 32 KB) or chunks 4-8 (the other 256 latent dims and the RoPE key, 40 KB).
+// One SM's copy engine sustains about 5 M bulk copies a second, so 8 KB copies cap an SM near
+// 42 GB/s while 32-40 KB copies run it at 90+ GB/s.
+__host__ __device__ constexpr int half_chunks(int half) { return half ? 5 : 4; }
+constexpr uint32_t kKStageBytes = 5 * kChunkBytes;                 // 40960 (room for the larger half)
 constexpr uint32_t kVStageBytes = 4 * kChunkBytes;                 // 32768
 constexpr uint32_t kPBytes = kRows * kTileKeys * 2;                // 16384
 constexpr int kPSlots = 5;                         // P page tiles in flight from the score CTA to the value CTA
@@ -135,6 +140,7 @@ struct TcParams {
   const unsigned char *tiled;        // tiled page pool (pages move by bulk copy), or NULL: row pool via TMA maps
   const unsigned char *row_pool;     // row pool base (c_kv) for L2 prefetch
   int rows_contig;                   // row pool with fused 576-wide rows: a page is 73728 contiguous bytes
+  int kv_begin, kv_end;              // attend to keys in [kv_begin, kv_end) only (kv_begin a multiple of 64)
 };
 
 __device__ __forceinline__ int seq_len_clamped(const TcParams &p, int b) {
@@ -142,8 +148,16 @@ __device__ __forceinline__ int seq_len_clamped(const TcParams &p, int b) {
   return S < 0 ? 0 : (S > p.max_seqlen ? p.max_seqlen : S);
 }
 
+// End of the keys a unit reads: the sequence's end or the key range's, whichever comes first.
+__device__ __forceinline__ int key_end(const TcParams &p, int b) {
+  const int S = seq_len_clamped(p, b);
+  return S < p.kv_end ? S : p.kv_end;
+}
+
+// Tiles (64-key pages) of a unit inside the key range; tile t holds keys kv_begin + 64 t ...
 __device__ __forceinline__ int unit_tiles(const TcParams &p, int u) {
-  return (seq_len_clamped(p, u / p.n_rb) + kTileKeys - 1) / kTileKeys;
+  const int e = key_end(p, u / p.n_rb) - p.kv_begin;
+  return e > 0 ? (e + kTileKeys - 1) / kTileKeys : 0;
 }
 
 // Cluster owning global tile t when T tiles are cut into C even ranges
@@ -290,7 +304,7 @@ __device__ __forceinline__ bool warp_wait(SmemB &sb, uint32_t bar, uint32_t pari
 }
 
 __device__ __forceinline__ int64_t tile_row(const TcParams &p, int b, int t) {
-  const int key = t * kTileKeys;
+  const int key = p.kv_begin + t * kTileKeys;
   const int lb = key / p.block_size;
   if (lb >= p.max_blocks_per_seq) return -1;
   const int blk = p.block_table ? p.block_table[(int64_t)b * p.max_blocks_per_seq + lb]
@@ -392,8 +406,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
     if (rank == 0) {
       if (warp == 0) {
       // ---- key producer (whole warp: page lookups in warp-wide batches; lane 0 issues): a score
-      // tile is up to 2 pages (128 keys), streamed as 9 stages of [128 keys x 64 dims] (8 latent
-      // chunks, then the RoPE key).  Optionally, pages further ahead are prefetched into L2.
+      // tile is up to 2 pages (128 keys); each page is streamed as two stages, one bulk copy each
+      // (chunks 0-3, then chunks 4-8).  Optionally, pages further ahead are prefetched into L2.
       grid_dep_wait();
       SegIter it = it0;
       PageRows pr;
@@ -419,27 +433,29 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             if (p.tiled) prefetch_l2(p.tiled + (prow / kTileKeys) * (9 * kChunkBytes), 9 * kChunkBytes);
             else if (p.rows_contig) prefetch_l2(p.row_pool + prow * (int64_t)kW * 2, kTileKeys * kW * 2);
           }
-          // Lane 0 streams the tile's 9 stages: a stage is chunk j of each page (8 KB each).
+          // Lane 0 streams the tile's pages, two stages per page: chunks 0-3, then chunks 4-8.
           int ok = 1;
           if (lane == 0) {
-            for (int j = 0; j < 9; ++j, ++n) {
-              sb.prog[warp] = (int)n;
-              const int s = n % kKStages;
-              if (n >= kKStages &&
-                  !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) {
-                ok = 0;
-                break;
-              }
-              const uint32_t dst = smem_u32(tiles + kKOff + s * kKStageBytes);
-              mbar_expect_tx(bar(B_KFULL + s), npg * kChunkBytes);
-#pragma unroll
-              for (int pg = 0; pg < kSuper; ++pg) {
-                if (pg >= npg) break;
-                if (p.tiled)   // chunk j of a page is 8 KB, already in the order the MMA reads it
-                  bulk_load(dst + pg * kChunkBytes, p.tiled + (int64_t)(rows[pg] / kTileKeys) * (9 * kChunkBytes) + j * kChunkBytes,
-                            kChunkBytes, bar(B_KFULL + s));
-                else if (j < 8) tma_load_2d(dst + pg * kChunkBytes, &map_c, 64 * j, rows[pg], bar(B_KFULL + s));
-                else tma_load_2d(dst + pg * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
+            for (int pg = 0; pg < npg && ok; ++pg) {
+              for (int half = 0; half < 2; ++half, ++n) {
+                sb.prog[warp] = (int)n;
+                const int s = n % kKStages;
+                if (n >= kKStages &&
+                    !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) {
+                  ok = 0;
+                  break;
+                }
+                const uint32_t dst = smem_u32(tiles + kKOff + s * kKStageBytes);
+                const int c0 = 4 * half, nc = half_chunks(half);
+                mbar_expect_tx(bar(B_KFULL + s), nc * kChunkBytes);
+                if (p.tiled)   // chunks c0 .. c0+nc-1 of a page are contiguous, already in the order the MMA reads them
+                  bulk_load(dst, p.tiled + (int64_t)(rows[pg] / kTileKeys) * (9 * kChunkBytes) + c0 * kChunkBytes,
+                            nc * kChunkBytes, bar(B_KFULL + s));
+                else
+                  for (int c = 0; c < nc; ++c) {
+                    if (c0 + c < 8) tma_load_2d(dst + c * kChunkBytes, &map_c, 64 * (c0 + c), rows[pg], bar(B_KFULL + s));
+                    else tma_load_2d(dst + c * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
+                  }
               }
             }
           }
@@ -455,7 +471,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           if (const uint32_t uses = n / kKStages + (s < (int)(n % kKStages) ? 1u : 0u))
             mbar_wait(bar(B_KFULL + s), (uses - 1) & 1, kWaitNs);
       } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: S [128 x N] = Q . K^T, N = 64 * pages (128 for a full score tile), into
+      // ---- MMA issuer: S [128 x 64 per page] = Q . K^T for the tile's pages side by side, into
       // one of two tensor-memory buffers so that the next tile's MMAs overlap this tile's softmax.
       // The latent part of Q is the A operand from tensor memory; the RoPE part is in shared memory.
       SegIter it = it0;
@@ -466,25 +482,32 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         tc_fence_after();
         for (int T = t0; T < t1; T += kSuper, ++ns) {
           const int npg = min(kSuper, t1 - T);
-          const uint32_t idesc = idesc_bf16_f32(kRows, kTileKeys * npg, false, false);
+          const uint32_t idesc = idesc_bf16_f32(kRows, kTileKeys, false, false);
           const uint32_t sbuf = ns & 1, dcol = tbase + kSCol + 128 * sbuf;
           if (ns >= 2 && !wait_or_abort(sb, bar(B_SEMPTY + sbuf), ((ns >> 1) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
           tc_fence_after();
-          for (int j = 0; j < 9; ++j, ++n) {
-            sb.prog[warp] = (int)n;
-            const int s = n % kKStages;
-            if (!wait_or_abort(sb, bar(B_KFULL + s), (n / kKStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t kt = smem_u32(tiles + kKOff + s * kKStageBytes);
+          // Page pg of the tile fills S columns 64 pg .. 64 pg + 63 (N = 64 MMAs), one half-page stage at a time.
+          for (int pg = 0; pg < npg && ok; ++pg) {
+            for (int half = 0; half < 2; ++half, ++n) {
+              sb.prog[warp] = (int)n;
+              const int s = n % kKStages;
+              if (!wait_or_abort(sb, bar(B_KFULL + s), (n / kKStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t kt = smem_u32(tiles + kKOff + s * kKStageBytes);
+              const uint32_t dcol_pg = dcol + 64 * pg;
+              for (int c = 0; c < half_chunks(half); ++c) {
+                const int j = 4 * half + c;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd = smem_desc_sw128(kt + kk * 32, 16, 1024);
-              if (j < 8)
-                mma_ts(dcol, tbase + kQCol + 32 * j + 8 * kk, bd, idesc, (j | kk) ? 1u : 0u);
-              else
-                mma_ss(dcol, smem_desc_sw128(smem_u32(tiles + kQpeOff) + kk * 32, 16, 1024), bd, idesc, 1u);
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t bd = smem_desc_sw128(kt + c * kChunkBytes + kk * 32, 16, 1024);
+                  if (j < 8)
+                    mma_ts(dcol_pg, tbase + kQCol + 32 * j + 8 * kk, bd, idesc, (j | kk) ? 1u : 0u);
+                  else
+                    mma_ss(dcol_pg, smem_desc_sw128(smem_u32(tiles + kQpeOff) + kk * 32, 16, 1024), bd, idesc, 1u);
+                }
+              }
+              tc_commit(bar(B_KEMPTY + s));
             }
-            tc_commit(bar(B_KEMPTY + s));
           }
           if (!ok) break;
           tc_commit(bar(B_SFULL + sbuf));
@@ -562,7 +585,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             ok = false;
             break;
           }
-          const bool tail = (t + 1) * kTileKeys > S;
+          const bool tail = p.kv_begin + (t + 1) * kTileKeys > S;
           const bool resc = t != t0 && (__float_as_uint(sb.pa[pb][0][32]) | __float_as_uint(sb.pa[pb][1][32]) |
                                         __float_as_uint(sb.pa[pb][2][32]) | __float_as_uint(sb.pa[pb][3][32])) != 0;
           bool have_v = false;
@@ -574,7 +597,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             have_v = true;
             if (resc && !wait_or_abort(sb, bar(B_PVDONE + (np - 1) % kPSlots), ((np - 1) / kPSlots) & 1, p.dev_status,
                                        false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            sb.req = Req{0, sv[0], sv[1], pb, S - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
+            sb.req = Req{0, sv[0], sv[1], pb, S - p.kv_begin - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
             mbar_arrive(bar(B_REQ));
             if (!wait_or_abort(sb, bar(B_REQDONE), nfix & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
             ++nfix;
@@ -710,7 +733,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
           // Valid while below the row's causal limit and inside the pages this tile holds.
-          const int nvalid = min(visible - (T + h) * kTileKeys, (npg - h) * kTileKeys);
+          const int nvalid = min(min(visible, p.kv_end) - (p.kv_begin + (T + h) * kTileKeys), (npg - h) * kTileKeys);
           float mx = -CUDART_INF_F;
 #pragma unroll
           for (int k = 0; k < 64; ++k)
@@ -1190,7 +1213,9 @@ size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q) {
 }
 
 int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, const CacheView &cache,
-                        const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st) {
+                        const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st,
+                        int kv_begin, int kv_end) {
+  if (kv_begin < 0 || kv_begin % kTileKeys) return MLA_ERR_INVALID_ARG;
   const bool tiled = cache.layout == MLA_CACHE_TILED;
   if ((reinterpret_cast<uintptr_t>(cache.c_kv) & 15) || (!tiled && (reinterpret_cast<uintptr_t>(cache.k_pe) & 15)) ||
       (reinterpret_cast<uintptr_t>(q_abs) & 15))
@@ -1232,6 +1257,8 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
   p.seg_info = reinterpret_cast<int *>(w + L.seg_info);
   p.timeout_rec = p.seg_info + 2 * p.U;
   p.dev_status = dev_status;
+  p.kv_begin = kv_begin;
+  p.kv_end = kv_end;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * C);
   cfg.blockDim = dim3(kThreads);

@@ -11,9 +11,11 @@ bool tc_decode_supported(const mla_dims &d, int n_q);
 int tc_decode_kernel_launches();
 // Scratch bytes the tcgen05 path needs beyond the absorbed query buffer.
 size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q);
-// Split-KV attention from an absorbed query buffer; partials stay in ws.
+// Split-KV attention from an absorbed query buffer; partials stay in ws.  Only keys in
+// [kv_begin, kv_end) are read (kv_begin a multiple of 64); the full decode passes 0, INT_MAX.
 int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, const CacheView &cache,
-                        const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st);
+                        const int32_t *seqlens, int max_seqlen, void *ws, int *dev_status, cudaStream_t st,
+                        int kv_begin, int kv_end);
 // Merge of the partials (+ W_UV when w_uv != NULL).
 int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
                       void *out, float *lse, void *ws, int *dev_status, cudaStream_t st);

@@ -72,12 +72,13 @@ struct AttnArgs {
   float *o_part;            // [B, max_chunks, n_q*H, d_c], normalised by the split's own sum
   float *lse_part;          // [B, max_chunks, n_q*H]
   int *dev_status;
+  int kv_begin, kv_end;     // only keys in [kv_begin, kv_end) are read
 };
 
 // Merge of the split partials and the per-head up-projection.
 struct CombineArgs {
   int B, n_q, H, d_c, d_v;
-  const int32_t *seqlens;
+  const int32_t *seqlens;   // NULL: every one of the max_chunks splits holds a partial
   int chunk, max_chunks;
   const float *o_part, *lse_part;
   const void *w_uv;         // [H, d_c, d_v], NULL: write o_lat instead
@@ -122,6 +123,10 @@ bool append_tc_supported(const AppendArgs &a, bool bf16);
 int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split, cudaStream_t st);
 int launch_append_finish(const AppendArgs &a, const void *ws, int nsplit, cudaStream_t st);
 int launch_cache_convert(const void *src, void *dst, int64_t num_rows, int W, bool to_tiled, cudaStream_t st);
+// Cross-device merge: partials [N][B][n_q][H][d_c] (dtype) and lses [N][B][n_q][H] -> the split
+// layout launch_combine reads (o_part [B][N][n_q*H][d_c] fp32, lse_part [B][N][n_q*H]).
+int launch_partials_to_splits(int N, int B, int n_q, int H, int d_c, const void *o_parts, const float *lse_parts,
+                              bool bf16, float *o_part, float *lse_part, cudaStream_t st);
 // Sparse decode: compact each query token's listed cache rows into its own run of 64-token pages.
 int launch_sparse_gather(int B, int n_q, int topk, const int32_t *idx, const int32_t *seqlens, int max_seqlen,
                          const CacheView &src, void *pool, bool dst_tiled, int elem, int32_t *counts,

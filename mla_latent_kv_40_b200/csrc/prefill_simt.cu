@@ -17,32 +17,38 @@ namespace mla {
 constexpr int kPfThreads = 256;
 
 // (1) qbuf[t, s, :] = [q_nope | RoPE(q_pe, position of t)]
+// One CTA per query token: the token's position and its d_R/2 rotation angles are computed once
+// and shared by every head; then one element per thread, in row order (coalesced).
 template <typename T>
-__global__ void prefill_q_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(kPfThreads) prefill_q_kernel(PrefillArgs a) {
+  extern __shared__ float rot[];          // [d_rope / 2][2]: cos, sin
+  __shared__ int pos;
+  const int t = blockIdx.x;
+  if (threadIdx.x == 0) {                 // position of row t within its sequence
+    int lo = 0, hi = a.B;                 // find b with cu[b] <= t < cu[b+1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (a.cu_seqlens[mid] <= t) lo = mid; else hi = mid;
+    }
+    pos = t - a.cu_seqlens[lo];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < (a.d_rope >> 1); i += blockDim.x)
+    rope_cos_sin(pos, i, a.d_rope, a.rope_base, &rot[2 * i], &rot[2 * i + 1]);
+  __syncthreads();
   const int dqk = a.d_nope + a.d_rope;
-  const int64_t n = (int64_t)a.total * a.H * dqk;
-  const T *qn = static_cast<const T *>(a.q_nope);
-  const T *qp = static_cast<const T *>(a.q_pe);
-  T *qb = static_cast<T *>(a.qbuf);
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
-    const int d = (int)(e % dqk);
-    const int64_t ts = e / dqk;           // t * H + s
-    const int t = (int)(ts / a.H);
+  const T *qn = static_cast<const T *>(a.q_nope) + (int64_t)t * a.H * a.d_nope;
+  const T *qp = static_cast<const T *>(a.q_pe) + (int64_t)t * a.H * a.d_rope;
+  T *qb = static_cast<T *>(a.qbuf) + (int64_t)t * a.H * dqk;
+  for (int e = threadIdx.x; e < a.H * dqk; e += blockDim.x) {
+    const int s = e / dqk, d = e % dqk;
     if (d < a.d_nope) {
-      qb[e] = qn[ts * a.d_nope + d];
+      qb[e] = qn[s * a.d_nope + d];
     } else {
       const int dr = d - a.d_nope, i = dr >> 1;
-      // position of row t within its sequence
-      int lo = 0, hi = a.B;                // find b with cu[b] <= t < cu[b+1]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (a.cu_seqlens[mid] <= t) lo = mid; else hi = mid;
-      }
-      const int p = t - a.cu_seqlens[lo];
-      float cs, sn;
-      rope_cos_sin(p, i, a.d_rope, a.rope_base, &cs, &sn);
-      const float x = to_f32(qp[ts * a.d_rope + 2 * i]), y = to_f32(qp[ts * a.d_rope + 2 * i + 1]);
-      qb[e] = from_f32<T>((dr & 1) ? (x * sn + y * cs) : (x * cs - y * sn));
+      const float x = to_f32(qp[s * a.d_rope + 2 * i]), y = to_f32(qp[s * a.d_rope + 2 * i + 1]);
+      const float c = rot[2 * i], sn = rot[2 * i + 1];
+      qb[e] = from_f32<T>((dr & 1) ? (x * sn + y * c) : (x * c - y * sn));
     }
   }
 }
@@ -232,7 +238,7 @@ prefill_attn_kernel(PrefillArgs a) {
 template <typename T>
 static int launch_prefill_t(const PrefillArgs &a, cudaStream_t st) {
   const int dqk = a.d_nope + a.d_rope;
-  prefill_q_kernel<T><<<1184, kPfThreads, 0, st>>>(a);
+  prefill_q_kernel<T><<<a.total, kPfThreads, sizeof(float) * a.d_rope, st>>>(a);
   const size_t smem_dec = sizeof(float) * kDecRows * a.d_c;
   if (cudaFuncSetAttribute(prefill_decompress_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dec))
     return MLA_ERR_CUDA;
