@@ -343,6 +343,134 @@ def measure_decode_configs(mla, torch, peaks, steps, names=("v2lite_bf16", "v3_r
     return res
 
 
+def measure_sparse(mla, torch, peaks, steps, topk=2048):
+    """Sparse decode (mla_decode_sparse) on the V3 batch-64 x 4096 workload with `topk` tokens selected
+    per query token (seeded random distinct positions): the gather of the selected rows, absorption,
+    attention over them and the combine, per call.  Roofline: the selected rows read once
+    (gathered, then streamed) against HBM, or the attention FLOPs over the selected keys."""
+    import numpy as np
+    from workloads import DECODE_CASES, make_decode_inputs_device
+    case = DECODE_CASES["v3_bf16"]
+    d = case.dims
+    inp = make_decode_inputs_device(case)
+    dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                         rope_base=d.rope_base, rms_eps=d.rms_eps, cache_layout=1)
+    packed = torch.empty_like(inp["pool"])
+    mla.mla_cache_pack(dims, inp["pool"], packed)
+    torch.cuda.synchronize()
+    inp["pool"] = packed
+    B, n_q, H = case.batch, case.n_q, d.n_heads
+    sl = inp["seqlens"]
+    g = np.random.default_rng(case.seed)
+    sel = np.stack([np.stack([g.permutation(int(sl[b]) - n_q + j + 1)[:topk] for j in range(n_q)]) for b in range(B)])
+    sel_d = torch.from_numpy(sel.astype(np.int32)).cuda()
+    ws = mla.alloc_workspace(mla.mla_decode_sparse_workspace_size(dims, B, n_q, topk))
+    out = torch.empty((B, n_q, H, d.d_v), dtype=d.torch_dtype, device="cuda")
+    lse = torch.empty((B, n_q, H), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bt, sl_d = inp["block_table"].cuda(), sl.cuda()
+
+    def run():
+        mla.mla_decode_sparse(dims, inp["q_nope"], inp["q_pe"], packed, packed, bt, inp["max_blocks_per_seq"],
+                              inp["num_blocks"], sl_d, int(sl.max()), sel_d, inp["w_uk"], inp["w_uv"], out, lse, ws, st)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the sparse decode")
+    ms = e0.elapsed_time(e1) / steps
+    keys = B * n_q * topk
+    W = d.d_c + d.d_rope
+    att_flops = keys * H * (2 * W + 2 * d.d_c)
+    flops = att_flops + B * n_q * H * 2 * d.d_c * (d.d_nope + d.d_v)
+    sel_bytes = keys * W * 2
+    t_roof = max(sel_bytes / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    res = {"workload": f"v3_bf16 with {topk} selected tokens per query", "ms": ms,
+           "tflops": flops / (ms * 1e-3) / 1e12, "selected_kv_gbs": sel_bytes / (ms * 1e-3) / 1e9,
+           "decode_tokens_per_s": B * n_q / (ms * 1e-3), "roofline_us": t_roof * 1e6,
+           "roofline_frac": t_roof / (ms * 1e-3), "call": "mla_decode_sparse (gather + absorb + attention + combine)"}
+    del inp, packed, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_split_kv(mla, torch, peaks, steps, world=4):
+    """The V3 long workload (4 x 131072 keys, 2 query tokens) split into `world` key ranges, each
+    range's partial (mla_decode_partial) timed alone on this GPU, as one of `world` devices would
+    run it, and the merge of the `world` partials (mla_merge_partials).  The all-gather between
+    devices (world x 1 MB here) is not part of it: every run here has one GPU."""
+    import importlib
+    sharded = importlib.import_module("mla_latent_kv_40_b200.sharded")
+    from workloads import DECODE_CASES, decode_flops, latent_bytes, make_decode_inputs_device
+    case = DECODE_CASES["v3_long_bf16"]
+    d = case.dims
+    inp = make_decode_inputs_device(case)
+    dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                         rope_base=d.rope_base, rms_eps=d.rms_eps, cache_layout=1)
+    packed = torch.empty_like(inp["pool"])
+    mla.mla_cache_pack(dims, inp["pool"], packed)
+    torch.cuda.synchronize()
+    inp["pool"] = packed
+    B, n_q, H = case.batch, case.n_q, d.n_heads
+    sl = inp["seqlens"]
+    max_seqlen = int(sl.max())
+    bt, sl_d = inp["block_table"].cuda(), sl.cuda()
+    ws = mla.alloc_workspace(mla.mla_decode_workspace_size(dims, B, n_q, max_seqlen))
+    o_parts = torch.empty((world, B, n_q, H, d.d_c), dtype=d.torch_dtype, device="cuda")
+    l_parts = torch.empty((world, B, n_q, H), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ranges = sharded.kv_shard_ranges(max_seqlen, world)
+    part_ms = []
+    for r, (k0, k1) in enumerate(ranges):
+        def run():
+            mla.mla_decode_partial(dims, inp["q_nope"], inp["q_pe"], packed, packed, bt, inp["max_blocks_per_seq"],
+                                   inp["num_blocks"], sl_d, max_seqlen, k0, k1, inp["w_uk"], o_parts[r], l_parts[r],
+                                   ws, st)
+        for _ in range(3):
+            run()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        part_ms.append(e0.elapsed_time(e1) / steps)
+    out = torch.empty((B, n_q, H, d.d_v), dtype=d.torch_dtype, device="cuda")
+    lse = torch.empty((B, n_q, H), dtype=torch.float32, device="cuda")
+    mws = mla.alloc_workspace(mla.mla_merge_workspace_size(dims, B, n_q, world))
+    for _ in range(3):
+        mla.mla_merge_partials(dims, o_parts, l_parts, inp["w_uv"], out, lse, mws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        mla.mla_merge_partials(dims, o_parts, l_parts, inp["w_uv"], out, lse, mws)
+    e1.record()
+    torch.cuda.synchronize()
+    merge_ms = e0.elapsed_time(e1) / steps
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the split decode")
+    fl = decode_flops(d, sl.tolist(), n_q)["total"]
+    lb = latent_bytes(d, sl.tolist())
+    per_dev = max(part_ms) + merge_ms
+    t_roof = max(lb / world / (peaks["hbm_gbs"] * 1e9), fl / world / (peaks["bf16_tflops"] * 1e12))
+    res = {"workload": f"v3_long_bf16 split over {world} key ranges", "ranges": ranges, "partial_ms": part_ms,
+           "merge_ms": merge_ms, "ms_per_device": per_dev, "tflops_per_device": fl / world / (per_dev * 1e-3) / 1e12,
+           "roofline_us_per_device": t_roof * 1e6, "roofline_frac": t_roof / (per_dev * 1e-3),
+           "note": "per device: its own range's partial plus the merge; the all-gather is not included"}
+    del inp, packed, ws
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_mla(args):
     import torch
     import torch.distributed as dist
@@ -607,6 +735,8 @@ def run_mla(args):
         del dev, pool, c_kv, k_pe, ws
         torch.cuda.empty_cache()
         line["configs"] = measure_decode_configs(mla, torch, peaks, max(args.steps, 5))
+        line["sparse"] = measure_sparse(mla, torch, peaks, max(args.steps, 5))
+        line["split_kv"] = measure_split_kv(mla, torch, peaks, max(args.steps, 5))
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
     if rank == 0:

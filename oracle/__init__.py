@@ -15,6 +15,7 @@ Nothing here is "parity unpinned".
 """
 from .mla_oracle import (  # noqa: F401
     rope_frequencies, rope_rotate, rms_norm, append_latent, gather_rows,
-    decompress_head, attend, decode, decode_one, decode_sparse, prefill, kv_cache_bytes_mha,
+    decompress_head, attend, decode, decode_one, decode_sparse, prefill, query_from_hidden,
+    output_projection, kv_cache_bytes_mha,
     latent_elems_per_token,
 )

@@ -209,6 +209,32 @@ def decode(dims, q_nope, q_pe, pool, block_table, block_size: int, seqlens, w_uk
     return out, lse
 
 
+# ---------------------------------------------------------------- query latent path and output projection
+
+def query_from_hidden(h, w_dq, w_uq, w_qr):
+    """Queries from the compressed query latent ("DeepSeek-V3 解读 1: MLA", section "MLA：高层次的思路":
+    queries too are projected into a low-dimensional latent space and restored from it; section
+    "为什么需要解耦 RoPE": an extra RoPE query per head, taken from the same latent).
+
+    c_Q = h W_DQ;  q_nope^(s) = c_Q W_UQ^(s);  q_pe^(s) = c_Q W_QR^(s) (not rotated: the decode
+    rotates it at the query's position).
+    h [..., D], w_dq [D, d_cq], w_uq [d_cq, H, d_nope], w_qr [d_cq, H, d_R].
+    Returns (q_nope [..., H, d_nope], q_pe [..., H, d_R]) in float64.
+    """
+    c_q = _f64(h) @ _f64(w_dq)
+    q_nope = np.einsum("...c,chd->...hd", c_q, _f64(w_uq))
+    q_pe = np.einsum("...c,chd->...hd", c_q, _f64(w_qr))
+    return q_nope, q_pe
+
+
+def output_projection(out_heads, w_o):
+    """The attention block's output u = [o^(1), ..., o^(H)] W^O ("DeepSeek-V3 解读 1: MLA": W^O maps the
+    concatenated head outputs, n_h d_h wide, back to the model width d).
+    out_heads [..., H, d_v], w_o [H d_v, D] -> [..., D] in float64."""
+    o = _f64(out_heads)
+    return o.reshape(o.shape[:-2] + (-1,)) @ _f64(w_o)
+
+
 # ---------------------------------------------------------------- sparse decode over selected tokens
 
 def decode_sparse(dims, q_nope, q_pe, pool, block_table, block_size: int, seqlens, topk_idx, w_uk, w_uv,

@@ -204,3 +204,21 @@ def test_sparse_decode_host_validation():
     rc = mla._lib.mla_decode_sparse(ctypes.byref(dims), 64, 1, fake, fake, fake, fake, None, 64, 4096, fake, 4096,
                                     None, 2048, fake, fake, fake, None, fake, n.value, None, None)
     assert rc == -1
+
+
+def test_split_kv_host_validation():
+    """mla_decode_partial needs a 64-aligned kv_begin, kv_end > kv_begin and an lse output;
+    mla_merge_partials needs at least one part.  Both are refused before any launch."""
+    import mla_latent_kv_40_b200 as mla
+    dims = mla.make_dims(128, 512, 64, 128, 128, 7168, 64, "bf16", cache_layout=1)
+    fake = ctypes.c_void_p(256)
+    base = [ctypes.byref(dims), 4, 2, fake, fake, fake, fake, None, 2048, 8192, fake, 131072]
+    tail = [fake, fake, fake, fake, 1 << 20, None, None]
+    assert mla._lib.mla_decode_partial(*base, 32, 4096, *tail) == -1        # kv_begin not a multiple of 64
+    assert mla._lib.mla_decode_partial(*base, 4096, 4096, *tail) == -1      # empty range
+    tail_no_lse = [fake, fake, None, fake, 1 << 20, None, None]
+    assert mla._lib.mla_decode_partial(*base, 0, 4096, *tail_no_lse) == -1  # lse is required
+    n = ctypes.c_size_t(0)
+    assert mla._lib.mla_merge_workspace_size(ctypes.byref(dims), 4, 2, 0, ctypes.byref(n)) == -1
+    assert mla._lib.mla_merge_workspace_size(ctypes.byref(dims), 4, 2, 4, ctypes.byref(n)) == 0
+    assert n.value >= 4 * 4 * 2 * 128 * 512 * 4

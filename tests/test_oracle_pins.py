@@ -517,3 +517,94 @@ def _sparse_variant(mistake):
 def test_planted_sparse_mistakes_are_caught(monkeypatch, mistake):
     _assert_some_pin_fails(monkeypatch, "decode_sparse", _sparse_variant(mistake),
                            [test_sparse_decode_brute_force_tiny])
+
+
+# ------------------------------------------------------------------ query latent path and output projection
+
+def test_query_from_hidden_brute_force_tiny():
+    r = _rng(31)
+    D, d_cq, H, d_nope, d_R = 5, 3, 2, 4, 2
+    h = r.standard_normal((2, D))
+    w_dq, w_uq, w_qr = r.standard_normal((D, d_cq)), r.standard_normal((d_cq, H, d_nope)), r.standard_normal((d_cq, H, d_R))
+    qn, qp = oracle.query_from_hidden(h, w_dq, w_uq, w_qr)
+    for t in range(2):
+        c = [sum(h[t][x] * w_dq[x][y] for x in range(D)) for y in range(d_cq)]
+        for s in range(H):
+            for k in range(d_nope):
+                assert abs(qn[t, s, k] - sum(c[y] * w_uq[y][s][k] for y in range(d_cq))) < 1e-12
+            for k in range(d_R):
+                assert abs(qp[t, s, k] - sum(c[y] * w_qr[y][s][k] for y in range(d_cq))) < 1e-12
+
+
+def test_output_projection_brute_force_tiny():
+    """u_j = sum over heads s and value dims v of o[s, v] * W_O[s * d_v + v, j]."""
+    r = _rng(32)
+    H, d_v, D = 3, 2, 4
+    o = r.standard_normal((2, H, d_v))
+    w_o = r.standard_normal((H * d_v, D))
+    u = oracle.output_projection(o, w_o)
+    for t in range(2):
+        for j in range(D):
+            want = sum(o[t, s, v] * w_o[s * d_v + v, j] for s in range(H) for v in range(d_v))
+            assert abs(u[t, j] - want) < 1e-12
+
+
+def _folded_block_output(d, h, w_dq, w_uq, w_qr, pool, bt, bs, seqlens, n_q, w_uk, w_uv, w_o):
+    """The decode written with the weights folded offline, in fp64: W_UQK^(s) = W_UQ^(s) W_UK^(s)T
+    turns c_Q straight into the latent query; W_UVO^(s) = W_UV^(s) W_O^(s) turns each head's latent
+    output straight into its share of u ("DeepSeek-V3 解读 1: MLA", section "为什么需要解耦 RoPE": W^UK
+    absorbed into W^Q; "Transformer升级之路：21", section 键值共享: the c -> v map absorbed on the W_o side)."""
+    H, d_c, d_v = d.n_heads, d.d_c, d.d_v
+    w_uqk = np.einsum("chn,hln->hcl", w_uq, w_uk)                  # [H, d_cq, d_c]
+    w_uvo = np.einsum("hlv,hvj->hlj", w_uv, w_o.reshape(H, d_v, -1))  # [H, d_c, D]
+    B = h.shape[0]
+    u = np.zeros((B, n_q, w_o.shape[1]))
+    scale = 1 / math.sqrt(d.d_nope + d.d_rope)
+    for b in range(B):
+        S = int(seqlens[b])
+        rows = bt[b, np.arange(S) // bs] * bs + np.arange(S) % bs
+        c, kpe = pool[rows, :d_c], pool[rows, d_c:]
+        for j in range(n_q):
+            p = S - n_q + j
+            c_q = h[b, j] @ w_dq
+            for s in range(H):
+                q_lat = c_q @ w_uqk[s]
+                q_rot = O.rope_rotate(c_q @ w_qr[:, s, :], p, d.rope_base)
+                z = (c[:p + 1] @ q_lat + kpe[:p + 1] @ q_rot) * scale
+                e = np.exp(z - z.max())
+                o_lat = (e / e.sum()) @ c[:p + 1]
+                u[b, j] += o_lat @ w_uvo[s]
+    return u
+
+
+def test_folded_weights_equal_the_unfolded_chain():
+    """Decode from hidden states with folded weights equals query_from_hidden -> decode (unabsorbed)
+    -> output_projection to 1e-12 (two causal query tokens, paged)."""
+    r = _rng(33)
+    d = Dims(n_heads=3, d_c=8, d_rope=4, d_nope=5, d_v=6, d_model=7, dtype="f32")
+    d_cq, n_q, B, bs = 6, 2, 2, 4
+    seqlens = np.array([7, 10])
+    pool = r.standard_normal((16, d.d_c + d.d_rope))
+    bt = np.array([[3, 0, 1], [2, 1, 0]])
+    h = r.standard_normal((B, n_q, d.d_model))
+    w_dq = r.standard_normal((d.d_model, d_cq))
+    w_uq = r.standard_normal((d_cq, d.n_heads, d.d_nope))
+    w_qr = r.standard_normal((d_cq, d.n_heads, d.d_rope))
+    w_uk = r.standard_normal((d.n_heads, d.d_c, d.d_nope))
+    w_uv = r.standard_normal((d.n_heads, d.d_c, d.d_v))
+    w_o = r.standard_normal((d.n_heads * d.d_v, d.d_model))
+    qn, qp = oracle.query_from_hidden(h, w_dq, w_uq, w_qr)
+    out, _ = oracle.decode(d, qn, qp, pool, bt, bs, seqlens, w_uk, w_uv)
+    u = oracle.output_projection(out, w_o)
+    u2 = _folded_block_output(d, h, w_dq, w_uq, w_qr, pool, bt, bs, seqlens, n_q, w_uk, w_uv, w_o)
+    np.testing.assert_allclose(u, u2, rtol=1e-12, atol=1e-12)
+
+
+def test_planted_output_projection_layout_is_caught(monkeypatch):
+    """Concatenating the head outputs dimension-major instead of head-major fails the pin."""
+    def wrong(out_heads, w_o):
+        o = np.asarray(out_heads, dtype=np.float64)
+        return np.swapaxes(o, -1, -2).reshape(o.shape[:-2] + (-1,)) @ np.asarray(w_o, dtype=np.float64)
+    monkeypatch.setattr(oracle, "output_projection", wrong)
+    with pytest.raises(AssertionError):
+        test_output_projection_brute_force_tiny()
