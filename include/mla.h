@@ -287,6 +287,50 @@ MLA_API int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts
                                size_t ws_bytes, mla_stream_t stream);
 
 /*
+ * mla_fold_query_weights / mla_fold_output_weights — the offline folds of the
+ *   fully absorbed decode.
+ *   "DeepSeek-V3 解读 1: MLA", section "为什么需要解耦 RoPE": W^UK can be absorbed
+ *   into the query projection, W_UQK^(s) = W_UQ^(s) W_UK^(s)T [d_cq x d_c], so the
+ *   query latent c_Q maps straight to the latent query.  "Transformer升级之路：
+ *   21", section 键值共享: the c -> v map is absorbed on the W_o side,
+ *   W_UVO^(s) = W_UV^(s) W_O^(s) [d_c x D], with W_O^(s) the d_v rows of the
+ *   output projection W^O [H d_v, D] that belong to head s.
+ *   w_uq [d_cq, H, d_nope], w_uk [H, d_c, d_nope] -> w_uqk [H, d_cq, d_c];
+ *   w_uv [H, d_c, d_v], w_o [H d_v, D] -> w_uvo [H, d_c, D]; dims->dtype,
+ *   fp32 accumulation, rounded once.  CUDA cores (run once per model).
+ *   Note the sizes: at V3 shapes (d_cq 1536, H 128, d_c 512, D 7168) the folded
+ *   W_UQK holds 201 MB and W_UVO 940 MB, against 67 MB for W_UQ and W_UK and
+ *   134 MB for W_UV and W^O: folding trades the per-step W_UK / W_UV products
+ *   for larger weights.
+ */
+MLA_API int mla_fold_query_weights(const mla_dims *dims, int d_cq, const void *w_uq, const void *w_uk, void *w_uqk,
+                                   mla_stream_t stream);
+MLA_API int mla_fold_output_weights(const mla_dims *dims, const void *w_uv, const void *w_o, void *w_uvo,
+                                    mla_stream_t stream);
+
+/*
+ * mla_decode_absorbed_workspace_size / mla_decode_absorbed — one decode step of
+ *   the attention block from the hidden states, in the fully absorbed form:
+ *   c_Q = h W_DQ ("DeepSeek-V3 解读 1: MLA", section "MLA：高层次的思路": queries
+ *   are compressed to a latent too), q_lat^(s) = c_Q W_UQK^(s),
+ *   q_pe^(s) = RoPE(c_Q W_QR^(s), seqlens[b] - n_q + j), the split-KV attention
+ *   of mla_decode over the latent cache, and u = sum_s o_lat^(s) W_UVO^(s).
+ *   h [B, n_q, D], w_dq [D, d_cq], w_uqk [H, d_cq, d_c] and w_uvo [H, d_c, D]
+ *   (from the folds above), w_qr [d_cq, H, d_R]; cache, seqlens, lse as
+ *   mla_decode.  Writes out [B, n_q, D] (dims->dtype; D = dims->d_model).
+ *   The four products run on CUDA cores; the attention on the same kernels as
+ *   mla_decode.  c_Q, the queries and o_lat are rounded to dims->dtype between
+ *   the steps.
+ */
+MLA_API int mla_decode_absorbed_workspace_size(const mla_dims *dims, int d_cq, int B, int n_q, int max_seqlen,
+                                               size_t *bytes);
+MLA_API int mla_decode_absorbed(const mla_dims *dims, int d_cq, int B, int n_q, const void *h, const void *w_dq,
+                                const void *w_uqk, const void *w_qr, const void *c_kv, const void *k_pe,
+                                const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                                const int32_t *seqlens, int max_seqlen, const void *w_uvo, void *out, float *lse,
+                                void *workspace, size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
  * mla_decode_sparse_workspace_size — scratch bytes of mla_decode_sparse for B
  *   sequences of n_q query tokens with lists of topk entries.
  */

@@ -68,6 +68,11 @@ _sigs = {
     "mla_decode_partial": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, ctypes.c_size_t,
                            _P, _P],
     "mla_merge_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_fold_query_weights": [_D, _I, _P, _P, _P, _P],
+    "mla_fold_output_weights": [_D, _P, _P, _P, _P],
+    "mla_decode_absorbed_workspace_size": [_D, _I, _I, _I, _I, _SZ],
+    "mla_decode_absorbed": [_D, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P,
+                            ctypes.c_size_t, _P, _P],
     "mla_merge_partials": [_D, _I, _I, _I, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P],
     "mla_decode_sparse": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P, _P,
                           ctypes.c_size_t, _P, _P],
@@ -253,6 +258,54 @@ def mla_merge_partials(dims, o_lat_parts, lse_parts, w_uv, out, lse, workspace, 
                                  _ptr(workspace, None, "workspace"),
                                  ctypes.c_size_t(workspace.numel() * workspace.element_size()), _stream(stream))
     _check("mla_merge_partials", rc)
+
+
+def mla_fold_query_weights(dims, w_uq, w_uk, w_uqk, stream=None):
+    """w_uq [d_cq, H, d_nope], w_uk [H, d_c, d_nope] -> w_uqk [H, d_cq, d_c] = W_UQ^(s) W_UK^(s)T."""
+    et = _elem_dtype(dims)
+    for n, t in (("w_uq", w_uq), ("w_uk", w_uk), ("w_uqk", w_uqk)):
+        _dense(t, n)
+    _check("mla_fold_query_weights", _lib.mla_fold_query_weights(ctypes.byref(dims), int(w_uq.shape[0]),
+                                                                 _ptr(w_uq, et, "w_uq"), _ptr(w_uk, et, "w_uk"),
+                                                                 _ptr(w_uqk, et, "w_uqk"), _stream(stream)))
+
+
+def mla_fold_output_weights(dims, w_uv, w_o, w_uvo, stream=None):
+    """w_uv [H, d_c, d_v], w_o [H * d_v, D] -> w_uvo [H, d_c, D] = W_UV^(s) W_O^(s)."""
+    et = _elem_dtype(dims)
+    for n, t in (("w_uv", w_uv), ("w_o", w_o), ("w_uvo", w_uvo)):
+        _dense(t, n)
+    _check("mla_fold_output_weights", _lib.mla_fold_output_weights(ctypes.byref(dims), _ptr(w_uv, et, "w_uv"),
+                                                                   _ptr(w_o, et, "w_o"), _ptr(w_uvo, et, "w_uvo"),
+                                                                   _stream(stream)))
+
+
+def mla_decode_absorbed_workspace_size(dims, d_cq, B, n_q, max_seqlen) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_decode_absorbed_workspace_size",
+           _lib.mla_decode_absorbed_workspace_size(ctypes.byref(dims), int(d_cq), int(B), int(n_q), int(max_seqlen),
+                                                   ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_absorbed(dims, h, w_dq, w_uqk, w_qr, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                        max_seqlen, w_uvo, out, lse, workspace, dev_status=None, stream=None):
+    """h [B, n_q, D] -> out [B, n_q, D]: the attention block's decode output with folded weights."""
+    et = _elem_dtype(dims)
+    B, n_q = h.shape[0], h.shape[1]
+    d_cq = w_dq.shape[1]
+    for n, t in (("h", h), ("w_dq", w_dq), ("w_uqk", w_uqk), ("w_qr", w_qr), ("block_table", block_table),
+                 ("seqlens", seqlens), ("w_uvo", w_uvo), ("out", out), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_decode_absorbed(ctypes.byref(dims), int(d_cq), B, n_q, _ptr(h, et, "h"), _ptr(w_dq, et, "w_dq"),
+                                  _ptr(w_uqk, et, "w_uqk"), _ptr(w_qr, et, "w_qr"), _ptr(c_kv, et, "c_kv"),
+                                  _ptr(k_pe, et, "k_pe"), _ptr(block_table, torch.int32, "block_table", True),
+                                  int(max_blocks_per_seq), int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"),
+                                  int(max_seqlen), _ptr(w_uvo, et, "w_uvo"), _ptr(out, et, "out"),
+                                  _ptr(lse, torch.float32, "lse", True), _ptr(workspace, None, "workspace"),
+                                  ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                                  _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_decode_absorbed", rc)
 
 
 def mla_decode_sparse_workspace_size(dims, B, n_q, topk) -> int:

@@ -164,9 +164,126 @@ SparseLayout sparse_layout(const mla_dims *d, int B, int n_q, int topk) {
   return L;
 }
 
+// K-split of a CUDA-core product so that about two CTAs per SM get work.
+int gemm_ksplit(int M, int N, int K) {
+  const int tiles = ((M + 63) / 64) * ((N + 63) / 64);
+  int ks = (296 + tiles - 1) / tiles;
+  ks = ks < 1 ? 1 : ks;
+  const int kmax = (K + 255) / 256;          // keep at least 256 of K per split
+  return ks > kmax ? kmax : ks;
+}
+
+GemmArgs gemm_args(int M, int N, int K, int batch, const void *A, int64_t sa_b, int64_t sa_m, int64_t sa_k,
+                   const void *B, int64_t sb_b, int64_t sb_k, int64_t sb_n, void *C, int64_t sc_b, int64_t sc_m,
+                   int64_t sc_n, bool split) {
+  return GemmArgs{M, N, K, batch, split ? gemm_ksplit(M, N, K) : 1, A, sa_b, sa_m, sa_k, B, sb_b, sb_k, sb_n,
+                  C, sc_b, sc_m, sc_n, nullptr};
+}
+
+// Decode from hidden states with folded weights: the workspace holds the decode workspace (whose
+// query region receives the absorbed queries), c_Q, the raw RoPE queries, o_lat and the K-split
+// partials of the products.
+struct AbsorbedLayout {
+  DecodeLayout dec;
+  size_t cq_off, qpe_off, olat_off, part_off, total;
+  GemmArgs g_cq, g_qlat, g_qpe, g_out;
+};
+
+AbsorbedLayout absorbed_layout(const mla_dims *d, int d_cq, int B, int n_q, int max_seqlen) {
+  AbsorbedLayout L{};
+  const int T = B * n_q, H = d->n_heads, W = d->d_c + d->d_rope, D = d->d_model;
+  const size_t e = elem(d);
+  L.dec = decode_layout(d, B, n_q, max_seqlen);
+  L.cq_off = L.dec.total;
+  L.qpe_off = L.cq_off + align256((size_t)T * d_cq * e);
+  L.olat_off = L.qpe_off + align256((size_t)T * H * d->d_rope * e + 16);
+  L.part_off = L.olat_off + align256((size_t)T * H * d->d_c * e);
+  // c_Q = h W_DQ;  q_lat^(s) = c_Q W_UQK^(s) into q_abs;  q_pe = c_Q W_QR;  u = o_lat W_UVO.
+  L.g_cq = gemm_args(T, d_cq, D, 1, nullptr, 0, D, 1, nullptr, 0, d_cq, 1, nullptr, 0, d_cq, 1, true);
+  L.g_qlat = gemm_args(T, d->d_c, d_cq, H, nullptr, 0, d_cq, 1, nullptr, (int64_t)d_cq * d->d_c, d->d_c, 1, nullptr, W,
+                       (int64_t)H * W, 1, false);
+  L.g_qpe = gemm_args(T, H * d->d_rope, d_cq, 1, nullptr, 0, d_cq, 1, nullptr, 0, (int64_t)H * d->d_rope, 1, nullptr,
+                      0, (int64_t)H * d->d_rope, 1, true);
+  L.g_out = gemm_args(T, D, H * d->d_c, 1, nullptr, 0, (int64_t)H * d->d_c, 1, nullptr, 0, D, 1, nullptr, 0, D, 1, true);
+  size_t part = 0;
+  for (const GemmArgs *g : {&L.g_cq, &L.g_qlat, &L.g_qpe, &L.g_out}) {
+    const size_t p = gemm_simt_workspace(*g);
+    part = p > part ? p : part;
+  }
+  L.total = L.part_off + align256(part);
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
+
+int mla_fold_query_weights(const mla_dims *dims, int d_cq, const void *w_uq, const void *w_uk, void *w_uqk,
+                           mla_stream_t stream) {
+  if (!dims_ok(dims) || d_cq <= 0 || !w_uq || !w_uk || !w_uqk) return MLA_ERR_INVALID_ARG;
+  const int H = dims->n_heads, dn = dims->d_nope, dc = dims->d_c;
+  // W_UQK[s] [d_cq x d_c] = W_UQ[:, s, :] [d_cq x d_nope] . W_UK[s]^T [d_nope x d_c]
+  GemmArgs g{d_cq, dc, dn, H, 1, w_uq, dn, (int64_t)H * dn, 1, w_uk, (int64_t)dc * dn, 1, dn, w_uqk,
+             (int64_t)d_cq * dc, dc, 1, nullptr};
+  return launch_gemm_simt(g, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_fold_output_weights(const mla_dims *dims, const void *w_uv, const void *w_o, void *w_uvo, mla_stream_t stream) {
+  if (!dims_ok(dims) || dims->d_model <= 0 || !w_uv || !w_o || !w_uvo) return MLA_ERR_INVALID_ARG;
+  const int H = dims->n_heads, dv = dims->d_v, dc = dims->d_c, D = dims->d_model;
+  // W_UVO[s] [d_c x D] = W_UV[s] [d_c x d_v] . W_O[s d_v .. (s+1) d_v - 1, :] [d_v x D]
+  GemmArgs g{dc, D, dv, H, 1, w_uv, (int64_t)dc * dv, dv, 1, w_o, (int64_t)dv * D, D, 1, w_uvo, (int64_t)dc * D, D, 1,
+             nullptr};
+  return launch_gemm_simt(g, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mla_decode_absorbed_workspace_size(const mla_dims *dims, int d_cq, int B, int n_q, int max_seqlen, size_t *bytes) {
+  if (!dims_ok(dims) || d_cq <= 0 || dims->d_model <= 0 || B <= 0 || n_q <= 0 || max_seqlen < n_q || !bytes)
+    return MLA_ERR_INVALID_ARG;
+  if (n_q * dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  *bytes = absorbed_layout(dims, d_cq, B, n_q, max_seqlen).total;
+  return MLA_OK;
+}
+
+int mla_decode_absorbed(const mla_dims *dims, int d_cq, int B, int n_q, const void *h, const void *w_dq,
+                        const void *w_uqk, const void *w_qr, const void *c_kv, const void *k_pe,
+                        const int32_t *block_table, int max_blocks_per_seq, int num_blocks, const int32_t *seqlens,
+                        int max_seqlen, const void *w_uvo, void *out, float *lse, void *workspace, size_t ws_bytes,
+                        int *dev_status, mla_stream_t stream) {
+  int rc = check_decode_args(dims, B, n_q, c_kv, k_pe, max_blocks_per_seq, num_blocks, seqlens, max_seqlen);
+  if (rc) return rc;
+  if (d_cq <= 0 || dims->d_model <= 0 || !h || !w_dq || !w_uqk || (!w_qr && dims->d_rope) || !w_uvo || !out)
+    return MLA_ERR_INVALID_ARG;
+  AbsorbedLayout L = absorbed_layout(dims, d_cq, B, n_q, max_seqlen);
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = dims->dtype == MLA_BF16;
+  char *ws = static_cast<char *>(workspace);
+  void *q_abs = ws + L.dec.q_off, *c_q = ws + L.cq_off, *q_pe = ws + L.qpe_off, *o_lat = ws + L.olat_off;
+  float *part = reinterpret_cast<float *>(ws + L.part_off);
+  // (1) c_Q = h W_DQ.
+  L.g_cq.A = h; L.g_cq.B = w_dq; L.g_cq.C = c_q; L.g_cq.part = part;
+  if ((rc = launch_gemm_simt(L.g_cq, bf16, st))) return rc;
+  // (2) latent queries q_lat^(s) = c_Q W_UQK^(s), straight into the absorbed query buffer.
+  L.g_qlat.A = c_q; L.g_qlat.B = w_uqk; L.g_qlat.C = q_abs; L.g_qlat.part = part;
+  if ((rc = launch_gemm_simt(L.g_qlat, bf16, st))) return rc;
+  // (3) RoPE queries q_pe^(s) = RoPE(c_Q W_QR^(s), position), into the query buffer's RoPE slots.
+  if (dims->d_rope) {
+    L.g_qpe.A = c_q; L.g_qpe.B = w_qr; L.g_qpe.C = q_pe; L.g_qpe.part = part;
+    if ((rc = launch_gemm_simt(L.g_qpe, bf16, st))) return rc;
+    if ((rc = launch_rope_into_query(B, n_q, dims->n_heads, dims->d_c, dims->d_rope, q_pe, seqlens, q_abs,
+                                     dims->rope_base, bf16, st)))
+      return rc;
+  }
+  // (4) split-KV attention and the merge of its partials into o_lat.
+  if ((rc = attention_impl(dims, B, n_q, q_abs, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                           max_seqlen, L.dec, ws, dev_status, st)))
+    return rc;
+  if ((rc = combine_impl(dims, B, n_q, seqlens, max_seqlen, nullptr, o_lat, lse, L.dec, ws, dev_status, st))) return rc;
+  // (5) u = sum_s o_lat^(s) W_UVO^(s).
+  L.g_out.A = o_lat; L.g_out.B = w_uvo; L.g_out.C = out; L.g_out.part = part;
+  return launch_gemm_simt(L.g_out, bf16, st);
+}
 
 int mla_decode_sparse_workspace_size(const mla_dims *dims, int B, int n_q, int topk, size_t *bytes) {
   if (!dims_ok(dims) || B <= 0 || n_q <= 0 || topk <= 0 || !bytes) return MLA_ERR_INVALID_ARG;

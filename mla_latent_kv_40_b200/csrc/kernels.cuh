@@ -127,6 +127,23 @@ int launch_cache_convert(const void *src, void *dst, int64_t num_rows, int W, bo
 // layout launch_combine reads (o_part [B][N][n_q*H][d_c] fp32, lse_part [B][N][n_q*H]).
 int launch_partials_to_splits(int N, int B, int n_q, int H, int d_c, const void *o_parts, const float *lse_parts,
                               bool bf16, float *o_part, float *lse_part, cudaStream_t st);
+// C[b] = A[b] B[b] with element strides (any transposition), fp32 accumulation on CUDA cores,
+// optionally split over K (fp32 partials in `part`, then summed into C).
+struct GemmArgs {
+  int M, N, K, batch, ksplit;
+  const void *A;
+  int64_t sa_b, sa_m, sa_k;
+  const void *B;
+  int64_t sb_b, sb_k, sb_n;
+  void *C;
+  int64_t sc_b, sc_m, sc_n;
+  float *part;              // [batch][ksplit][M][N] when ksplit > 1
+};
+size_t gemm_simt_workspace(const GemmArgs &g);
+int launch_gemm_simt(const GemmArgs &g, bool bf16, cudaStream_t st);
+// RoPE of the query-latent path's q_pe [T, H, d_R] into the RoPE slots of q_abs [T, H, d_c + d_R].
+int launch_rope_into_query(int B, int n_q, int H, int d_c, int d_rope, const void *q_pe_raw, const int32_t *seqlens,
+                           void *q_abs, float rope_base, bool bf16, cudaStream_t st);
 // Sparse decode: compact each query token's listed cache rows into its own run of 64-token pages.
 int launch_sparse_gather(int B, int n_q, int topk, const int32_t *idx, const int32_t *seqlens, int max_seqlen,
                          const CacheView &src, void *pool, bool dst_tiled, int elem, int32_t *counts,

@@ -23,7 +23,7 @@ __all__ = [
     "Dims", "DecodeCase", "PrefillCase", "DECODE_CASES", "PREFILL_CASES",
     "make_decode_inputs", "make_prefill_inputs", "make_append_inputs",
     "cache_row_of", "latent_bytes", "decode_flops", "prefill_flops", "make_decode_step_inputs", "append_flops",
-    "make_decode_inputs_device",
+    "make_decode_inputs_device", "make_query_path_inputs",
 ]
 
 
@@ -359,3 +359,19 @@ def make_decode_inputs_device(case: DecodeCase, device="cuda") -> dict:
     return dict(case=case, dims=d, seqlens=seqlens, block_table=bt, num_blocks=num_blocks,
                 max_blocks_per_seq=mbps, block_size=case.block_size, pool=pool,
                 q_nope=q_nope, q_pe=q_pe, w_uk=w_uk, w_uv=w_uv)
+
+
+def make_query_path_inputs(case: DecodeCase, d_cq: int, seed: int) -> dict:
+    """Hidden states and the query-side and output weights of the attention block, for the decode from
+    hidden states: h [B, n_q, D] ~ N(0,1); W_DQ [D, d_cq], W_UQ [d_cq, H, d_nope], W_QR [d_cq, H, d_R]
+    and W^O [H d_v, D], each ~ N(0,1)/sqrt(fan_in)."""
+    d = case.dims
+    gen = torch.Generator().manual_seed(seed)
+    dt = d.torch_dtype
+    return dict(
+        h=_randn(gen, (case.batch, case.n_q, d.d_model)).to(dt),
+        w_dq=_randn(gen, (d.d_model, d_cq), 1.0 / math.sqrt(d.d_model)).to(dt),
+        w_uq=_randn(gen, (d_cq, d.n_heads, d.d_nope), 1.0 / math.sqrt(d_cq)).to(dt),
+        w_qr=_randn(gen, (d_cq, d.n_heads, d.d_rope), 1.0 / math.sqrt(d_cq)).to(dt),
+        w_o=_randn(gen, (d.n_heads * d.d_v, d.d_model), 1.0 / math.sqrt(d.n_heads * d.d_v)).to(dt),
+    )
