@@ -146,6 +146,30 @@ MLA_API int mla_append_latent(const mla_dims *dims, int T, const void *h, const 
 MLA_API int mla_append_workspace_size(const mla_dims *dims, int T, size_t *bytes);
 
 /*
+ * mla_decode_step_workspace_size / mla_decode_step — one whole decode step:
+ *   the append of the step's n_q new tokens of every sequence, then mla_decode.
+ *   "DeepSeek-V3 解读 1: MLA", section "Key-Value 缓存": every generated token's
+ *   key and value enter the cache before it is attended to; here its latent
+ *   row c_KV = RMSNorm(h W_DKV) and its RoPE key (as mla_append_latent) are
+ *   written at positions seqlens[b] - n_q .. seqlens[b] - 1 of sequence b, and
+ *   the decode of mla_decode reads them.  On the tensor-core shapes the append
+ *   and the query absorption run as ONE kernel launch ahead of the attention
+ *   (its append-finish CTAs wait, with a bounded wait, for its projection CTAs);
+ *   other shapes run the same steps as separate launches.
+ *   h_new [B, n_q, D] (the new tokens' hidden states, token j of sequence b at
+ *   row b n_q + j); w_dkv, w_kr, rms_gamma as mla_append_latent; seqlens count
+ *   the cached tokens including the new ones; the other arguments as
+ *   mla_decode.  The cache rows of the new tokens are written (c_kv, k_pe).
+ *   workspace: >= mla_decode_step_workspace_size bytes, 256-byte aligned.
+ */
+MLA_API int mla_decode_step_workspace_size(const mla_dims *dims, int B, int n_q, int max_seqlen, size_t *bytes);
+MLA_API int mla_decode_step(const mla_dims *dims, int B, int n_q, const void *h_new, const void *w_dkv,
+                            const void *w_kr, const void *rms_gamma, const void *q_nope, const void *q_pe, void *c_kv,
+                            void *k_pe, const int32_t *block_table, int max_blocks_per_seq, int num_blocks,
+                            const int32_t *seqlens, int max_seqlen, const void *w_uk, const void *w_uv, void *out,
+                            float *lse, void *workspace, size_t ws_bytes, int *dev_status, mla_stream_t stream);
+
+/*
  * mla_absorb_q — the decode query in latent space.
  *   "Transformer升级之路：21、MLA好在哪里?（下）", section 双重投影, decoding
  *   column: q^(s) = x W_q^(s) W_k^(s)T lies in R^{d_c}; here

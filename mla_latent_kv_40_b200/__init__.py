@@ -68,6 +68,9 @@ _sigs = {
     "mla_decode_partial": [_D, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, ctypes.c_size_t,
                            _P, _P],
     "mla_merge_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode_step_workspace_size": [_D, _I, _I, _I, _SZ],
+    "mla_decode_step": [_D, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _I, _P, _P, _P, _P, _P,
+                        ctypes.c_size_t, _P, _P],
     "mla_fold_query_weights": [_D, _I, _P, _P, _P, _P],
     "mla_fold_output_weights": [_D, _P, _P, _P, _P],
     "mla_decode_absorbed_workspace_size": [_D, _I, _I, _I, _I, _SZ],
@@ -217,6 +220,36 @@ def mla_decode_noalloc(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_p
                                  _ptr(lse, torch.float32, "lse", True), _ptr(dev_status, torch.int32, "dev_status", True),
                                  _stream(stream))
     _check("mla_decode_noalloc", rc)
+
+
+def mla_decode_step_workspace_size(dims, B, n_q, max_seqlen) -> int:
+    n = ctypes.c_size_t(0)
+    _check("mla_decode_step_workspace_size",
+           _lib.mla_decode_step_workspace_size(ctypes.byref(dims), int(B), int(n_q), int(max_seqlen), ctypes.byref(n)))
+    return int(n.value)
+
+
+def mla_decode_step(dims, h_new, w_dkv, w_kr, rms_gamma, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq,
+                    num_blocks, seqlens, max_seqlen, w_uk, w_uv, out, lse, workspace, dev_status=None, stream=None):
+    """Append of the n_q new tokens of every sequence (h_new [B, n_q, D]) and the decode, in one call."""
+    et = _elem_dtype(dims)
+    B, n_q = q_nope.shape[0], q_nope.shape[1]
+    if h_new.shape[0] * (h_new.shape[1] if h_new.dim() == 3 else 1) != B * n_q:
+        raise ValueError("h_new must hold B * n_q rows")
+    for n, t in (("h_new", h_new), ("w_dkv", w_dkv), ("w_kr", w_kr), ("rms_gamma", rms_gamma), ("q_nope", q_nope),
+                 ("q_pe", q_pe), ("block_table", block_table), ("seqlens", seqlens), ("w_uk", w_uk), ("w_uv", w_uv),
+                 ("out", out), ("lse", lse)):
+        _dense(t, n)
+    rc = _lib.mla_decode_step(ctypes.byref(dims), B, n_q, _ptr(h_new, et, "h_new"), _ptr(w_dkv, et, "w_dkv"),
+                              _ptr(w_kr, et, "w_kr"), _ptr(rms_gamma, et, "rms_gamma", True),
+                              _ptr(q_nope, et, "q_nope"), _ptr(q_pe, et, "q_pe"), _ptr(c_kv, et, "c_kv"),
+                              _ptr(k_pe, et, "k_pe"), _ptr(block_table, torch.int32, "block_table", True),
+                              int(max_blocks_per_seq), int(num_blocks), _ptr(seqlens, torch.int32, "seqlens"),
+                              int(max_seqlen), _ptr(w_uk, et, "w_uk"), _ptr(w_uv, et, "w_uv"), _ptr(out, et, "out"),
+                              _ptr(lse, torch.float32, "lse", True), _ptr(workspace, None, "workspace"),
+                              ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+                              _ptr(dev_status, torch.int32, "dev_status", True), _stream(stream))
+    _check("mla_decode_step", rc)
 
 
 def mla_decode_partial(dims, q_nope, q_pe, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,

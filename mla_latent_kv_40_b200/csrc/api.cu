@@ -214,6 +214,39 @@ AbsorbedLayout absorbed_layout(const mla_dims *d, int d_cq, int B, int n_q, int 
   return L;
 }
 
+// Sequence and position of each new token of a decode step: token t = b n_q + j sits at
+// seqlens[b] - n_q + j.
+__global__ void step_positions_kernel(int B, int n_q, const int32_t *seqlens, int32_t *seq_idx, int32_t *pos) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= B * n_q) return;
+  const int b = t / n_q;
+  seq_idx[t] = b;
+  pos[t] = seqlens[b] - n_q + t % n_q;
+}
+
+// Decode step workspace: the fused kernel's completion counter, the append's split-K partials, the
+// new tokens' (sequence, position) for the unfused path, then the decode workspace.
+struct StepLayout {
+  size_t counter_off, part_off, idx_off, dec_off, total;
+  int nsplit, kps;
+  DecodeLayout dec;
+};
+
+StepLayout step_layout(const mla_dims *d, int B, int n_q, int max_seqlen) {
+  StepLayout L{};
+  const int T = B * n_q, W = d->d_c + d->d_rope;
+  L.counter_off = 0;
+  L.part_off = 256;
+  L.nsplit = 1;
+  L.kps = d->d_model;
+  const size_t part = append_mma_workspace(T, d->d_model, W, &L.nsplit, &L.kps);
+  L.idx_off = L.part_off + align256(part);
+  L.dec_off = L.idx_off + align256((size_t)2 * T * sizeof(int32_t));
+  L.dec = decode_layout(d, B, n_q, max_seqlen);
+  L.total = L.dec_off + L.dec.total;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -392,6 +425,57 @@ int mla_append_latent(const mla_dims *dims, int T, const void *h, const void *w_
     return launch_append_mma(a, workspace, st);
   }
   return launch_append(a, bf16, st);
+}
+
+int mla_decode_step_workspace_size(const mla_dims *dims, int B, int n_q, int max_seqlen, size_t *bytes) {
+  if (!dims_ok(dims) || dims->d_model <= 0 || B <= 0 || n_q <= 0 || max_seqlen < n_q || !bytes)
+    return MLA_ERR_INVALID_ARG;
+  if (n_q * dims->n_heads > 256) return MLA_ERR_UNSUPPORTED;
+  *bytes = step_layout(dims, B, n_q, max_seqlen).total;
+  return MLA_OK;
+}
+
+int mla_decode_step(const mla_dims *dims, int B, int n_q, const void *h_new, const void *w_dkv, const void *w_kr,
+                    const void *rms_gamma, const void *q_nope, const void *q_pe, void *c_kv, void *k_pe,
+                    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, const int32_t *seqlens,
+                    int max_seqlen, const void *w_uk, const void *w_uv, void *out, float *lse, void *workspace,
+                    size_t ws_bytes, int *dev_status, mla_stream_t stream) {
+  int rc = check_decode_args(dims, B, n_q, c_kv, k_pe, max_blocks_per_seq, num_blocks, seqlens, max_seqlen);
+  if (rc) return rc;
+  if (dims->d_model <= 0 || !h_new || !w_dkv || (!w_kr && dims->d_rope) || !q_nope || (!q_pe && dims->d_rope) ||
+      !w_uk || !w_uv || !out)
+    return MLA_ERR_INVALID_ARG;
+  const StepLayout L = step_layout(dims, B, n_q, max_seqlen);
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char *ws = static_cast<char *>(workspace);
+  const int T = B * n_q;
+  int32_t *seq_idx = reinterpret_cast<int32_t *>(ws + L.idx_off), *pos = seq_idx + T;
+  char *dws = ws + L.dec_off;
+  void *qbuf = dws + L.dec.q_off;
+  const bool bf16 = dims->dtype == MLA_BF16;
+  AppendArgs ap = append_args(dims, T, h_new, w_dkv, w_kr, rms_gamma, seq_idx, pos, c_kv, k_pe, block_table, B,
+                              max_blocks_per_seq, num_blocks, dev_status);
+  AbsorbArgs ab{B, n_q, dims->n_heads, dims->d_c, dims->d_rope, dims->d_nope,
+                q_nope, q_pe, w_uk, seqlens, qbuf, dims->rope_base};
+  if (bf16 && L.dec.use_tc && decode_prep_supported(ap, ab)) {
+    // One launch: append of the new tokens and the query absorption.
+    if ((rc = launch_decode_prep(ap, ab, ws + L.part_off, L.nsplit, L.kps, reinterpret_cast<unsigned *>(ws + L.counter_off),
+                                 st)))
+      return rc;
+  } else {
+    step_positions_kernel<<<(T + 255) / 256, 256, 0, st>>>(B, n_q, seqlens, seq_idx, pos);
+    if (cudaGetLastError() != cudaSuccess) return MLA_ERR_CUDA;
+    if ((rc = mla_append_latent(dims, T, h_new, w_dkv, w_kr, rms_gamma, seq_idx, pos, c_kv, k_pe, block_table, B,
+                                max_blocks_per_seq, num_blocks, ws + L.part_off, L.idx_off - L.part_off, dev_status,
+                                stream)))
+      return rc;
+    if ((rc = absorb_dispatch(ab, bf16, dev_status, st))) return rc;
+  }
+  if ((rc = attention_impl(dims, B, n_q, qbuf, c_kv, k_pe, block_table, max_blocks_per_seq, num_blocks, seqlens,
+                           max_seqlen, L.dec, dws, dev_status, st)))
+    return rc;
+  return combine_impl(dims, B, n_q, seqlens, max_seqlen, w_uv, out, lse, L.dec, dws, dev_status, st);
 }
 
 int mla_absorb_q(const mla_dims *dims, int B, int n_q, const void *q_nope, const void *q_pe,

@@ -122,6 +122,11 @@ int launch_absorb_tc(const AbsorbArgs &a, int *dev_status, cudaStream_t st);
 bool append_tc_supported(const AppendArgs &a, bool bf16);
 int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split, cudaStream_t st);
 int launch_append_finish(const AppendArgs &a, const void *ws, int nsplit, cudaStream_t st);
+// Fused decode-step preparation: the append of the step's new tokens and the query absorption in
+// one launch (tensor-core shapes only).  `counter` is 4 bytes of workspace, zeroed by the launcher.
+bool decode_prep_supported(const AppendArgs &ap, const AbsorbArgs &ab);
+int launch_decode_prep(const AppendArgs &ap, const AbsorbArgs &ab, void *part, int nsplit, int k_per_split,
+                       unsigned *counter, cudaStream_t st);
 int launch_cache_convert(const void *src, void *dst, int64_t num_rows, int W, bool to_tiled, cudaStream_t st);
 // Cross-device merge: partials [N][B][n_q][H][d_c] (dtype) and lses [N][B][n_q][H] -> the split
 // layout launch_combine reads (o_part [B][N][n_q*H][d_c] fp32, lse_part [B][N][n_q*H]).

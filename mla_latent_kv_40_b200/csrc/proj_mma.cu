@@ -9,6 +9,7 @@
 //    ("Transformer升级之路：21、MLA好在哪里?（下）", section 双重投影, decoding column).
 // Tiles are 64 rows x 64 or 128 columns, 4 warps of 16 rows each, operands
 // staged by cp.async into padded shared tiles and read with ldmatrix.
+#include "append_finish.cuh"
 #include "kernels.cuh"
 #include "mma_tile.cuh"
 #include "sm100.cuh"
@@ -104,69 +105,11 @@ constexpr int kFinThreads = 288;   // (d_c + d_R) / 2 column pairs of the V3 and
 
 __global__ void __launch_bounds__(kFinThreads)
 append_finish_kernel(AppendArgs a, const float *part, int nsplit) {
-  __shared__ float red[kFinThreads / 32];
-  const int W = a.d_c + a.d_rope, npair = W / 2;
-  const int tok = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  __shared__ float red[kFinishScratch];
   sm100::grid_dep_launch();
   sm100::grid_dep_wait();   // the partials come from the projection kernel just before
-  const int64_t split_stride = (int64_t)a.T * W / 2;   // in float2
-  const float2 *pp = reinterpret_cast<const float2 *>(part) + (int64_t)tok * npair;
-  constexpr int kMaxPairsPerThr = 2;
-  float2 v[kMaxPairsPerThr];
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < kMaxPairsPerThr; ++i) {
-    const int j2 = tid + i * kFinThreads;
-    float2 acc = make_float2(0.f, 0.f);
-    if (j2 < npair) {
-#pragma unroll 8
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float2 x = pp[sp * split_stride + j2];
-        acc.x += x.x;
-        acc.y += x.y;
-      }
-      if (2 * j2 < a.d_c) ss += acc.x * acc.x + acc.y * acc.y;
-    }
-    v[i] = acc;
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if (lane == 0) red[warp] = ss;
-  __syncthreads();
-  float tot = 0.f;
-#pragma unroll
-  for (int w = 0; w < kFinThreads / 32; ++w) tot += red[w];
-  const float inv = rsqrtf(tot / (float)a.d_c + a.rms_eps);
-  const int b = a.seq_idx[tok], p = a.pos[tok];
-  if (b < 0 || b >= a.num_seqs || p < 0 || (int64_t)p >= (int64_t)a.max_blocks_per_seq * a.block_size) {
-    if (tid == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
-    return;
-  }
-  const int64_t row = cache_row(a.block_table, a.max_blocks_per_seq, a.num_blocks, a.block_size, b, p);
-  if (row < 0) {
-    if (tid == 0) report(a.dev_status, MLA_ERR_BAD_INDEX);
-    return;
-  }
-  auto at = [&](int d) {
-    return latent_elem<__nv_bfloat16>(a.c_kv, a.k_pe, a.ckv_stride, a.kpe_stride, a.layout, a.d_c, W, row, d);
-  };
-  const __nv_bfloat16 *gm = static_cast<const __nv_bfloat16 *>(a.gamma);
-#pragma unroll
-  for (int i = 0; i < kMaxPairsPerThr; ++i) {
-    const int j2 = tid + i * kFinThreads, j = 2 * j2;
-    if (j2 >= npair) continue;
-    if (j < a.d_c) {
-      const float g0 = gm ? __bfloat162float(gm[j]) : 1.f, g1 = gm ? __bfloat162float(gm[j + 1]) : 1.f;
-      *at(j) = __float2bfloat16_rn(v[i].x * inv * g0);
-      *at(j + 1) = __float2bfloat16_rn(v[i].y * inv * g1);
-    } else {
-      float cs_, sn_;
-      rope_cos_sin(p, (j - a.d_c) / 2, a.d_rope, a.rope_base, &cs_, &sn_);
-      *at(j) = __float2bfloat16_rn(v[i].x * cs_ - v[i].y * sn_);
-      *at(j + 1) = __float2bfloat16_rn(v[i].x * sn_ + v[i].y * cs_);
-    }
-  }
+  const int tok = blockIdx.x;
+  append_finish_token<kFinThreads>(a, part, nsplit, tok, a.seq_idx[tok], a.pos[tok], red);
 }
 
 size_t append_mma_workspace(int T, int d_model, int W, int *nsplit, int *k_per_split) {

@@ -13,6 +13,7 @@
 // once, by TMA), the activation rows are the N side (N = 64 per CTA), and the
 // fp32 accumulator sits in 64 tensor-memory columns.  One elected thread
 // issues the TMA loads and the MMAs; all warps drain tensor memory.
+#include "append_finish.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 #include "tmap.cuh"
@@ -40,11 +41,10 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int *dev
 // CTA = (head s, 128 latent columns m0.., 64 query rows r0..):
 //   D[m][r] = sum_k W_UK[s][m0 + m][k] q_nope[r0 + r][s][k]   (A and B both K-major)
 // The CTAs with blockIdx.y == 0 .. 3 share the RoPE of their 64 rows.
-__global__ void __launch_bounds__(kTcThreads)
-absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_q, AbsorbArgs a,
-                 int *dev_status) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// (s, by, bz) play the roles of (blockIdx.x, blockIdx.y, blockIdx.z) of a grid (H, d_c / 128, rows / 64)
+// whose y extent is ny; sm is the CTA's 1024-byte aligned dynamic shared memory.
+__device__ __forceinline__ void absorb_tc_body(const CUtensorMap &map_w, const CUtensorMap &map_q, const AbsorbArgs &a,
+                                               int *dev_status, int s, int by, int bz, int ny, unsigned char *sm) {
   __shared__ __align__(8) uint64_t bar_full, bar_mma;
   __shared__ uint32_t tmem_slot;
   const int nkc = a.d_nope / 64;
@@ -52,7 +52,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
   unsigned char *Bs = As + nkc * kAChunk;                  // [nkc][64 x 128 B]
   __nv_bfloat16 *Os = reinterpret_cast<__nv_bfloat16 *>(Bs + nkc * kBChunk);   // [64][128 + 8]
   constexpr int ldo = 128 + 8;
-  const int s = blockIdx.x, m0 = blockIdx.y * 128, r0 = blockIdx.z * kTcN;
+  const int m0 = by * 128, r0 = bz * kTcN;
   const int R = a.B * a.n_q, W = a.d_c + a.d_rope;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   grid_dep_launch();   // reads below touch inputs only; q_out is written after grid_dep_wait()
@@ -93,13 +93,13 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
     asm volatile("bar.sync 1, 96;" ::: "memory");       // warps 1-3 only
     grid_dep_wait();                                       // q_out may still be read by an earlier kernel
     constexpr int kRowsPerWarp = 8;
-    const int nr = (kTcN - (int)blockIdx.y + (int)gridDim.y - 1) / (int)gridDim.y;
+    const int nr = (kTcN - by + ny - 1) / ny;
     for (int w0 = (warp - 1) * kRowsPerWarp; w0 < nr; w0 += 3 * kRowsPerWarp) {
       int pos[kRowsPerWarp];
       __nv_bfloat162 xy[kRowsPerWarp];
 #pragma unroll
       for (int k = 0; k < kRowsPerWarp; ++k) {
-        const int gr = r0 + blockIdx.y + gridDim.y * (w0 + k);
+        const int gr = r0 + by + ny * (w0 + k);
         const bool live = w0 + k < nr && gr < R && lane < half;
         pos[k] = live ? max(0, a.seqlens[gr / a.n_q] - a.n_q + gr % a.n_q) : -1;   // -1: nothing to do
         xy[k] = live ? *reinterpret_cast<const __nv_bfloat162 *>(qp + ((int64_t)gr * a.H + s) * a.d_rope + 2 * lane)
@@ -108,7 +108,7 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
 #pragma unroll
       for (int k = 0; k < kRowsPerWarp; ++k) {
         if (pos[k] < 0) continue;
-        const int gr = r0 + blockIdx.y + gridDim.y * (w0 + k);
+        const int gr = r0 + by + ny * (w0 + k);
         float cs, sn;
         rope_cos_sin_theta(pos[k], theta[lane], &cs, &sn);
         const float x = __low2float(xy[k]), y = __high2float(xy[k]);
@@ -167,6 +167,17 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
   }
 }
 
+__device__ __forceinline__ unsigned char *align1024(unsigned char *p) {
+  return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__global__ void __launch_bounds__(kTcThreads)
+absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_q, AbsorbArgs a,
+                 int *dev_status) {
+  extern __shared__ unsigned char smem_raw[];
+  absorb_tc_body(map_w, map_q, a, dev_status, blockIdx.x, blockIdx.y, blockIdx.z, gridDim.y, align1024(smem_raw));
+}
+
 // ------------------------------------------------------------------ append projection
 // CTA = (128 output columns m0.. of [W_DKV | W_KR], K-split ks, 64 tokens t0..):
 //   D[m][t] = sum_{k in split} W[k][m0 + m] h[t0 + t][k]     (A = W^T is M-major, B = h is K-major)
@@ -174,16 +185,15 @@ absorb_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constan
 constexpr int kApStages = 4;
 constexpr uint32_t kApStageBytes = kAChunk + kBChunk;      // A: 2 M-chunks of [64 K x 128 B]; B: [64 x 128 B]
 
-__global__ void __launch_bounds__(kTcThreads)
-append_tc_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_constant__ CUtensorMap map_wr,
-                 const __grid_constant__ CUtensorMap map_h, int T, int d_c, int d_rope, int k_per_split, int D,
-                 float *part, int *dev_status) {
-  extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// (bx, ks, bz) play the roles of (blockIdx.x, blockIdx.y, blockIdx.z) of a grid (columns / 128, splits, T / 64).
+__device__ __forceinline__ void append_tc_body(const CUtensorMap &map_wd, const CUtensorMap &map_wr,
+                                               const CUtensorMap &map_h, int T, int d_c, int d_rope, int k_per_split,
+                                               int D, float *part, int *dev_status, int bx, int ks, int bz,
+                                               unsigned char *sm) {
   __shared__ __align__(8) uint64_t bar_full[kApStages], bar_empty[kApStages], bar_mma;
   __shared__ uint32_t tmem_slot;
   const int W = d_c + d_rope;
-  const int m0 = blockIdx.x * 128, ks = blockIdx.y, t0 = blockIdx.z * kTcN;
+  const int m0 = bx * 128, t0 = bz * kTcN;
   const int kbeg = ks * k_per_split, kend = min(D, kbeg + k_per_split);
   const int nst = (kend - kbeg + 63) / 64;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -274,6 +284,85 @@ append_tc_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_consta
   }
 }
 
+__global__ void __launch_bounds__(kTcThreads)
+append_tc_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_constant__ CUtensorMap map_wr,
+                 const __grid_constant__ CUtensorMap map_h, int T, int d_c, int d_rope, int k_per_split, int D,
+                 float *part, int *dev_status) {
+  extern __shared__ unsigned char smem_raw[];
+  append_tc_body(map_wd, map_wr, map_h, T, d_c, d_rope, k_per_split, D, part, dev_status, blockIdx.x, blockIdx.y,
+                 blockIdx.z, align1024(smem_raw));
+}
+
+// ------------------------------------------------------------------ fused decode-step preparation
+// One launch does the work that precedes the attention of a decode step: the append of the step's
+// new tokens (projection, then RMSNorm / RoPE / scatter) and the query absorption.  Its CTAs take
+// three roles by block index:
+//   [0, nA)            append projection CTAs (split-K partials); each signals the counter when done;
+//   [nA, nA + nB)      absorption CTAs (independent of the append);
+//   [nA + nB, + T)     append finish CTAs, one per new token: they wait (bounded) until all nA
+//                      projection CTAs have signalled, then finish their token.
+// The finish CTAs come last, so every CTA they wait for is dispatched before them.
+struct PrepParams {
+  AppendArgs ap;
+  AbsorbArgs ab;
+  float *part;
+  int nsplit, k_per_split;
+  int nA, a_nx, a_ny;                 // append grid (columns / 128, splits, tokens / 64)
+  int nB, b_ny, b_nz;                 // absorb grid (H, d_c / 128, rows / 64)
+  unsigned *counter;                  // zeroed before the launch
+};
+
+__global__ void __launch_bounds__(kTcThreads)
+decode_prep_kernel(const __grid_constant__ CUtensorMap map_wd, const __grid_constant__ CUtensorMap map_wr,
+                   const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_w,
+                   const __grid_constant__ CUtensorMap map_q, const PrepParams pp) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *sm = align1024(smem_raw);
+  int id = blockIdx.x;
+  if (id < pp.nA) {
+    const int bx = id % pp.a_nx, ks = (id / pp.a_nx) % pp.a_ny, bz = id / (pp.a_nx * pp.a_ny);
+    append_tc_body(map_wd, map_wr, map_h, pp.ap.T, pp.ap.d_c, pp.ap.d_rope, pp.k_per_split, pp.ap.d_model, pp.part,
+                   pp.ap.dev_status, bx, ks, bz, sm);
+    __threadfence();                  // this CTA's partials, then its signal (release at GPU scope)
+    __syncthreads();
+    if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(pp.counter) : "memory");
+    return;
+  }
+  id -= pp.nA;
+  if (id < pp.nB) {
+    const int s = id % pp.ab.H, by = (id / pp.ab.H) % pp.b_ny, bz = id / (pp.ab.H * pp.b_ny);
+    absorb_tc_body(map_w, map_q, pp.ab, pp.ap.dev_status, s, by, bz, pp.b_ny, sm);
+    return;
+  }
+  const int tok = id - pp.nB;
+  __shared__ float red[kFinishScratch];
+  __shared__ int ready;
+  grid_dep_launch();
+  grid_dep_wait();                    // earlier kernels may still read the cache rows written below
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      unsigned v;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(pp.counter) : "memory");
+      if ((int)v >= pp.nA) break;
+      if (globaltimer_ns() - t0 > kWaitNs) {
+        report(pp.ap.dev_status, MLA_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(200);
+    }
+    ready = ok;
+  }
+  __syncthreads();
+  if (!ready) return;
+  const int n_q = pp.ab.n_q;
+  const int b = tok / n_q;
+  const int p = pp.ab.seqlens[b] - n_q + tok % n_q;
+  append_finish_token<kTcThreads>(pp.ap, pp.part, pp.nsplit, tok, b, p, red);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------ host side
@@ -319,6 +408,46 @@ int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split,
   const dim3 grid((W + 127) / 128, nsplit, (a.T + kTcN - 1) / kTcN);
   return launch_pdl(append_tc_kernel, grid, dim3(kTcThreads), smem, st, mwd, mwr, mh, a.T, a.d_c, a.d_rope,
                     k_per_split, a.d_model, static_cast<float *>(ws), a.dev_status) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+bool decode_prep_supported(const AppendArgs &ap, const AbsorbArgs &ab) {
+  return append_tc_supported(ap, true) && append_mma_supported(ap, true) && absorb_tc_supported(ab, true);
+}
+
+int launch_decode_prep(const AppendArgs &ap, const AbsorbArgs &ab, void *part, int nsplit, int k_per_split,
+                       unsigned *counter, cudaStream_t st) {
+  const int W = ap.d_c + ap.d_rope, R = ab.B * ab.n_q;
+  CUtensorMap mwd, mwr, mh, mw, mq;
+  if (!make_tmap_bf16(&mwd, ap.w_dkv, ap.d_c, ap.d_model, (uint64_t)ap.d_c * 2, 64) ||
+      !make_tmap_bf16(&mwr, ap.w_kr, ap.d_rope, ap.d_model, (uint64_t)ap.d_rope * 2, 64) ||
+      !make_tmap_bf16(&mh, ap.h, ap.d_model, ap.T, (uint64_t)ap.d_model * 2, kTcN) ||
+      !make_tmap_bf16(&mw, ab.w_uk, ab.d_nope, (uint64_t)ab.H * ab.d_c, (uint64_t)ab.d_nope * 2, 128) ||
+      !make_tmap_bf16(&mq, ab.q_nope, (uint64_t)ab.H * ab.d_nope, R, (uint64_t)ab.H * ab.d_nope * 2, kTcN))
+    return MLA_ERR_CUDA;
+  PrepParams pp;
+  pp.ap = ap;
+  pp.ab = ab;
+  pp.part = static_cast<float *>(part);
+  pp.nsplit = nsplit;
+  pp.k_per_split = k_per_split;
+  pp.a_nx = (W + 127) / 128;
+  pp.a_ny = nsplit;
+  pp.nA = pp.a_nx * nsplit * ((ap.T + kTcN - 1) / kTcN);
+  pp.b_ny = ab.d_c / 128;
+  pp.b_nz = (R + kTcN - 1) / kTcN;
+  pp.nB = ab.H * pp.b_ny * pp.b_nz;
+  pp.counter = counter;
+  const int nkc = ab.d_nope / 64;
+  const size_t smem_ab = 1024 + nkc * (kAChunk + kBChunk) + sizeof(__nv_bfloat16) * kTcN * (128 + 8);
+  const size_t smem_ap = 1024 + kApStages * kApStageBytes;
+  const size_t smem = smem_ab > smem_ap ? smem_ab : smem_ap;
+  if (cudaFuncSetAttribute(decode_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+    return MLA_ERR_CUDA;
+  if (cudaMemsetAsync(counter, 0, sizeof(unsigned), st) != cudaSuccess) return MLA_ERR_CUDA;
+  return launch_pdl(decode_prep_kernel, dim3(pp.nA + pp.nB + ap.T), dim3(kTcThreads), smem, st, mwd, mwr, mh, mw, mq,
+                    pp) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
 }
