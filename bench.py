@@ -609,6 +609,28 @@ def run_mla(args):
     barrier()
     api_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
 
+    # The whole step as one call: mla_decode_step (append of the new tokens and the query absorption
+    # in one launch on these shapes, then attention and combine).
+    step_ws = mla.alloc_workspace(mla.mla_decode_step_workspace_size(dims, B, n_q, max_seqlen))
+    h_step = dev["h_new"].view(B, n_q, -1)
+
+    def fused_step():
+        mla.mla_decode_step(dims, h_step, dev["w_dkv"], dev["w_kr"], dev["gamma"], dev["q_nope"], dev["q_pe"], c_kv,
+                            k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"], dev["seqlens"], max_seqlen,
+                            dev["w_uk"], dev["w_uv"], out, lse, step_ws, status)
+
+    for _ in range(3):
+        fused_step()
+    torch.cuda.synchronize()
+    barrier()
+    a0.record(stream)
+    for _ in range(args.steps):
+        fused_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    fused_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
+
     # End to end through the public calls: pinned host inputs in, result out, every step's copies inside the
     # timed region.  The inputs of step i+1 are copied (copy stream) while step i computes, into the other of
     # two device buffer sets, and step i's result goes back (a second copy stream) while step i+1 computes.
@@ -723,12 +745,15 @@ def run_mla(args):
         "api_step": {"calls": "mla_append_latent + mla_decode, one stream", "ms_per_step": api_ms,
                      "tflops": step_flops * world / (api_ms * 1e-3) / 1e12,
                      "roofline_frac": max(t_hbm, t_flop) / (api_ms * 1e-3)},
+        "fused_step": {"calls": "mla_decode_step (append + absorption in one launch, attention, combine)",
+                       "ms_per_step": fused_ms, "tflops": step_flops * world / (fused_ms * 1e-3) / 1e12,
+                       "roofline_frac": max(t_hbm, t_flop) / (fused_ms * 1e-3)},
     }
     if e2e:
         line["e2e"] = {"value": step_flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": UNIT,
                        "h2d_bytes_per_step": e2e["h2d_bytes_per_step"], "d2h_bytes_per_step": e2e["d2h_bytes_per_step"],
                        "ms_per_step": e2e["ms_per_step"]}
-    del dec_ws
+    del dec_ws, step_ws
     if world == 1 and rank == 0 and not args.no_prefill and args.only == "all":
         line["prefill"] = measure_prefill(mla, torch, peaks)
     if world == 1 and rank == 0 and not args.no_configs and args.only == "all":

@@ -71,13 +71,16 @@ constexpr uint32_t kPWriters = 4;                 // softmax warps that write on
 constexpr uint32_t kPaWords = 36;                  // per writer warp: 32 row rescale factors, a flag word, padding
 constexpr uint32_t kStgBytes = 4096 + kPaWords * 4;                // score CTA: one warp's P rows + factors, staged
 constexpr uint32_t kPTxBytes = kPWriters * kStgBytes;              // bytes that fill one P slot
+// A P slot (value CTA) and a P staging tile (score CTA) hold a page of P (16 KB) followed by its
+// rescale factors, so that ONE bulk copy moves both; the stride keeps every P page 1024-aligned.
+constexpr uint32_t kPSlotBytes = ((kPTxBytes + 1023) / 1024) * 1024;   // 17408
 constexpr uint32_t kQpeOff = 0;                                    // score CTA: Q rope part, [128 x 64] bf16
 constexpr uint32_t kKOff = kRows * 128;                            // score CTA: key stages
 constexpr uint32_t kPOff = kVStages * kVStageBytes;                // value CTA: P slots
 constexpr uint32_t kStgOff = kKOff + kKStages * kKStageBytes;      // score CTA: P pages of both halves, factors
-constexpr uint32_t kScoreEnd = kStgOff + 2 * kPTxBytes, kValueEnd = kPOff + kPSlots * kPBytes;
+constexpr uint32_t kScoreEnd = kStgOff + 2 * kPSlotBytes, kValueEnd = kPOff + kPSlots * kPSlotBytes;
 constexpr uint32_t kRegionA = ((kScoreEnd > kValueEnd ? kScoreEnd : kValueEnd) + 1023) & ~1023u;   // 214016
-static_assert(kPOff + kPSlots * kPBytes <= kRegionA, "value-CTA tiles must fit the shared region");
+static_assert(kPOff + kPSlots * kPSlotBytes <= kRegionA, "value-CTA tiles must fit the shared region");
 #ifndef MLA_TC_PREFETCH_PAGES
 #define MLA_TC_PREFETCH_PAGES 0
 #endif
@@ -108,9 +111,6 @@ struct Req {
 };
 
 struct SmemB {                       // small region after the tiles
-  // value CTA, per P slot and writer warp: the rescale factors of its 32 rows, then a flag word
-  // ("some row of this tile rescaled") and padding; filled by the score CTA's bulk copies.
-  float pa[kPSlots][kPWriters][kPaWords];
   float stat_l[kRows], stat_m[kRows];// value CTA: row sum and reference max of a finished unit
   float xmax[2][2][kRows];           // score CTA: the two softmax halves' tile maxima (double-buffered)
   float xl[2][kRows];                // score CTA: the two halves' row sums at the end of a unit
@@ -126,8 +126,21 @@ struct SmemB {                       // small region after the tiles
 constexpr size_t kSmemBytes = 1024 + kRegionA + sizeof(SmemB);
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 
+// Value CTA: shared address of the rescale factors that arrived with P slot pb, per writer warp: its
+// 32 rows' factors, a flag word ("some row of this tile rescaled") and padding.
+__device__ __forceinline__ uint32_t slot_factors(uint32_t tiles_s, int pb) {
+  return tiles_s + kPOff + pb * kPSlotBytes + kPBytes;
+}
+
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 struct TcParams {
   int B, n_q, H, n_rb, U, max_seqlen;
+  int kv_begin, kv_end;              // attend to keys in [kv_begin, kv_end) only (kv_begin a multiple of 64)
   const __nv_bfloat16 *q;            // [B, n_q, H, 576]
   const int32_t *seqlens, *block_table;
   int max_blocks_per_seq, num_blocks, block_size;
@@ -140,7 +153,6 @@ struct TcParams {
   const unsigned char *tiled;        // tiled page pool (pages move by bulk copy), or NULL: row pool via TMA maps
   const unsigned char *row_pool;     // row pool base (c_kv) for L2 prefetch
   int rows_contig;                   // row pool with fused 576-wide rows: a page is 73728 contiguous bytes
-  int kv_begin, kv_end;              // attend to keys in [kv_begin, kv_end) only (kv_begin a multiple of 64)
 };
 
 __device__ __forceinline__ int seq_len_clamped(const TcParams &p, int b) {
@@ -168,7 +180,7 @@ __device__ __forceinline__ int cluster_of(long long t, long long T, long long C)
 
 // Warp-level plan: total tiles, this cluster's range, its first unit and the
 // tile / segment prefixes of that unit.  Every CTA computes the same values.
-__device__ void make_plan(const TcParams &p, SmemB &sb, int cid, int C) {
+__device__ __forceinline__ void make_plan(const TcParams &p, SmemB &sb, int cid, int C) {
   const int lane = threadIdx.x & 31;
   long long total = 0;
   for (int u0 = 0; u0 < p.U; u0 += 32) {
@@ -232,7 +244,7 @@ struct SegIter {
   int u, prefix, seg_prefix;
   long long pos, end, total;
   int C;
-  __device__ bool next(const TcParams &p, int cid, int &b, int &rb, int &t0, int &t1, int &segid, bool &first_of_unit,
+  __device__ __forceinline__ bool next(const TcParams &p, int cid, int &b, int &rb, int &t0, int &t1, int &segid, bool &first_of_unit,
                        int &nseg_unit) {
     while (pos < end && u < p.U) {
       const int nt = unit_tiles(p, u);
@@ -319,12 +331,12 @@ __device__ __forceinline__ int64_t tile_row(const TcParams &p, int b, int t) {
 struct PageRows {
   int b = -1, base = 0;
   int64_t r0 = -1, r1 = -1;
-  __device__ void load(const TcParams &p) {
+  __device__ __forceinline__ void load(const TcParams &p) {
     const int lane = threadIdx.x & 31;
     r0 = tile_row(p, b, base + lane);
     r1 = tile_row(p, b, base + 32 + lane);
   }
-  __device__ int64_t get(const TcParams &p, int seq, int page) {
+  __device__ __forceinline__ int64_t get(const TcParams &p, int seq, int page) {
     if (seq != b || page < base || page >= base + 96) {
       b = seq;
       base = page;
@@ -341,7 +353,7 @@ struct PageRows {
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_pe,
-                     const TcParams p) {
+                     const __grid_constant__ TcParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *tiles = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   SmemB &sb = *reinterpret_cast<SmemB *>(tiles + kRegionA);
@@ -586,8 +598,10 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             break;
           }
           const bool tail = p.kv_begin + (t + 1) * kTileKeys > S;
-          const bool resc = t != t0 && (__float_as_uint(sb.pa[pb][0][32]) | __float_as_uint(sb.pa[pb][1][32]) |
-                                        __float_as_uint(sb.pa[pb][2][32]) | __float_as_uint(sb.pa[pb][3][32])) != 0;
+          const uint32_t fa = slot_factors(smem_u32(tiles), pb);
+          const bool resc = t != t0 && (ld_shared_u32(fa + 4 * 32) | ld_shared_u32(fa + 4 * (kPaWords + 32)) |
+                                        ld_shared_u32(fa + 4 * (2 * kPaWords + 32)) |
+                                        ld_shared_u32(fa + 4 * (3 * kPaWords + 32))) != 0;
           bool have_v = false;
           if (tail || resc) {
             // Rare: let the epilogue warps zero the rows past the end and/or rescale O first.
@@ -602,7 +616,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             if (!wait_or_abort(sb, bar(B_REQDONE), nfix & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
             ++nfix;
           }
-          const uint32_t pt = smem_u32(tiles + kPOff + pb * kPBytes);
+          const uint32_t pt = smem_u32(tiles + kPOff + pb * kPSlotBytes);
           // O[:, 256h .. 256h+255] += P . C[:, 256h ..]: one half-page stage per group of 4 MMAs.
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -664,10 +678,9 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       SegIter it = it0;
       uint32_t ns = 0, np = 0, uc = 0;
       const uint32_t pbuf_remote = mapa(smem_u32(tiles + kPOff), peer);
-      const uint32_t pa_remote = mapa(smem_u32(&sb.pa[0][0][0]), peer);
       // Staging of this half's P page (all four lane quadrants) and of its rescale factors.
-      unsigned char *stgp = tiles + kStgOff + h * kPBytes;
-      unsigned char *stga = tiles + kStgOff + 2 * kPBytes + h * (kPWriters * kPaWords * 4);
+      unsigned char *stgp = tiles + kStgOff + h * kPSlotBytes;
+      unsigned char *stga = stgp + kPBytes;
       const uint32_t statl_remote = mapa(smem_u32(&sb.stat_l[0]), peer);
       const uint32_t statm_remote = mapa(smem_u32(&sb.stat_m[0]), peer);
       const uint32_t pfull_remote = mapa(bar(B_PFULL), peer);
@@ -707,7 +720,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         }
         const int S = seq_len_clamped(p, b);
         const int j = real ? gr / p.H : 0;
-        const int visible = real ? S - p.n_q + j + 1 : 0;
+        // Keys this row may see, counted from the key range's first key.
+        const int vis_end = (real ? min(S - p.n_q + j + 1, p.kv_end) : 0) - p.kv_begin;
         float m_ref = -CUDART_INF_F, l = 0.f;
         for (int T = t0; T < t1; T += kSuper, ++ns) {
           if (lane == 0) sb.prog[warp] = (int)np;
@@ -733,7 +747,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
           // Valid while below the row's causal limit and inside the pages this tile holds.
-          const int nvalid = min(min(visible, p.kv_end) - (p.kv_begin + (T + h) * kTileKeys), (npg - h) * kTileKeys);
+          const int nvalid = min(vis_end - (T + h) * kTileKeys, (npg - h) * kTileKeys);
           float mx = -CUDART_INF_F;
 #pragma unroll
           for (int k = 0; k < 64; ++k)
@@ -785,9 +799,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             if (issuer && (pn < kPSlots || wait_or_abort(sb, bar(B_PEMPTY + pb), ((pn / kPSlots) - 1) & 1, p.dev_status,
                                                          true, p.timeout_rec, __LINE__))) {
               const uint32_t pfull = pfull_remote + 8 * pb;
-              bulk_copy_to_peer(pbuf_remote + pb * kPBytes, smem_u32(stgp), kPBytes, pfull);
-              bulk_copy_to_peer(pa_remote + pb * (kPWriters * kPaWords * 4), smem_u32(stga), kPWriters * kPaWords * 4,
-                                pfull);
+              bulk_copy_to_peer(pbuf_remote + pb * kPSlotBytes, smem_u32(stgp), kPTxBytes, pfull);
               bulk_commit();
             }
           }
@@ -835,7 +847,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             }
             if (q.rescale) {
               tc_fence_after();
-              const float a = sb.pa[q.slot][r >> 5][r & 31];
+              const float a = __uint_as_float(ld_shared_u32(slot_factors(smem_u32(tiles), q.slot) +
+                                                            4 * ((r >> 5) * kPaWords + (r & 31))));
 #pragma unroll 1
               for (int c = 0; c < 16; ++c) {
                 uint32_t v[32];
