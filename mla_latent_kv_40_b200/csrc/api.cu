@@ -599,7 +599,10 @@ int mla_prefill_workspace_size(const mla_dims *dims, int B, int total_tokens, in
     return MLA_ERR_INVALID_ARG;
   const size_t dqk = (size_t)dims->d_nope + dims->d_rope;
   const size_t rows = (size_t)total_tokens * dims->n_heads;
-  *bytes = 2 * align256(rows * dqk * elem(dims)) + align256(rows * dims->d_v * elem(dims));
+  const size_t row_layout = 2 * align256(rows * dqk * elem(dims)) + align256(rows * dims->d_v * elem(dims));
+  // The tensor-core path keeps its Q/K/V in per-(head, sequence) tiles padded to max_seqlen.
+  const size_t tiled = dims->dtype == MLA_BF16 ? prefill_tiled_bytes(B, dims->n_heads, max_seqlen) : 0;
+  *bytes = row_layout > tiled ? row_layout : tiled;
   return MLA_OK;
 }
 
@@ -628,7 +631,8 @@ int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, int max_
                 cu_seqlens, q_nope, q_pe, w_uk, w_uv,
                 CacheView{c_kv, k_pe, dims->ckv_stride, dims->kpe_stride, block_table, max_blocks_per_seq,
                           num_blocks, dims->block_size, dims->cache_layout, dims->d_c, dims->d_c + dims->d_rope},
-                qbuf, kbuf, vbuf, out, lse, default_scale(*dims), dims->rope_base, dev_status};
+                qbuf, kbuf, vbuf, out, lse, default_scale(*dims), dims->rope_base, dev_status, 0, 0, 0,
+                static_cast<unsigned char *>(workspace), nullptr};
   return launch_prefill_simt(a, dims->dtype == MLA_BF16, reinterpret_cast<cudaStream_t>(stream));
 }
 

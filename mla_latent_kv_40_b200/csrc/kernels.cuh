@@ -96,7 +96,27 @@ struct PrefillArgs {
   float *lse;
   float scale, rope_base;
   int *dev_status;
+  // Tiled workspace of the tensor-core prefill (set by the launcher): per head s and sequence b,
+  // Q in tiles of 128 query rows [3 chunks][128 rows x 128 B] (48 KB) at q_tiles, and K with V in
+  // tiles of 64 tokens [3 K chunks | 2 V chunks][64 rows x 128 B] (40 KB) at kv_tiles; chunks
+  // 128-byte swizzled like the tiled latent pool, so each tile moves as one bulk copy.
+  int tiled, nqt, nkt;        // tiles per (head, sequence): nqt = ceil(max_seqlen / 128), nkt = 2 nqt
+  unsigned char *q_tiles, *kv_tiles;
 };
+
+// Byte offset of element (row, dim) inside a tile of `rows` rows and 64-dim chunks.
+__host__ __device__ __forceinline__ int64_t swz_tile_offset(int rows, int row, int dim) {
+  const int c = dim >> 6, g = (dim >> 3) & 7, e = dim & 7;
+  return (int64_t)c * rows * 128 + row * 128 + ((g ^ (row & 7)) << 4) + e * 2;
+}
+constexpr int64_t kPfQTileBytes = 128 * 192 * 2;     // 49152
+constexpr int64_t kPfKVTileBytes = 64 * (192 + 128) * 2;   // 40960
+// Workspace bytes of the tiled prefill layout.
+inline size_t prefill_tiled_bytes(int B, int H, int max_seqlen) {
+  const size_t nqt = (size_t)(max_seqlen + 127) / 128;
+  const size_t q = (size_t)H * B * nqt * kPfQTileBytes;
+  return ((q + 255) & ~size_t(255)) + (size_t)H * B * 2 * nqt * kPfKVTileBytes;
+}
 
 int launch_append(const AppendArgs &a, bool bf16, cudaStream_t st);
 int launch_absorb(const AbsorbArgs &a, bool bf16, cudaStream_t st);

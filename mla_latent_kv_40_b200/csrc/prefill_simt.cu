@@ -22,7 +22,7 @@ constexpr int kPfThreads = 256;
 template <typename T>
 __global__ void __launch_bounds__(kPfThreads) prefill_q_kernel(PrefillArgs a) {
   extern __shared__ float rot[];          // [d_rope / 2][2]: cos, sin
-  __shared__ int pos;
+  __shared__ int pos_s, seq_s;
   const int t = blockIdx.x;
   if (threadIdx.x == 0) {                 // position of row t within its sequence
     int lo = 0, hi = a.B;                 // find b with cu[b] <= t < cu[b+1]
@@ -30,9 +30,11 @@ __global__ void __launch_bounds__(kPfThreads) prefill_q_kernel(PrefillArgs a) {
       const int mid = (lo + hi) >> 1;
       if (a.cu_seqlens[mid] <= t) lo = mid; else hi = mid;
     }
-    pos = t - a.cu_seqlens[lo];
+    pos_s = t - a.cu_seqlens[lo];
+    seq_s = lo;
   }
   __syncthreads();
+  const int pos = pos_s, seq = seq_s;
   for (int i = threadIdx.x; i < (a.d_rope >> 1); i += blockDim.x)
     rope_cos_sin(pos, i, a.d_rope, a.rope_base, &rot[2 * i], &rot[2 * i + 1]);
   __syncthreads();
@@ -40,16 +42,23 @@ __global__ void __launch_bounds__(kPfThreads) prefill_q_kernel(PrefillArgs a) {
   const T *qn = static_cast<const T *>(a.q_nope) + (int64_t)t * a.H * a.d_nope;
   const T *qp = static_cast<const T *>(a.q_pe) + (int64_t)t * a.H * a.d_rope;
   T *qb = static_cast<T *>(a.qbuf) + (int64_t)t * a.H * dqk;
+  // Tiled workspace: row pos % 128 of tile pos / 128 of (head s, sequence seq).
   for (int e = threadIdx.x; e < a.H * dqk; e += blockDim.x) {
     const int s = e / dqk, d = e % dqk;
+    T v;
     if (d < a.d_nope) {
-      qb[e] = qn[s * a.d_nope + d];
+      v = qn[s * a.d_nope + d];
     } else {
       const int dr = d - a.d_nope, i = dr >> 1;
       const float x = to_f32(qp[s * a.d_rope + 2 * i]), y = to_f32(qp[s * a.d_rope + 2 * i + 1]);
       const float c = rot[2 * i], sn = rot[2 * i + 1];
-      qb[e] = from_f32<T>((dr & 1) ? (x * sn + y * c) : (x * c - y * sn));
+      v = from_f32<T>((dr & 1) ? (x * sn + y * c) : (x * c - y * sn));
     }
+    if (a.tiled)
+      *reinterpret_cast<T *>(a.q_tiles + (((int64_t)s * a.B + seq) * a.nqt + pos / 128) * kPfQTileBytes +
+                             swz_tile_offset(128, pos % 128, d)) = v;
+    else
+      qb[e] = v;
   }
 }
 
@@ -236,8 +245,16 @@ prefill_attn_kernel(PrefillArgs a) {
 }
 
 template <typename T>
-static int launch_prefill_t(const PrefillArgs &a, cudaStream_t st) {
+static int launch_prefill_t(PrefillArgs a, cudaStream_t st) {
   const int dqk = a.d_nope + a.d_rope;
+  // Both tensor-core steps available: Q, K and V go to the tiled workspace (one bulk copy per tile).
+  if (sizeof(T) == 2 && decompress_tc_supported(a, true) && prefill_tc_supported(a, true)) {
+    a.tiled = 1;
+    a.nqt = (a.max_seqlen + 127) / 128;
+    a.nkt = 2 * a.nqt;
+    const size_t qbytes = (size_t)a.H * a.B * a.nqt * kPfQTileBytes;
+    a.kv_tiles = a.q_tiles + ((qbytes + 255) & ~size_t(255));
+  }
   prefill_q_kernel<T><<<a.total, kPfThreads, sizeof(float) * a.d_rope, st>>>(a);
   const size_t smem_dec = sizeof(float) * kDecRows * a.d_c;
   if (cudaFuncSetAttribute(prefill_decompress_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dec))

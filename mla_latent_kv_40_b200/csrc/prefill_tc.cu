@@ -63,6 +63,8 @@ static_assert(kPfSmem <= 232448, "prefill shared memory budget");
 
 struct PfParams {
   int B, H, max_seqlen, total;
+  int tiled, nqt, nkt;          // tiled workspace: Q and K|V tiles per (head, sequence), one bulk copy each
+  const unsigned char *q_tiles, *kv_tiles;
   const int32_t *cu_seqlens;
   float scale_log2;
   __nv_bfloat16 *out;           // [total, H, 128]
@@ -130,22 +132,32 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
   if (warp == 0 && lane == 0) {
     // ---- producer: Q once, then one stage (K and V of 64 tokens) per key tile
     grid_dep_wait();
-    tma_prefetch_desc(&mq);
-    tma_prefetch_desc(&mk);
-    tma_prefetch_desc(&mv);
+    if (!p.tiled) {
+      tma_prefetch_desc(&mq);
+      tma_prefetch_desc(&mk);
+      tma_prefetch_desc(&mv);
+    }
     mbar_expect_tx(bar(P_QFULL), kQBytes);
-    for (int c = 0; c < 3; ++c)
-      tma_load_2d(smem_u32(tiles + c * (kPq * 128)), &mq, s * kDqk + 64 * c, start + q0, bar(P_QFULL));
+    const int64_t hs = (int64_t)s * p.B + b;   // (head, sequence) of the tiled workspace
+    if (p.tiled)
+      bulk_load(smem_u32(tiles), p.q_tiles + (hs * p.nqt + qt) * kPfQTileBytes, kQBytes, bar(P_QFULL));
+    else
+      for (int c = 0; c < 3; ++c)
+        tma_load_2d(smem_u32(tiles + c * (kPq * 128)), &mq, s * kDqk + 64 * c, start + q0, bar(P_QFULL));
     int kt = 0;
     for (; kt < nk; ++kt) {
       const int st = kt % kPStages;
       if (kt >= kPStages && !pwait(sb, bar(P_KVEMPTY + st), ((kt / kPStages) - 1) & 1, p.dev_status)) break;
       unsigned char *stg = tiles + kOffStages + st * kStageBytes;
       mbar_expect_tx(bar(P_KVFULL + st), kStageBytes);
-      for (int c = 0; c < 3; ++c)
-        tma_load_2d(smem_u32(stg + c * kKChunk), &mk, s * kDqk + 64 * c, start + kPk * kt, bar(P_KVFULL + st));
-      for (int c = 0; c < 2; ++c)
-        tma_load_2d(smem_u32(stg + (3 + c) * kKChunk), &mv, s * kDvp + 64 * c, start + kPk * kt, bar(P_KVFULL + st));
+      if (p.tiled) {   // K (3 chunks) and V (2 chunks) of 64 tokens: one 40 KB copy
+        bulk_load(smem_u32(stg), p.kv_tiles + (hs * p.nkt + kt) * kPfKVTileBytes, kStageBytes, bar(P_KVFULL + st));
+      } else {
+        for (int c = 0; c < 3; ++c)
+          tma_load_2d(smem_u32(stg + c * kKChunk), &mk, s * kDqk + 64 * c, start + kPk * kt, bar(P_KVFULL + st));
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(smem_u32(stg + (3 + c) * kKChunk), &mv, s * kDvp + 64 * c, start + kPk * kt, bar(P_KVFULL + st));
+      }
     }
     // Every issued load lands before the CTA may leave.
     for (int j = max(0, kt - kPStages); j < kt; ++j) pwait(sb, bar(P_KVFULL + j % kPStages), (j / kPStages) & 1, p.dev_status);
@@ -310,6 +322,8 @@ constexpr size_t kDcSmem = 1024 + kDcStages * kDcStage + 64;
 
 struct DcParams {
   int H, d_c, block_size, max_blocks_per_seq, num_blocks, total;
+  int tiled, B, nkt;            // tiled workspace: write K|V tiles per (head, sequence, 64-token page)
+  unsigned char *kv_tiles;
   const int32_t *cu_seqlens, *block_table;
   const __nv_bfloat16 *k_pe;
   int64_t kpe_stride;
@@ -410,16 +424,32 @@ decompress_tc_kernel(const __grid_constant__ CUtensorMap mc, const __grid_consta
   if (ok2) mbar_wait(smem_u32(&done), 0, kWait);
   tc_fence_after();
   grid_dep_wait();
-  // Thread = token p0 + 32w + lane (its tensor-memory lane): 256 outputs -> kbuf / vbuf rows.
+  // Thread = token p0 + 32w + lane (its tensor-memory lane): 256 outputs -> kbuf / vbuf rows, or
+  // its row of the K|V tile of its 64-token page (rows past the sequence end are zeroed there, so
+  // the attention's masked products meet finite values).
   const int tok = 32 * warp + lane, pos = p0 + tok;
   const bool real = ok2 && pos < L && page_row[tok >> 6] >= 0;
   const int64_t t = start + pos;
+  unsigned char *tile = p.tiled ? p.kv_tiles + (((int64_t)s * p.B + b) * p.nkt + pos / 64) * kPfKVTileBytes : nullptr;
+  const int prow = pos & 63;
 #pragma unroll 1
   for (int c = 0; c < 8; ++c) {
     uint32_t v[32];
     tmem_ld32(tbase + ((uint32_t)(32 * warp) << 16) + 32 * c, v);
     tmem_wait_ld();
-    if (real) {
+    if (p.tiled) {
+      // columns 32c .. 32c+31: K dims 32c.. (c < 4) or V dims 32(c-4).. (V follows the 3 K chunks)
+      unsigned char *base = c < 4 ? tile : tile + 3 * kKChunk;
+      const int d0 = c < 4 ? 32 * c : 32 * (c - 4);
+#pragma unroll
+      for (int i = 0; i < 32; i += 8)
+        *reinterpret_cast<uint4 *>(base + swz_tile_offset(64, prow, d0 + i)) =
+            real ? make_uint4(pack_bf16x2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                              pack_bf16x2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3])),
+                              pack_bf16x2(__uint_as_float(v[i + 4]), __uint_as_float(v[i + 5])),
+                              pack_bf16x2(__uint_as_float(v[i + 6]), __uint_as_float(v[i + 7])))
+                 : make_uint4(0, 0, 0, 0);
+    } else if (real) {
       __nv_bfloat16 *dst = c < 4 ? p.kbuf + (t * p.H + s) * kDqk + 32 * c : p.vbuf + (t * p.H + s) * kDvp + 32 * (c - 4);
 #pragma unroll
       for (int i = 0; i < 32; i += 8)
@@ -430,9 +460,14 @@ decompress_tc_kernel(const __grid_constant__ CUtensorMap mc, const __grid_consta
                        pack_bf16x2(__uint_as_float(v[i + 6]), __uint_as_float(v[i + 7])));
     }
   }
-  if (real) {   // the shared RoPE key, already rotated in the cache
-    const int64_t row = (int64_t)page_row[tok >> 6] + (tok & 63);
-    const uint4 *src = reinterpret_cast<const uint4 *>(p.k_pe + row * p.kpe_stride);
+  // the shared RoPE key, already rotated in the cache (zeros past the end in the tiled layout)
+  const int64_t row = real ? (int64_t)page_row[tok >> 6] + (tok & 63) : 0;
+  const uint4 *src = reinterpret_cast<const uint4 *>(p.k_pe + row * p.kpe_stride);
+  if (p.tiled) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint4 *>(tile + swz_tile_offset(64, prow, 128 + 8 * i)) = real ? src[i] : make_uint4(0, 0, 0, 0);
+  } else if (real) {
     uint4 *dst = reinterpret_cast<uint4 *>(p.kbuf + (t * p.H + s) * kDqk + 128);
 #pragma unroll
     for (int i = 0; i < 8; ++i) dst[i] = src[i];
@@ -486,6 +521,10 @@ int launch_decompress_tc(const PrefillArgs &a, cudaStream_t st) {
   p.kbuf = static_cast<__nv_bfloat16 *>(a.kbuf);
   p.vbuf = static_cast<__nv_bfloat16 *>(a.vbuf);
   p.dev_status = a.dev_status;
+  p.tiled = a.tiled;
+  p.B = a.B;
+  p.nkt = a.nkt;
+  p.kv_tiles = a.kv_tiles;
   const dim3 grid((a.max_seqlen + kDcTok - 1) / kDcTok, a.H, a.B);
   return launch_pdl(decompress_tc_kernel, grid, dim3(128), kDcSmem, st, mc, mwk, mwv, p) == cudaSuccess ? MLA_OK
                                                                                                     : MLA_ERR_CUDA;
@@ -503,6 +542,11 @@ int launch_prefill_tc_attention(const PrefillArgs &a, cudaStream_t st) {
   PfParams p;
   p.B = a.B;
   p.H = a.H;
+  p.tiled = a.tiled;
+  p.nqt = a.nqt;
+  p.nkt = a.nkt;
+  p.q_tiles = a.q_tiles;
+  p.kv_tiles = a.kv_tiles;
   p.max_seqlen = a.max_seqlen;
   p.total = a.total;
   p.cu_seqlens = a.cu_seqlens;
