@@ -52,18 +52,22 @@ def test_kv_shard_ranges_cover_the_keys(max_seqlen, world):
     assert covered == max_seqlen
 
 
-def _partials(inp, ranges, latent=True):
+def _partials(inp, ranges, heads=None):
     """The oracle's partial of each key range: the decode over that range's visible keys, with
     W_UV = I (the latent), as (o [N, B, n_q, H, d_c], lse [N, B, n_q, H]); empty ranges give
-    (0, -inf)."""
+    (0, -inf).  With `heads`, only those heads are computed (the others stay NaN)."""
     d = inp["dims"]
     B, n_q, H = inp["q_nope"].shape[:3]
     sl = inp["seqlens"].numpy()
     eye = np.broadcast_to(np.eye(d.d_c), (H, d.d_c, d.d_c))
     import dataclasses
     dl = dataclasses.replace(d, d_v=d.d_c)
+    heads = list(range(H)) if heads is None else list(heads)
     o = np.zeros((len(ranges), B, n_q, H, d.d_c))
     lse = np.full((len(ranges), B, n_q, H), -np.inf)
+    skip = [x for x in range(H) if x not in heads]
+    o[:, :, :, skip] = np.nan
+    lse[:, :, :, skip] = np.nan
     for r, (k0, k1) in enumerate(ranges):
         for b in range(B):
             for j in range(n_q):
@@ -73,11 +77,11 @@ def _partials(inp, ranges, latent=True):
                     continue
                 sel = np.full((B, n_q, len(toks)), -1)
                 sel[b, j] = toks
-                picks = [(b, j, s) for s in range(H)]
+                picks = [(b, j, s) for s in heads]
                 ob, lb = oracle.decode_sparse(dl, inp["q_nope"], inp["q_pe"], inp["pool"], inp["block_table"],
                                               inp["block_size"], inp["seqlens"], sel, inp["w_uk"], eye, picks=picks)
-                o[r, b, j] = ob[b, j]
-                lse[r, b, j] = lb[b, j]
+                o[r, b, j, heads] = ob[b, j, heads]
+                lse[r, b, j, heads] = lb[b, j, heads]
     return o, lse
 
 
