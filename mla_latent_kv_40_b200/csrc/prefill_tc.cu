@@ -49,7 +49,8 @@ constexpr float kRescale = 8.f;
 constexpr uint64_t kWait = 2000000000ull;
 
 enum PBar { P_QFULL = 0, P_KVFULL = 1, P_KVEMPTY = P_KVFULL + kPStages, P_SFULL = P_KVEMPTY + kPStages,
-            P_SEMPTY = P_SFULL + 2, P_PFULL = P_SEMPTY + 2, P_PVDONE = P_PFULL + 2, P_COUNT = P_PVDONE + 1 };
+            P_SEMPTY = P_SFULL + 2, P_PFULL = P_SEMPTY + 2, P_PVDONE = P_PFULL + 2, P_COUNT = P_PVDONE + 2 };
+// P_PVDONE + b completes when the product O += P V that read P buffer b has completed.
 
 struct PfSmem {
   uint64_t bars[P_COUNT];
@@ -195,7 +196,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
           mma_ss(tbase + kOCols, smem_desc_sw128(pa + kk * 32, 16, 1024), smem_desc_sw128(vb + kk * 2048, kKChunk, 1024),
                  idO, (j | kk) ? 1u : 0u);
         tc_commit(bar(P_KVEMPTY + st));
-        tc_commit(bar(P_PVDONE));
+        tc_commit(bar(P_PVDONE + pb));
       }
     }
   } else if (warp >= 4) {
@@ -242,12 +243,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
         psum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
       }
       l += psum;
-      // O and the P tile are free once the previous tile's O += P V has completed.
-      if (kt >= 1) {
-        pwarp_wait(sb, bar(P_PVDONE), (kt - 1) & 1, p.dev_status);
+      // P buffer kt & 1 is free once its last reader, the product of tile kt - 2, has completed; the
+      // products of the previous tile may still run.  Only when a row's reference moved must O
+      // hold every earlier product (tile kt - 1) before it is rescaled.
+      if (kt >= 2) pwarp_wait(sb, bar(P_PVDONE + (kt & 1)), ((kt - 2) >> 1) & 1, p.dev_status);
+      if (kt >= 1 && __any_sync(0xffffffffu, need)) {
+        pwarp_wait(sb, bar(P_PVDONE + ((kt - 1) & 1)), ((kt - 1) >> 1) & 1, p.dev_status);
         tc_fence_after();
-        // Rescale my rows' O columns when the reference moved (never before the first product).
-        if (__any_sync(0xffffffffu, need)) {
+        {
 #pragma unroll 1
           for (int c = 0; c < 2; ++c) {
             uint32_t v[32];
@@ -275,7 +278,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant_
     sb.xl[h][r] = l;
     asm volatile("bar.sync 1, 256;" ::: "memory");
     l += sb.xl[h ^ 1][r];
-    pwarp_wait(sb, bar(P_PVDONE), (nk - 1) & 1, p.dev_status);
+    pwarp_wait(sb, bar(P_PVDONE + ((nk - 1) & 1)), ((nk - 1) >> 1) & 1, p.dev_status);
     tc_fence_after();
     grid_dep_wait();   // the outputs may still be read by an earlier kernel
     const float inv = l > 0.f ? 1.f / l : 0.f;
