@@ -22,6 +22,13 @@
 //     normalises and writes the unit's partial output.
 // The score CTA does 53% of the MMA work and the value CTA 47%.
 //
+// One thread issues a tcgen05.mma about every 128 cycles, whatever N is: enough
+// to keep the tensor pipe busy at N = 256, a quarter of its rate at N = 64.  So
+// each CTA issues from two threads on different SM sub-partitions, each with its
+// own accumulator: in the score CTA one thread per page of a score tile (N = 64
+// each), in the value CTA one thread per 256-column half of O (N = 256), served
+// by its own group of four epilogue warps.
+//
 // Online softmax uses a lazy reference maximum (kept in log2 units): P is
 // exp2(s - m_ref) and m_ref only moves when a tile's maximum exceeds it by more
 // than 8, so the O accumulator is rescaled (tcgen05.ld / st by the value CTA)
@@ -54,6 +61,7 @@ constexpr int kSuper = 2;                          // page tiles per score tile:
 constexpr int kDc = 512, kDr = 64, kW = kDc + kDr;
 constexpr int kRows = 128;                         // M of every MMA: query rows per unit
 constexpr int kKStages = 4;                        // score CTA: half-page stages in flight (two pages)
+static_assert(kKStages == 2 * 2, "one stage pair per page position of a score tile");
 constexpr int kVStages = 4;                        // value CTA: [64 keys x 256 dims] half-page stages in flight
 constexpr int kThreads = 384;
 constexpr int kLaunchRegs = 168;                   // per thread (65536 / 384, rounded down to 8)
@@ -81,14 +89,10 @@ constexpr uint32_t kStgOff = kKOff + kKStages * kKStageBytes;      // score CTA:
 constexpr uint32_t kScoreEnd = kStgOff + 2 * kPSlotBytes, kValueEnd = kPOff + kPSlots * kPSlotBytes;
 constexpr uint32_t kRegionA = ((kScoreEnd > kValueEnd ? kScoreEnd : kValueEnd) + 1023) & ~1023u;   // 214016
 static_assert(kPOff + kPSlots * kPSlotBytes <= kRegionA, "value-CTA tiles must fit the shared region");
-#ifndef MLA_TC_PREFETCH_PAGES
-#define MLA_TC_PREFETCH_PAGES 0
-#endif
-constexpr int kPrefetchPages = MLA_TC_PREFETCH_PAGES;  // score CTA: pages prefetched into L2 ahead of the smem stream
 constexpr float kRescaleLog2 = 8.f;
 constexpr uint64_t kWaitNs = 2000000000ull;        // 2 s per wait
 constexpr int kMaxClusters = 128;
-constexpr int kTimeoutRecInts = 1 + 6 * 16;
+constexpr int kTimeoutRecInts = 1 + 6 * 2 * (kThreads / 32);
 
 // TMEM columns
 constexpr uint32_t kQCol = 0;      // score CTA: latent part of Q, 256 columns (2 bf16 per column)
@@ -100,14 +104,14 @@ enum Bar {
   B_KFULL = 0, B_KEMPTY = B_KFULL + kKStages, B_SFULL = B_KEMPTY + kKStages, B_SEMPTY = B_SFULL + 2,
   B_QREADY = B_SEMPTY + 2, B_PEMPTY = B_QREADY + 1, B_STATSEMPTY = B_PEMPTY + kPSlots,
   B_VFULL = B_STATSEMPTY + 1, B_VEMPTY = B_VFULL + kVStages, B_PFULL = B_VEMPTY + kVStages,
-  B_PVDONE = B_PFULL + kPSlots, B_REQ = B_PVDONE + kPSlots, B_REQDONE = B_REQ + 1, B_STATSFULL = B_REQDONE + 1,
+  B_PVDONE = B_PFULL + kPSlots, B_REQ = B_PVDONE + kPSlots, B_REQDONE = B_REQ + 2, B_STATSFULL = B_REQDONE + 2,
   B_OFREE = B_STATSFULL + 1, B_COUNT = B_OFREE + 1
 };
 
 // A request from the value CTA's MMA thread to its epilogue warps.
 struct Req {
   int kind;        // 0: fix up a tile before its MMA, 1: unit epilogue
-  int vstage0, vstage1, slot, nvalid, tail, rescale, segid, last_slot, last_parity;
+  int vstage, slot, nvalid, tail, rescale, segid, last_slot, last_parity;
 };
 
 struct SmemB {                       // small region after the tiles
@@ -115,12 +119,12 @@ struct SmemB {                       // small region after the tiles
   float xmax[2][2][kRows];           // score CTA: the two softmax halves' tile maxima (double-buffered)
   float xl[2][kRows];                // score CTA: the two halves' row sums at the end of a unit
   uint64_t bars[B_COUNT];
-  Req req;
+  Req req[2];                        // value CTA: one request channel per O half (issuer -> epilogue group)
   uint32_t tmem_base;
   int abort;
   int plan_u0, plan_p0, plan_s0;     // first unit of this cluster, its tile prefix and segment prefix
   int plan_C;                        // clusters that get work: min(launched clusters, total tiles)
-  int prog[8];                       // per-warp progress (tiles handled), kept for timeout records
+  int prog[kThreads / 32];           // per-warp progress (tiles handled), kept for timeout records
   long long plan_start, plan_end, plan_total;
 };
 constexpr size_t kSmemBytes = 1024 + kRegionA + sizeof(SmemB);
@@ -279,7 +283,7 @@ struct SegIter {
 };
 
 // Bounded wait that turns a timeout into the CTA-wide abort state.  The first
-// timeout of each (CTA rank, warp) in the grid is recorded in rec[1 + 6 * (8 * rank + warp) ..]:
+// timeout of each (CTA rank, warp) in the grid is recorded in rec[1 + 6 * (12 * rank + warp) ..]:
 // cluster, barrier slot, parity, source line, the warp's progress counter.
 __device__ __forceinline__ bool wait_or_abort(SmemB &sb, uint32_t bar, uint32_t parity, int *dev_status,
                                               bool cluster_scope = false, int *rec = nullptr, int tag = 0) {
@@ -289,7 +293,7 @@ __device__ __forceinline__ bool wait_or_abort(SmemB &sb, uint32_t bar, uint32_t 
   report(dev_status, MLA_ERR_TIMEOUT);
   if (rec) {
     const int w = (int)(threadIdx.x >> 5);
-    int *e = rec + 1 + 6 * (8 * (int)cluster_ctarank() + w);
+    int *e = rec + 1 + 6 * ((kThreads / 32) * (int)cluster_ctarank() + w);
     if (atomicCAS(e, 0, 1) == 0) {
       e[1] = (int)cluster_id_x();
       e[2] = (int)((bar - smem_u32(&sb.bars[0])) / 8);
@@ -374,11 +378,13 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
     for (int i = 0; i < B_COUNT; ++i) counts[i] = 1;
     counts[B_SEMPTY] = counts[B_SEMPTY + 1] = 8;      // one per softmax warp
     counts[B_QREADY] = 8;
-    counts[B_STATSEMPTY] = 4;                         // remote, one per value-CTA epilogue warp
+    counts[B_SFULL] = counts[B_SFULL + 1] = 2;      // one commit per score-MMA issuer
+    counts[B_STATSEMPTY] = 8;                         // remote, one per value-CTA epilogue warp
+    for (int i = 0; i < kPSlots; ++i) counts[B_PVDONE + i] = 2;   // one commit per value-MMA issuer
     // P full: the relay's arrival, which also arms the bytes the four writer warps' bulk copies bring.
-    counts[B_REQDONE] = kRows;
+    counts[B_REQDONE] = counts[B_REQDONE + 1] = kRows;   // the four warps of one epilogue group
     counts[B_STATSFULL] = kRows;                      // remote, every softmax thread
-    counts[B_OFREE] = kRows;
+    counts[B_OFREE] = 2 * kRows;                      // both epilogue groups
     for (int i = 0; i < B_COUNT; ++i) mbar_init(bar(i), counts[i]);
     if (rank == 1)
       for (int i = 0; i < kPSlots; ++i) mbar_expect_tx(bar(B_PFULL + i), kPTxBytes);
@@ -419,13 +425,13 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       if (warp == 0) {
       // ---- key producer (whole warp: page lookups in warp-wide batches; lane 0 issues): a score
       // tile is up to 2 pages (128 keys); each page is streamed as two stages, one bulk copy each
-      // (chunks 0-3, then chunks 4-8).  Optionally, pages further ahead are prefetched into L2.
+      // (chunks 0-3, then chunks 4-8).  Page pg of a tile always goes to stages 2 pg and 2 pg + 1,
+      // which only its MMA issuer reads, so each stage's uses are consumed in order.
       grid_dep_wait();
       SegIter it = it0;
       PageRows pr;
-      uint32_t n = 0;
+      uint32_t u[kKStages] = {};   // loads issued so far into each stage
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        int pf = t0 + kSuper;   // next page to prefetch
         for (int T = t0; T < t1; T += kSuper) {
           const int npg = min(kSuper, t1 - T);
           int32_t rows[kSuper];
@@ -438,22 +444,15 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             }
             rows[pg] = (int32_t)row;
           }
-          const int pf_end = kPrefetchPages > 0 ? min(t1, T + kSuper + kPrefetchPages) : pf;
-          for (; pf < pf_end; ++pf) {
-            const int64_t prow = pr.get(p, b, pf);
-            if (prow < 0 || lane != 0) continue;
-            if (p.tiled) prefetch_l2(p.tiled + (prow / kTileKeys) * (9 * kChunkBytes), 9 * kChunkBytes);
-            else if (p.rows_contig) prefetch_l2(p.row_pool + prow * (int64_t)kW * 2, kTileKeys * kW * 2);
-          }
           // Lane 0 streams the tile's pages, two stages per page: chunks 0-3, then chunks 4-8.
           int ok = 1;
           if (lane == 0) {
             for (int pg = 0; pg < npg && ok; ++pg) {
-              for (int half = 0; half < 2; ++half, ++n) {
-                sb.prog[warp] = (int)n;
-                const int s = n % kKStages;
-                if (n >= kKStages &&
-                    !wait_or_abort(sb, bar(B_KEMPTY + s), ((n / kKStages) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) {
+              sb.prog[warp] = (int)(u[0] + u[2]);
+              for (int half = 0; half < 2; ++half) {
+                const int s = 2 * pg + half;
+                if (u[s] > 0 &&
+                    !wait_or_abort(sb, bar(B_KEMPTY + s), (u[s] - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) {
                   ok = 0;
                   break;
                 }
@@ -468,11 +467,11 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
                     if (c0 + c < 8) tma_load_2d(dst + c * kChunkBytes, &map_c, 64 * (c0 + c), rows[pg], bar(B_KFULL + s));
                     else tma_load_2d(dst + c * kChunkBytes, &map_pe, 0, rows[pg], bar(B_KFULL + s));
                   }
+                ++u[s];
               }
             }
           }
           ok = __shfl_sync(0xffffffffu, ok, 0);
-          n = __shfl_sync(0xffffffffu, n, 0);
           if (!ok) goto prod_done0;
         }
       }
@@ -480,14 +479,17 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       // Drain: the last load issued on each stage must have landed before exit.
       if (lane == 0)
         for (int s = 0; s < kKStages; ++s)
-          if (const uint32_t uses = n / kKStages + (s < (int)(n % kKStages) ? 1u : 0u))
-            mbar_wait(bar(B_KFULL + s), (uses - 1) & 1, kWaitNs);
-      } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: S [128 x 64 per page] = Q . K^T for the tile's pages side by side, into
+          if (u[s]) mbar_wait(bar(B_KFULL + s), (u[s] - 1) & 1, kWaitNs);
+      } else if ((warp == 1 || warp == 2) && lane == 0) {
+      // ---- MMA issuers: S [128 x 64 per page] = Q . K^T for the tile's pages side by side, into
       // one of two tensor-memory buffers so that the next tile's MMAs overlap this tile's softmax.
       // The latent part of Q is the A operand from tensor memory; the RoPE part is in shared memory.
+      // One thread issues a tcgen05.mma only every ~120 cycles whatever N is, well below the tensor
+      // pipe's rate for N = 64, so each page of a tile has its own issuing thread (page 0: warp 1,
+      // page 1: warp 2, on different SM sub-partitions); both commit the tile's S-full barrier.
+      const int my_pg = warp - 1;
       SegIter it = it0;
-      uint32_t n = 0, ns = 0, uc = 0;
+      uint32_t u = 0, ns = 0, uc = 0;   // u: pages this issuer has consumed (uses of its stage pair)
       bool ok = true;
       while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         if (!wait_or_abort(sb, bar(B_QREADY), uc & 1, p.dev_status, false, p.timeout_rec, __LINE__)) break;
@@ -498,15 +500,16 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           const uint32_t sbuf = ns & 1, dcol = tbase + kSCol + 128 * sbuf;
           if (ns >= 2 && !wait_or_abort(sb, bar(B_SEMPTY + sbuf), ((ns >> 1) - 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
           tc_fence_after();
-          // Page pg of the tile fills S columns 64 pg .. 64 pg + 63 (N = 64 MMAs), one half-page stage at a time.
-          for (int pg = 0; pg < npg && ok; ++pg) {
-            for (int half = 0; half < 2; ++half, ++n) {
-              sb.prog[warp] = (int)n;
-              const int s = n % kKStages;
-              if (!wait_or_abort(sb, bar(B_KFULL + s), (n / kKStages) & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          // This issuer's page of the tile fills S columns 64 pg .. 64 pg + 63 (N = 64 MMAs), one
+          // half-page stage at a time.
+          if (my_pg < npg) {
+            sb.prog[warp] = (int)u;
+            for (int half = 0; half < 2; ++half) {
+              const int s = 2 * my_pg + half;
+              if (!wait_or_abort(sb, bar(B_KFULL + s), u & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
               tc_fence_after();
               const uint32_t kt = smem_u32(tiles + kKOff + s * kKStageBytes);
-              const uint32_t dcol_pg = dcol + 64 * pg;
+              const uint32_t dcol_pg = dcol + 64 * my_pg;
               for (int c = 0; c < half_chunks(half); ++c) {
                 const int j = 4 * half + c;
 #pragma unroll
@@ -520,6 +523,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
               }
               tc_commit(bar(B_KEMPTY + s));
             }
+            ++u;
           }
           if (!ok) break;
           tc_commit(bar(B_SFULL + sbuf));
@@ -579,8 +583,11 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         for (int s = 0; s < kVStages; ++s)
           if (const uint32_t uses = n / kVStages + (s < (int)(n % kVStages) ? 1u : 0u))
             mbar_wait(bar(B_VFULL + s), (uses - 1) & 1, kWaitNs);
-      } else if (warp == 1 && lane == 0) {
-      // ---- MMA issuer: O += P . C
+      } else if ((warp == 1 || warp == 3) && lane == 0) {
+      // ---- MMA issuers: O += P . C.  Issuer hv (warp 1: hv = 0, warp 3: hv = 1) owns O columns
+      // 256 hv .. 256 hv + 255 and reads only the page's latent half hv (stage hv of every stage
+      // pair), so the two issue streams and their fix-up requests run independently.
+      const int hv = warp == 1 ? 0 : 1;
       SegIter it = it0;
       uint32_t n = 0, np = 0, uc = 0, nfix = 0;
       const uint32_t idesc = idesc_bf16_f32(kRows, 256, false, true);
@@ -591,8 +598,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         for (int t = t0; t < t1; ++t, n += 2, ++np) {
           sb.prog[warp] = (int)n;
           const int pb = np % kPSlots;
-          const int sv[2] = {(int)(n % kVStages), (int)((n + 1) % kVStages)};
-          const uint32_t pv[2] = {(n / kVStages) & 1, ((n + 1) / kVStages) & 1};
+          const int sv = (int)((n + hv) % kVStages);
+          const uint32_t pv = ((n + hv) / kVStages) & 1;
           if (!wait_or_abort(sb, bar(B_PFULL + pb), (np / kPSlots) & 1, p.dev_status, true, p.timeout_rec, __LINE__)) {
             ok = false;
             break;
@@ -602,47 +609,39 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           const bool resc = t != t0 && (ld_shared_u32(fa + 4 * 32) | ld_shared_u32(fa + 4 * (kPaWords + 32)) |
                                         ld_shared_u32(fa + 4 * (2 * kPaWords + 32)) |
                                         ld_shared_u32(fa + 4 * (3 * kPaWords + 32))) != 0;
-          bool have_v = false;
+          if (!wait_or_abort(sb, bar(B_VFULL + sv), pv, p.dev_status, false, p.timeout_rec, __LINE__)) {
+            ok = false;
+            break;
+          }
           if (tail || resc) {
-            // Rare: let the epilogue warps zero the rows past the end and/or rescale O first.
-            // A rescale reads O back, so every earlier MMA must have completed.
-            if (!wait_or_abort(sb, bar(B_VFULL + sv[0]), pv[0], p.dev_status, false, p.timeout_rec, __LINE__) ||
-                !wait_or_abort(sb, bar(B_VFULL + sv[1]), pv[1], p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            have_v = true;
+            // Rare: this half's epilogue group zeroes the latent rows past the end and/or rescales
+            // its O columns first.  A rescale reads O back, so the previous page's MMAs (both
+            // halves: the slot's P.V barrier counts both issuers) must have completed.
             if (resc && !wait_or_abort(sb, bar(B_PVDONE + (np - 1) % kPSlots), ((np - 1) / kPSlots) & 1, p.dev_status,
                                        false, p.timeout_rec, __LINE__)) { ok = false; break; }
-            sb.req = Req{0, sv[0], sv[1], pb, S - p.kv_begin - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
-            mbar_arrive(bar(B_REQ));
-            if (!wait_or_abort(sb, bar(B_REQDONE), nfix & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+            sb.req[hv] = Req{0, sv, pb, S - p.kv_begin - t * kTileKeys, tail ? 1 : 0, resc ? 1 : 0, 0, 0, 0};
+            mbar_arrive(bar(B_REQ + hv));
+            if (!wait_or_abort(sb, bar(B_REQDONE + hv), nfix & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
             ++nfix;
           }
+          tc_fence_after();
           const uint32_t pt = smem_u32(tiles + kPOff + pb * kPSlotBytes);
-          // O[:, 256h .. 256h+255] += P . C[:, 256h ..]: one half-page stage per group of 4 MMAs.
+          const uint32_t vt = smem_u32(tiles + sv * kVStageBytes);
+          // O[:, 256 hv ..] += P . C[:, 256 hv ..]: four K = 16 steps over the page's 64 keys.
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (!have_v && !wait_or_abort(sb, bar(B_VFULL + sv[h]), pv[h], p.dev_status, false, p.timeout_rec, __LINE__)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            fence_proxy_async_smem();
-            const uint32_t vt = smem_u32(tiles + sv[h] * kVStageBytes);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = smem_desc_sw128(pt + ks * 32, 16, 1024);
-              const uint64_t bd = smem_desc_sw128(vt + ks * 2048, kChunkBytes, 1024);
-              mma_ss(tbase + 256 * h, ad, bd, idesc, (t != t0 || ks > 0) ? 1u : 0u);
-            }
-            tc_commit(bar(B_VEMPTY + sv[h]));
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = smem_desc_sw128(pt + ks * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(vt + ks * 2048, kChunkBytes, 1024);
+            mma_ss(tbase + 256 * hv, ad, bd, idesc, (t != t0 || ks > 0) ? 1u : 0u);
           }
-          if (!ok) break;
+          tc_commit(bar(B_VEMPTY + sv));
           tc_commit(bar(B_PVDONE + pb));
         }
         if (!ok) break;
-        // Unit epilogue request: the epilogue warps wait for the last MMAs themselves.
+        // Unit epilogue request: the epilogue group waits for the last MMAs itself.
         const uint32_t last = np - 1;
-        sb.req = Req{1, 0, 0, 0, 0, 0, 0, segid, (int)(last % kPSlots), (int)((last / kPSlots) & 1)};
-        mbar_arrive(bar(B_REQ));
+        sb.req[hv] = Req{1, 0, 0, 0, 0, 0, segid, (int)(last % kPSlots), (int)((last / kPSlots) & 1)};
+        mbar_arrive(bar(B_REQ + hv));
         ++uc;
       }
       } else if (warp == 2 && lane == 0) {
@@ -819,10 +818,14 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
         ++uc;
       }
       if (lane == 0) bulk_wait_all();   // the staged copies have landed before this CTA may exit
-    } else if (warp < 8) {
-      // ---- epilogue warps: tile fix-ups on request, then each unit's epilogue
-      const int r = (warp - 4) * 32 + lane;
-      const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    } else {
+      // ---- epilogue warps, two groups of four: group g (warps 4 + 4g .. 7 + 4g) serves the MMA
+      // issuer of O half g (columns 256 g .. 256 g + 255): tile fix-ups on request, then each
+      // unit's epilogue for those columns.  Warp w owns rows (TMEM lanes) 32 (w & 3) ...
+      const int g = (warp - 4) >> 2;
+      const int r = (warp & 3) * 32 + lane;
+      const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+      const uint32_t ocol = 256 * g;
       grid_dep_wait();
       SegIter it = it0;
       uint32_t nreq = 0, uc = 0;
@@ -831,17 +834,18 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       while (ok && it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
         for (;;) {
           if (lane == 0) sb.prog[warp] = (int)nreq;
-          if (!warp_wait(sb, bar(B_REQ), nreq & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
+          if (!warp_wait(sb, bar(B_REQ + g), nreq & 1, p.dev_status, false, p.timeout_rec, __LINE__)) { ok = false; break; }
           ++nreq;
-          const Req q = sb.req;
+          const Req q = sb.req[g];
           if (q.kind == 0) {
             if (q.tail) {
-              // Rows past the sequence end may hold anything (NaN): zero them so 0 * row stays 0.
+              // Rows past the sequence end may hold anything (NaN): zero them in this half's latent
+              // stage so that 0 * row stays 0.
               const int nrow = kTileKeys - q.nvalid;
-              for (int e = threadIdx.x - 128; e < nrow * 64; e += 128) {
-                const int row = q.nvalid + e / 64, rest = e % 64, ch = rest / 8, piece = rest % 8;
-                unsigned char *vt = tiles + (ch < 4 ? q.vstage0 : q.vstage1) * kVStageBytes;
-                *reinterpret_cast<uint4 *>(vt + (ch & 3) * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
+              unsigned char *vt = tiles + q.vstage * kVStageBytes;
+              for (int e = r; e < nrow * 32; e += kRows) {
+                const int row = q.nvalid + e / 32, rest = e % 32, ch = rest / 8, piece = rest % 8;
+                *reinterpret_cast<uint4 *>(vt + ch * kChunkBytes + row * 128 + piece * 16) = make_uint4(0, 0, 0, 0);
               }
               fence_proxy_async_smem();
             }
@@ -850,18 +854,18 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
               const float a = __uint_as_float(ld_shared_u32(slot_factors(smem_u32(tiles), q.slot) +
                                                             4 * ((r >> 5) * kPaWords + (r & 31))));
 #pragma unroll 1
-              for (int c = 0; c < 16; ++c) {
+              for (int c = 0; c < 8; ++c) {
                 uint32_t v[32];
-                tmem_ld32(tbase + lane_off + 32 * c, v);
+                tmem_ld32(tbase + lane_off + ocol + 32 * c, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-                tmem_st32(tbase + lane_off + 32 * c, v);
+                tmem_st32(tbase + lane_off + ocol + 32 * c, v);
               }
               tmem_wait_st();
               tc_fence_before();
             }
-            mbar_arrive(bar(B_REQDONE));
+            mbar_arrive(bar(B_REQDONE + g));
             continue;
           }
           // Unit epilogue: the unit's last MMAs and the row statistics.
@@ -875,11 +879,11 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(statsempty_remote);
           const float inv = l > 0.f ? 1.f / l : 0.f;
-          __nv_bfloat16 *dst = p.o_part + ((int64_t)q.segid * kRows + r) * kDc;
+          __nv_bfloat16 *dst = p.o_part + ((int64_t)q.segid * kRows + r) * kDc + ocol;
 #pragma unroll 1
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 8; ++c) {
             uint32_t v[32];
-            tmem_ld32(tbase + lane_off + 32 * c, v);
+            tmem_ld32(tbase + lane_off + ocol + 32 * c, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; i += 8)
@@ -889,7 +893,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
                              pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
                              pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
           }
-          p.lse_part[(int64_t)q.segid * kRows + r] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
+          if (g == 0) p.lse_part[(int64_t)q.segid * kRows + r] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
           tc_fence_before();
           mbar_arrive(bar(B_OFREE));
           ++uc;
