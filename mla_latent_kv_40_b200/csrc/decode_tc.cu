@@ -284,11 +284,10 @@ struct SegIter {
 
 // Bounded wait that turns a timeout into the CTA-wide abort state.  The first
 // timeout of each (CTA rank, warp) in the grid is recorded in rec[1 + 6 * (12 * rank + warp) ..]:
-// cluster, barrier slot, parity, source line, the warp's progress counter.
-__device__ __forceinline__ bool wait_or_abort(SmemB &sb, uint32_t bar, uint32_t parity, int *dev_status,
-                                              bool cluster_scope = false, int *rec = nullptr, int tag = 0) {
-  if (*(volatile int *)&sb.abort) return false;
-  if (mbar_wait(bar, parity, kWaitNs, cluster_scope)) return true;
+// cluster, barrier slot, parity, source line, the warp's progress counter.  The record is
+// written out of line (it only runs after a timeout), which keeps the many inlined waits small.
+__device__ __noinline__ bool wait_timed_out(SmemB &sb, uint32_t bar, uint32_t parity, int *dev_status, int *rec,
+                                            int tag) {
   *(volatile int *)&sb.abort = 1;
   report(dev_status, MLA_ERR_TIMEOUT);
   if (rec) {
@@ -304,6 +303,13 @@ __device__ __forceinline__ bool wait_or_abort(SmemB &sb, uint32_t bar, uint32_t 
     atomicAdd(rec, 1);
   }
   return false;
+}
+
+__device__ __forceinline__ bool wait_or_abort(SmemB &sb, uint32_t bar, uint32_t parity, int *dev_status,
+                                              bool cluster_scope = false, int *rec = nullptr, int tag = 0) {
+  if (*(volatile int *)&sb.abort) return false;
+  if (mbar_wait(bar, parity, kWaitNs, cluster_scope)) return true;
+  return wait_timed_out(sb, bar, parity, dev_status, rec, tag);
 }
 
 // Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast, and then
@@ -728,29 +734,30 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           const uint32_t sbuf = ns & 1;
           warp_wait(sb, bar(B_SFULL + sbuf), (ns >> 1) & 1, p.dev_status, false, p.timeout_rec, __LINE__);
           tc_fence_after();
-          // My page of the tile is page h: keys 64T + 64h + k, k < 64.  The scores come into
-          // registers and the buffer is released at once for the tile after next.
-          uint32_t sc[64];
-          {
-            uint32_t v0[32], v1[32];
-            tmem_ld32(tbase + lane_off + kSCol + 128 * sbuf + 64 * h, v0);
-            tmem_ld32(tbase + lane_off + kSCol + 128 * sbuf + 64 * h + 32, v1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              sc[i] = v0[i];
-              sc[32 + i] = v1[i];
-            }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
+          // My page of the tile is page h: keys 64T + 64h + k, k < 64.  Its scores are read from
+          // tensor memory twice, 32 columns at a time (for the maximum, then for P), so that at most
+          // 32 of them are live in registers; the buffer is released after the last read.
+          const uint32_t scol = tbase + lane_off + kSCol + 128 * sbuf + 64 * h;
+          auto release_s = [&]() {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SEMPTY + sbuf));
+          };
           // Valid while below the row's causal limit and inside the pages this tile holds.
           const int nvalid = min(vis_end - (T + h) * kTileKeys, (npg - h) * kTileKeys);
           float mx = -CUDART_INF_F;
+#pragma unroll 1
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t v[32];
+            tmem_ld32(scol + 32 * c2, v);
+            tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 64; ++k)
-            if (k < nvalid) mx = fmaxf(mx, __uint_as_float(sc[k]) * p.scale_log2);
+            for (int k = 0; k < 32; ++k)   // a select, not a branch: nvalid differs between rows
+              mx = fmaxf(mx, 32 * c2 + k < nvalid ? __uint_as_float(v[k]) : -CUDART_INF_F);
+          }
+          // The scale is positive: the scaled maximum is the maximum of the scaled scores.
+          mx *= p.scale_log2;
+          if (h >= npg) release_s();   // no page here: nothing more to read
           sb.xmax[ns & 1][h][r] = mx;
           asm volatile("bar.sync 1, 256;" ::: "memory");
           mx = fmaxf(mx, sb.xmax[ns & 1][h ^ 1][r]);
@@ -773,18 +780,26 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             // page of a score tile carries the tile's factors) and the warp's flag word.
             unsigned char *prow = stgp + 4096 * q4 + (lane >> 3) * 1024 + (lane & 7) * 128;
             float psum = 0.f;
+#pragma unroll 1
+            for (int c2 = 0; c2 < 2; ++c2) {
+              uint32_t v[32];
+              tmem_ld32(scol + 32 * c2, v);
+              tmem_wait_ld();
+              if (c2 == 1) release_s();
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint32_t pk[4];
+              for (int c = 0; c < 4; ++c) {
+                uint32_t pk[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int kk = 8 * c + 2 * e;
-                const float p0 = (kk < nvalid) ? exp2f(__uint_as_float(sc[kk]) * p.scale_log2 - m_ref) : 0.f;
-                const float p1 = (kk + 1 < nvalid) ? exp2f(__uint_as_float(sc[kk + 1]) * p.scale_log2 - m_ref) : 0.f;
-                pk[e] = pack_bf16x2(p0, p1);
-                psum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+                for (int e = 0; e < 4; ++e) {
+                  const int k = 8 * c + 2 * e, kk = 32 * c2 + k;
+                  // Keys past the row's limit get exponent -inf: exp2 gives exactly 0, without a branch.
+                  const float p0 = exp2f(kk < nvalid ? __uint_as_float(v[k]) * p.scale_log2 - m_ref : -CUDART_INF_F);
+                  const float p1 = exp2f(kk + 1 < nvalid ? __uint_as_float(v[k + 1]) * p.scale_log2 - m_ref : -CUDART_INF_F);
+                  pk[e] = pack_bf16x2(p0, p1);
+                  psum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+                }
+                *reinterpret_cast<uint4 *>(prow + (((4 * c2 + c) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
               }
-              *reinterpret_cast<uint4 *>(prow + ((c ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             }
             l += psum;
             float *pa = reinterpret_cast<float *>(stga) + q4 * kPaWords;
