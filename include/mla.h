@@ -410,8 +410,10 @@ MLA_API int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, 
 
 /*
  * mla_decode_launches — how many kernels one mla_decode call launches for this
- *   shape (query absorption, attention, combine); for launch accounting in
- *   profilers and benchmarks.  Writes *count; no device work.
+ *   shape (query absorption, attention, and the combine: on the tensor-core
+ *   path a merge of the split partials and the W_UV product, on the CUDA-core
+ *   path one kernel); for launch accounting in profilers and benchmarks.
+ *   Writes *count; no device work.
  */
 MLA_API int mla_decode_launches(const mla_dims *dims, int n_q, int *count);
 

@@ -927,166 +927,135 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   cluster_sync();   // no CTA leaves while its peer may still touch its shared memory
 }
 
-// ------------------------------------------------------------ combine (+ W_UV)
-// CTA = (head s, 64 query rows (b, j)).  The split partials of each row are
-// merged by their log-sum-exps into a bf16 [64 x 512] tile o_lat, which is then
-// multiplied by W_UV[s] ([512 x d_v]) on the tensor cores, transposed so that
-// W_UV supplies the 128-row M side: out^T [d_v x 64] = W_UV^(s)T . o_lat^T
-// (A = W_UV^T, M-major; B = o_lat, K-major; fp32 accumulator in 64 tensor-memory
-// columns).  All of W_UV[s] (128 KB) is requested at the start, straight into
-// the MMA's 128-byte-swizzled operand layout, so its transfer overlaps the merge.
+// ------------------------------------------------------------ merge of the split partials
+// One warp per (query row g = (b, j), head s): the pieces of g's unit are merged by their
+// log-sum-exps into o_lat[g][s][0 .. 512) (bf16) and lse_out[g][s] = log of the summed exp.  Each
+// lane owns 16 latent columns (8 in each half of the row), and the loads of up to kMergeUnroll
+// pieces are in flight together, so a unit cut into a few pieces costs one round of loads.
+constexpr int kMergeThreads = 256;
+constexpr int kMergeUnroll = 4;
+constexpr int kMaxSegPerUnit = kMaxClusters + 1;
+
+__global__ void __launch_bounds__(kMergeThreads)
+tc_merge_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part,
+                const float *lse_part, __nv_bfloat16 *o_lat, float *lse_out) {
+  sm100::grid_dep_launch();
+  sm100::grid_dep_wait();   // the partials and the segment table come from the attention kernel
+  const int lane = threadIdx.x & 31;
+  const int64_t item = (int64_t)blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
+  if (item >= (int64_t)B * n_q * H) return;
+  const int g = (int)(item / H), s = (int)(item % H);
+  const int b = g / n_q, j = g % n_q;
+  const int gr = j * H + s;
+  const int u = b * n_rb + gr / kRows, lr = gr % kRows;
+  int s0 = seg_info[2 * u], ns = seg_info[2 * u + 1];
+  ns = ns < 0 ? 0 : (ns > kMaxSegPerUnit ? kMaxSegPerUnit : ns);
+  if (s0 < 0 || s0 + ns > max_segs) {
+    s0 = 0;
+    ns = 0;
+  }
+  const float *lse_row = lse_part + (int64_t)s0 * kRows + lr;
+  float m = -CUDART_INF_F;
+  for (int k = lane; k < ns; k += 32) m = fmaxf(m, lse_row[(int64_t)k * kRows]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.f;
+  if (m != -CUDART_INF_F)
+    for (int k = lane; k < ns; k += 32) sum += __expf(lse_row[(int64_t)k * kRows] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  float v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = 0.f;
+  for (int k0 = 0; k0 < ns; k0 += kMergeUnroll) {
+    uint4 x[kMergeUnroll][2];
+    float wk[kMergeUnroll];
+#pragma unroll
+    for (int i = 0; i < kMergeUnroll; ++i) {
+      const int k = k0 + i;
+      const bool have = k < ns;
+      const __nv_bfloat16 *src = o_part + ((int64_t)(s0 + (have ? k : 0)) * kRows + lr) * kDc + 8 * lane;
+      x[i][0] = have ? *reinterpret_cast<const uint4 *>(src) : make_uint4(0, 0, 0, 0);
+      x[i][1] = have ? *reinterpret_cast<const uint4 *>(src + 256) : make_uint4(0, 0, 0, 0);
+      wk[i] = have && m != -CUDART_INF_F ? __expf(lse_row[(int64_t)k * kRows] - m) * inv : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kMergeUnroll; ++i)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[i][hh]);
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 f = __bfloat1622float2(xh[e2]);
+          v[8 * hh + 2 * e2] = fmaf(wk[i], f.x, v[8 * hh + 2 * e2]);
+          v[8 * hh + 2 * e2 + 1] = fmaf(wk[i], f.y, v[8 * hh + 2 * e2 + 1]);
+        }
+      }
+  }
+  __nv_bfloat16 *dst = o_lat + ((int64_t)g * H + s) * kDc + 8 * lane;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint4 packed;
+    __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) ph[e2] = __floats2bfloat162_rn(v[8 * hh + 2 * e2], v[8 * hh + 2 * e2 + 1]);
+    *reinterpret_cast<uint4 *>(dst + 256 * hh) = packed;
+  }
+  if (lane == 0 && lse_out) lse_out[(int64_t)g * H + s] = sum > 0.f ? m + logf(sum) : -CUDART_INF_F;
+}
+
+// ------------------------------------------------------------ W_UV product
+// CTA = (head s, 64 query rows (b, j)): out^T [d_v x 64] = W_UV^(s)T . o_lat^T on the tensor cores,
+// with W_UV supplying the 128-row M side (A = W_UV^T, M-major; B = o_lat, K-major; fp32
+// accumulator in 64 tensor-memory columns).  All of W_UV[s] (128 KB) is requested before the
+// kernel waits for the merge, straight into the MMA's 128-byte-swizzled operand layout, so its
+// transfer overlaps the merge; the 64 rows of o_lat follow the same way.
 constexpr int kCombRows = 64;
 constexpr int kCombThreads = 256;
-constexpr int kMaxSegPerUnit = kMaxClusters + 1;
 constexpr int kDv = 128;                                   // the W_UV tile width this kernel takes
 constexpr uint32_t kOlBytes = kCombRows * kDc * 2;         // o_lat: [8 K-chunks][64 rows][128 B]
 constexpr uint32_t kWuvBytes = kDc * kDv * 2;              // W_UV^T: [8 K-chunks][2 M-chunks][64 K rows][128 B]
 
 __global__ void __launch_bounds__(kCombThreads)
-tc_combine_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part,
-                  const float *lse_part, const __nv_bfloat16 *w_uv, int d_v, __nv_bfloat16 *out, float *lse_out,
+tc_combine_kernel(int rows, int H, const __nv_bfloat16 *o_lat, const __nv_bfloat16 *w_uv, __nv_bfloat16 *out,
                   int *dev_status) {
   extern __shared__ unsigned char csm_raw[];
   unsigned char *csm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *ol = csm;                                                          // o_lat, K-major, swizzled
   unsigned char *wa = csm + kOlBytes;                                               // W_UV^T, M-major, swizzled
-  float *wgt = reinterpret_cast<float *>(wa + kWuvBytes);                           // [64][kMaxSegPerUnit]
-  int *sinfo = reinterpret_cast<int *>(wgt + kCombRows * kMaxSegPerUnit);          // [64][3]
   __shared__ __align__(8) uint64_t bar_mma;
   __shared__ uint32_t tmem_slot;
   const int s = blockIdx.x;
   const int g0 = blockIdx.y * kCombRows;
-  const int rows = B * n_q;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  (void)d_v;
   sm100::grid_dep_launch();
-  const __nv_bfloat16 *w = w_uv ? w_uv + (int64_t)s * kDc * kDv : nullptr;
-
-  if (w) {
-    if (tid == 0) {
-      mbar_init(smem_u32(&bar_mma), 1);
-      fence_mbar_init();
-    }
-    if (warp == 0) {
-      tmem_alloc(smem_u32(&tmem_slot), kCombRows);
-      tmem_relinquish();
-    }
-    // W_UV[s] (an input: no need to wait): row k, 16-byte group q (8 output columns) ->
-    // K-chunk k/64, M-chunk q/8, row k%64, group (q%8) XOR (k%8).
-    for (int c = tid; c < kDc * (kDv / 8); c += kCombThreads) {
-      const int k = c >> 4, q = c & 15;
-      const int kc = k >> 6, kr = k & 63, mc = q >> 3, qq = q & 7;
-      mma::cp16(wa + ((kc * 2 + mc) * 64 + kr) * 128 + ((qq ^ (kr & 7)) << 4), w + (int64_t)k * kDv + q * 8, true);
-    }
-    mma::cp_commit();
+  const __nv_bfloat16 *w = w_uv + (int64_t)s * kDc * kDv;
+  if (tid == 0) {
+    mbar_init(smem_u32(&bar_mma), 1);
+    fence_mbar_init();
   }
-  sm100::grid_dep_wait();   // the partials and the segment table come from the attention kernel
-
-  // Merge weights: four threads per row, so every row's segment info and log-sum-exps are
-  // fetched at once rather than one row after another.
-  {
-    const int rr = tid >> 2, sub = tid & 3;
-    const int g = g0 + rr;
-    int s0 = 0, ns = 0, lr = 0;
-    if (g < rows) {
-      const int b = g / n_q, j = g % n_q;
-      const int gr = j * H + s;
-      const int u = b * n_rb + gr / kRows;
-      lr = gr % kRows;
-      s0 = seg_info[2 * u];
-      ns = seg_info[2 * u + 1];
-      ns = ns < 0 ? 0 : (ns > kMaxSegPerUnit ? kMaxSegPerUnit : ns);
-      if (s0 < 0 || s0 + ns > max_segs) { s0 = 0; ns = 0; }
-    }
-    float m = -CUDART_INF_F;
-    for (int k = sub; k < ns; k += 4) {
-      const float l = lse_part[(int64_t)(s0 + k) * kRows + lr];
-      wgt[rr * kMaxSegPerUnit + k] = l;
-      m = fmaxf(m, l);
-    }
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    float sum = 0.f;
-    for (int k = sub; k < ns; k += 4) {
-      const float e = m == -CUDART_INF_F ? 0.f : __expf(wgt[rr * kMaxSegPerUnit + k] - m);
-      wgt[rr * kMaxSegPerUnit + k] = e;
-      sum += e;
-    }
-    sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-    sum += __shfl_xor_sync(0xffffffffu, sum, 2);
-    const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    for (int k = sub; k < ns; k += 4) wgt[rr * kMaxSegPerUnit + k] *= inv;
-    if (sub == 0) {
-      sinfo[3 * rr] = s0;
-      sinfo[3 * rr + 1] = ns;
-      sinfo[3 * rr + 2] = lr;
-      if (g < rows && lse_out) lse_out[(int64_t)g * H + s] = sum > 0.f ? m + logf(sum) : -CUDART_INF_F;
-    }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_slot), kCombRows);
+    tmem_relinquish();
   }
-  __syncthreads();
-  // Merge, 8 latent columns (16 bytes of every partial) per item.  A thread owns one column
-  // group and, per pass, 8 rows; it walks the segments outermost so that its 8 loads of one
-  // segment are independent and in flight together.
-  {
-    constexpr int kGroups = kDc / 8;                         // 64 column groups
-    constexpr int kRowStep = kCombThreads / kGroups;         // 4
-    constexpr int kItems = 8;
-    constexpr int kPasses = kCombRows / (kRowStep * kItems); // 2
-    const int c8 = tid % kGroups, rr0 = tid / kGroups;
-#pragma unroll 1
-    for (int pass = 0; pass < kPasses; ++pass) {
-      float v[kItems][8];
-      int maxns = 0;
-#pragma unroll
-      for (int i = 0; i < kItems; ++i) {
-        maxns = max(maxns, sinfo[3 * (rr0 + kRowStep * (i + kItems * pass)) + 1]);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v[i][k] = 0.f;
-      }
-      for (int k = 0; k < maxns; ++k) {
-        uint4 x[kItems];
-#pragma unroll
-        for (int i = 0; i < kItems; ++i) {
-          const int rr = rr0 + kRowStep * (i + kItems * pass);
-          x[i] = k < sinfo[3 * rr + 1] ? *reinterpret_cast<const uint4 *>(
-                                             o_part + ((int64_t)(sinfo[3 * rr] + k) * kRows + sinfo[3 * rr + 2]) * kDc + c8 * 8)
-                                       : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int i = 0; i < kItems; ++i) {
-          const int rr = rr0 + kRowStep * (i + kItems * pass);
-          const float wk = k < sinfo[3 * rr + 1] ? wgt[rr * kMaxSegPerUnit + k] : 0.f;
-          const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[i]);
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            const float2 f = __bfloat1622float2(xh[e2]);
-            v[i][2 * e2] = fmaf(wk, f.x, v[i][2 * e2]);
-            v[i][2 * e2 + 1] = fmaf(wk, f.y, v[i][2 * e2 + 1]);
-          }
-        }
-      }
-      // Row rr, latent group c8 -> K-chunk c8/8, group (c8%8) XOR (rr%8) of the row's 128 bytes.
-#pragma unroll
-      for (int i = 0; i < kItems; ++i) {
-        const int rr = rr0 + kRowStep * (i + kItems * pass);
-        uint4 packed;
-        __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) ph[e2] = __floats2bfloat162_rn(v[i][2 * e2], v[i][2 * e2 + 1]);
-        *reinterpret_cast<uint4 *>(ol + (c8 >> 3) * 8192 + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4)) = packed;
-      }
-    }
+  // W_UV[s] (an input: no need to wait): row k, 16-byte group q (8 output columns) ->
+  // K-chunk k/64, M-chunk q/8, row k%64, group (q%8) XOR (k%8).
+  for (int c = tid; c < kDc * (kDv / 8); c += kCombThreads) {
+    const int k = c >> 4, q = c & 15;
+    const int kc = k >> 6, kr = k & 63, mc = q >> 3, qq = q & 7;
+    mma::cp16(wa + ((kc * 2 + mc) * 64 + kr) * 128 + ((qq ^ (kr & 7)) << 4), w + (int64_t)k * kDv + q * 8, true);
   }
-  if (!w) {   // latent output: o_lat itself
-    __syncthreads();
-    for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
-      const int rr = e / (kDc / 8), c8 = e % (kDc / 8), g = g0 + rr;
-      if (g < rows)
-        *reinterpret_cast<uint4 *>(out + ((int64_t)g * H + s) * kDc + c8 * 8) =
-            *reinterpret_cast<const uint4 *>(ol + (c8 >> 3) * 8192 + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4));
-    }
-    return;
+  mma::cp_commit();
+  sm100::grid_dep_wait();   // o_lat comes from the merge kernel
+  // Row rr, latent group c8 (8 columns) -> K-chunk c8/8, group (c8%8) XOR (rr%8) of the row's 128 bytes;
+  // rows past the end are zero.
+  for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
+    const int rr = e >> 6, c8 = e & 63, g = g0 + rr;
+    mma::cp16(ol + (c8 >> 3) * 8192 + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4),
+              o_lat + ((int64_t)(g < rows ? g : 0) * H + s) * kDc + c8 * 8, g < rows);
   }
+  mma::cp_commit();
   // Both operands written by this CTA's threads (generic proxy) -> visible to the tensor cores.
   mma::cp_wait<0>();
   fence_proxy_async_smem();
@@ -1167,7 +1136,7 @@ int make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, ui
 }
 
 struct WsLayout {
-  size_t seg_info, o_part, lse_part, total;
+  size_t seg_info, o_part, lse_part, o_lat, total;
 };
 
 int clusters_for_device();
@@ -1182,7 +1151,8 @@ WsLayout ws_layout(int B, int n_rb) {
   L.seg_info = 0;
   L.o_part = a256(U * 2 * sizeof(int) + kTimeoutRecInts * sizeof(int));
   L.lse_part = L.o_part + a256(segs * kRows * kDc * sizeof(__nv_bfloat16));
-  L.total = L.lse_part + a256(segs * kRows * sizeof(float));
+  L.o_lat = L.lse_part + a256(segs * kRows * sizeof(float));           // merged rows, [B n_q][H][512]
+  L.total = L.o_lat + a256(U * kRows * kDc * sizeof(__nv_bfloat16));
   return L;
 }
 
@@ -1237,7 +1207,7 @@ bool tc_decode_supported(const mla_dims &d, int n_q) {
          d.d_v == 128 && n_q * d.n_heads <= 2 * kRows;
 }
 
-int tc_decode_kernel_launches() { return 2; }
+int tc_decode_kernel_launches() { return 3; }   // attention, merge, W_UV product
 
 size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q) {
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
@@ -1312,17 +1282,25 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
   const WsLayout L = ws_layout(B, n_rb);
   char *w = static_cast<char *>(ws);
-  const size_t smem = 1024 + kOlBytes + kWuvBytes + sizeof(float) * kCombRows * kMaxSegPerUnit +
-                      sizeof(int) * 3 * kCombRows;
   if (w_uv && (d.d_v != kDv || (reinterpret_cast<uintptr_t>(w_uv) & 15))) return MLA_ERR_UNSUPPORTED;
+  const int rows = B * n_q;
+  // Merge into o_lat: the output itself when no W_UV is given, else the workspace's row buffer.
+  __nv_bfloat16 *o_lat = w_uv ? reinterpret_cast<__nv_bfloat16 *>(w + L.o_lat) : static_cast<__nv_bfloat16 *>(out);
+  const int64_t warps = (int64_t)rows * d.n_heads;
+  const dim3 mgrid((unsigned)((warps + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
+  if (launch_pdl(tc_merge_kernel, mgrid, dim3(kMergeThreads), 0, st, B, n_q, d.n_heads, n_rb,
+                 B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
+                 reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part), reinterpret_cast<const float *>(w + L.lse_part),
+                 o_lat, lse) != cudaSuccess)
+    return MLA_ERR_CUDA;
+  if (!w_uv) return MLA_OK;
+  const size_t smem = 1024 + kOlBytes + kWuvBytes;
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
-  const dim3 grid(d.n_heads, (B * n_q + kCombRows - 1) / kCombRows);
-  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, B, n_q, d.n_heads, n_rb,
-                    B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
-                    reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part),
-                    reinterpret_cast<const float *>(w + L.lse_part), static_cast<const __nv_bfloat16 *>(w_uv),
-                    d.d_v, static_cast<__nv_bfloat16 *>(out), lse, dev_status) == cudaSuccess
+  const dim3 grid(d.n_heads, (rows + kCombRows - 1) / kCombRows);
+  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, rows, d.n_heads,
+                    static_cast<const __nv_bfloat16 *>(o_lat), static_cast<const __nv_bfloat16 *>(w_uv),
+                    static_cast<__nv_bfloat16 *>(out), dev_status) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
 }
