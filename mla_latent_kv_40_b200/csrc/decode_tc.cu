@@ -123,7 +123,10 @@ struct SmemB {                       // small region after the tiles
   uint32_t tmem_base;
   int abort;
   int plan_u0, plan_p0, plan_s0;     // first unit of this cluster, its tile prefix and segment prefix
+  int plan_k0;                       // non-empty units before the first unit
   int plan_C;                        // clusters that get work: min(launched clusters, total tiles)
+  int plan_beta;                     // cost of a unit start, in tiles (see Split)
+  long long plan_W;                  // total cost
   int prog[kThreads / 32];           // per-warp progress (tiles handled), kept for timeout records
   long long plan_start, plan_end, plan_total;
 };
@@ -176,20 +179,35 @@ __device__ __forceinline__ int unit_tiles(const TcParams &p, int u) {
   return e > 0 ? (e + kTileKeys - 1) / kTileKeys : 0;
 }
 
-// Cluster owning global tile t when T tiles are cut into C even ranges
-// [floor(c T / C), floor((c+1) T / C)).
-__device__ __forceinline__ int cluster_of(long long t, long long T, long long C) {
-  return (int)(((t + 1) * C + T - 1) / T - 1);
+// Work split.  The units' 64-key tiles, in unit order, are cut into C ranges of about equal cost.
+// A tile costs 1, and every unit start after the first costs kBoundaryCost more: a cluster that
+// moves on to a new unit drains and refills its pipeline there (the next query block goes into
+// tensor memory, the finished unit's O is written out).  On V3 shapes at batch 64 x 4096, cluster
+// end times fit ~1.56 us per tile plus ~12.5 us per segment, so a unit start costs ~8 tiles.
+// Tile t of unit u costs t + beta k_u (k_u: non-empty units before u); cluster c owns the tiles
+// whose cost lies in [floor(c W / C), floor((c+1) W / C)).  beta is used only while one unit start
+// cannot jump over a whole cluster's share, (beta + 1) C <= W.
+constexpr int kBoundaryCost = 8;
+struct Split {
+  long long W;   // total cost: tiles + beta (non-empty units - 1)
+  int beta, C;
+};
+
+__device__ __forceinline__ int cluster_of(long long t, int k, const Split &sp) {
+  const long long cost = t + (long long)sp.beta * k;
+  return (int)(((cost + 1) * sp.C + sp.W - 1) / sp.W - 1);
 }
 
-// Warp-level plan: total tiles, this cluster's range, its first unit and the
-// tile / segment prefixes of that unit.  Every CTA computes the same values.
+// Warp-level plan: total tiles and cost, this cluster's tile range, its first unit and the tile,
+// non-empty-unit and segment prefixes of that unit.  Every CTA computes the same values.
 __device__ __forceinline__ void make_plan(const TcParams &p, SmemB &sb, int cid, int C) {
   const int lane = threadIdx.x & 31;
   long long total = 0;
+  int une = 0;
   for (int u0 = 0; u0 < p.U; u0 += 32) {
     const int u = u0 + lane;
     int nt = u < p.U ? unit_tiles(p, u) : 0;
+    une += __popc(__ballot_sync(0xffffffffu, nt > 0));
 #pragma unroll
     for (int o = 16; o; o >>= 1) nt += __shfl_xor_sync(0xffffffffu, nt, o);
     total += nt;
@@ -197,65 +215,104 @@ __device__ __forceinline__ void make_plan(const TcParams &p, SmemB &sb, int cid,
   // With fewer tiles than clusters only the first `total` clusters get work, so
   // that every active range is non-empty and segment ids have no gaps.
   C = (int)(total < C ? total : C);
-  const long long start = cid < C ? total * cid / C : 0, end = cid < C ? total * (cid + 1) / C : 0;
-  long long tp = 0, sp = 0;   // running tile / segment prefix
+  Split sp;
+  sp.C = C > 0 ? C : 1;
+  sp.beta = kBoundaryCost;
+  sp.W = total + (long long)sp.beta * (une > 0 ? une - 1 : 0);
+  if ((long long)(sp.beta + 1) * sp.C > sp.W) {
+    sp.beta = 0;
+    sp.W = total;
+  }
+  if (sp.W <= 0) sp.W = 1;
+  // Cluster c's range is [x_c, x_{c+1}) with x_c the first tile of cost >= floor(c W / C); inside
+  // unit u that is max(P_u, floor(c W / C) - beta k_u), in the first unit whose last tile reaches it.
+  const long long Ls = cid < C ? (long long)cid * sp.W / sp.C : 0;
+  const long long Le = cid < C ? (long long)(cid + 1) * sp.W / sp.C : 0;
+  const bool last_c = cid + 1 >= C;
+  long long tp = 0, sp_seg = 0;   // running tile / segment prefix
+  int kp = 0;                     // running count of non-empty units
   int found = -1;
-  long long fp = 0, fs = 0;
-  for (int u0 = 0; u0 < p.U && found < 0; u0 += 32) {
+  long long fp = 0, fs = 0, start = 0, end = last_c ? total : -1;
+  int fk = 0;
+  for (int u0 = 0; u0 < p.U && (found < 0 || end < 0); u0 += 32) {
     const int u = u0 + lane;
     const int nt = u < p.U ? unit_tiles(p, u) : 0;
-    // inclusive scan of nt
-    int inc = nt;
+    // inclusive scans of nt and of (nt > 0)
+    int inc = nt, kinc = nt > 0 ? 1 : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += v;
+      const int kv = __shfl_up_sync(0xffffffffu, kinc, o);
+      if (lane >= o) {
+        inc += v;
+        kinc += kv;
+      }
     }
     const long long my_p = tp + inc - nt;
+    const int my_k = kp + kinc - (nt > 0 ? 1 : 0);
     int ns = 0;
-    if (nt > 0 && total > 0) ns = cluster_of(my_p + nt - 1, total, C) - cluster_of(my_p, total, C) + 1;
+    if (nt > 0 && total > 0) ns = cluster_of(my_p + nt - 1, my_k, sp) - cluster_of(my_p, my_k, sp) + 1;
     int sinc = ns;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, sinc, o);
       if (lane >= o) sinc += v;
     }
-    const long long my_s = sp + sinc - ns;
-    const bool hit = u < p.U && nt > 0 && my_p <= start && start < my_p + nt;
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (m) {
-      const int src = __ffs(m) - 1;
-      found = u0 + src;
-      fp = __shfl_sync(0xffffffffu, my_p, src);
-      fs = __shfl_sync(0xffffffffu, my_s, src);
+    const long long my_s = sp_seg + sinc - ns;
+    const long long last_cost = my_p + nt - 1 + (long long)sp.beta * my_k;
+    if (found < 0) {
+      const unsigned m = __ballot_sync(0xffffffffu, u < p.U && nt > 0 && last_cost >= Ls);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        found = u0 + src;
+        fp = __shfl_sync(0xffffffffu, my_p, src);
+        fs = __shfl_sync(0xffffffffu, my_s, src);
+        fk = __shfl_sync(0xffffffffu, my_k, src);
+        const long long x = Ls - (long long)sp.beta * fk;
+        start = x > fp ? x : fp;
+      }
+    }
+    if (end < 0) {
+      const unsigned m = __ballot_sync(0xffffffffu, u < p.U && nt > 0 && last_cost >= Le);
+      if (m) {
+        const int src = __ffs(m) - 1;
+        const long long ep = __shfl_sync(0xffffffffu, my_p, src);
+        const long long x = Le - (long long)sp.beta * __shfl_sync(0xffffffffu, my_k, src);
+        end = x > ep ? x : ep;
+      }
     }
     tp += __shfl_sync(0xffffffffu, inc, 31);
-    sp += __shfl_sync(0xffffffffu, sinc, 31);
+    kp += __shfl_sync(0xffffffffu, kinc, 31);
+    sp_seg += __shfl_sync(0xffffffffu, sinc, 31);
   }
+  if (end < 0) end = total;
   if (lane == 0) {
-    sb.plan_C = C;
+    sb.plan_C = sp.C;
+    sb.plan_beta = sp.beta;
+    sb.plan_W = sp.W;
     sb.plan_total = total;
     sb.plan_start = start;
     sb.plan_end = (found < 0 || cid >= C) ? start : end;
     sb.plan_u0 = found < 0 ? 0 : found;
     sb.plan_p0 = (int)fp;
     sb.plan_s0 = (int)fs;
+    sb.plan_k0 = fk;
   }
 }
 
 // Iterates the (unit, tile range) segments of this cluster.
 struct SegIter {
-  int u, prefix, seg_prefix;
-  long long pos, end, total;
-  int C;
+  int u, prefix, seg_prefix, k;   // k: non-empty units before u
+  long long pos, end;
+  Split sp;
   __device__ __forceinline__ bool next(const TcParams &p, int cid, int &b, int &rb, int &t0, int &t1, int &segid, bool &first_of_unit,
                        int &nseg_unit) {
     while (pos < end && u < p.U) {
       const int nt = unit_tiles(p, u);
       const long long lo = pos > prefix ? pos : prefix;
       const long long hi = end < (long long)prefix + nt ? end : (long long)prefix + nt;
-      const int c0 = nt > 0 ? cluster_of(prefix, total, C) : 0;
-      const int ns = nt > 0 ? cluster_of((long long)prefix + nt - 1, total, C) - c0 + 1 : 0;
+      const int c0 = nt > 0 ? cluster_of(prefix, k, sp) : 0;
+      const int ns = nt > 0 ? cluster_of((long long)prefix + nt - 1, k, sp) - c0 + 1 : 0;
       if (lo < hi) {
         b = u / p.n_rb;
         rb = u % p.n_rb;
@@ -270,12 +327,14 @@ struct SegIter {
         if (hi == (long long)prefix + nt) {
           prefix += nt;
           seg_prefix += ns;
+          k += nt > 0 ? 1 : 0;
           u = cur_u + 1;
         }
         return true;
       }
       prefix += nt;
       seg_prefix += ns;
+      k += nt > 0 ? 1 : 0;
       ++u;
     }
     return false;
@@ -415,10 +474,12 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
   it0.u = sb.plan_u0;
   it0.prefix = sb.plan_p0;
   it0.seg_prefix = sb.plan_s0;
+  it0.k = sb.plan_k0;
   it0.pos = sb.plan_start;
   it0.end = sb.plan_end;
-  it0.total = sb.plan_total;
-  it0.C = sb.plan_C;
+  it0.sp.W = sb.plan_W;
+  it0.sp.beta = sb.plan_beta;
+  it0.sp.C = sb.plan_C;
 
   int b, rb, t0, t1, segid, nseg;
   bool first_u;
