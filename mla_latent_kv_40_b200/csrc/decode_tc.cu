@@ -1069,7 +1069,7 @@ tc_merge_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_in
 // ------------------------------------------------------------ W_UV product
 // CTA = (head s, 64 query rows (b, j)): out^T [d_v x 64] = W_UV^(s)T . o_lat^T on the tensor cores,
 // with W_UV supplying the 128-row M side (A = W_UV^T, M-major; B = o_lat, K-major; fp32
-// accumulator in 64 tensor-memory columns).  All of W_UV[s] (128 KB) is requested before the
+// accumulator in 64 tensor-memory columns).  All of W_UV[s] (128 KB) is requested by TMA before the
 // kernel waits for the merge, straight into the MMA's 128-byte-swizzled operand layout, so its
 // transfer overlaps the merge; the 64 rows of o_lat follow the same way.
 constexpr int kCombRows = 64;
@@ -1079,54 +1079,61 @@ constexpr uint32_t kOlBytes = kCombRows * kDc * 2;         // o_lat: [8 K-chunks
 constexpr uint32_t kWuvBytes = kDc * kDv * 2;              // W_UV^T: [8 K-chunks][2 M-chunks][64 K rows][128 B]
 
 __global__ void __launch_bounds__(kCombThreads)
-tc_combine_kernel(int rows, int H, const __nv_bfloat16 *o_lat, const __nv_bfloat16 *w_uv, __nv_bfloat16 *out,
-                  int *dev_status) {
+tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_o, int rows, int H,
+                  __nv_bfloat16 *out, int *dev_status) {
   extern __shared__ unsigned char csm_raw[];
   unsigned char *csm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *ol = csm;                                                          // o_lat, K-major, swizzled
   unsigned char *wa = csm + kOlBytes;                                               // W_UV^T, M-major, swizzled
-  __shared__ __align__(8) uint64_t bar_mma;
+  __shared__ __align__(8) uint64_t bar_w, bar_o, bar_mma;
   __shared__ uint32_t tmem_slot;
+  __shared__ int s_loaded;
   const int s = blockIdx.x;
   const int g0 = blockIdx.y * kCombRows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   sm100::grid_dep_launch();
-  const __nv_bfloat16 *w = w_uv + (int64_t)s * kDc * kDv;
+  // W_UV[s] (an input: no need to wait), as 16 TMA boxes of [64 K rows x 64 output columns] in the
+  // MMA's M-major, 128-byte-swizzled layout: box (K-chunk kc, M-chunk mc) at (kc * 2 + mc) * 8 KB.
   if (tid == 0) {
+    mbar_init(smem_u32(&bar_w), 1);
+    mbar_init(smem_u32(&bar_o), 1);
     mbar_init(smem_u32(&bar_mma), 1);
     fence_mbar_init();
+    tma_prefetch_desc(&map_w);
+    tma_prefetch_desc(&map_o);
+    mbar_expect_tx(smem_u32(&bar_w), kWuvBytes);
+    for (int kc = 0; kc < kDc / 64; ++kc)
+      for (int mc = 0; mc < 2; ++mc)
+        tma_load_2d(smem_u32(wa + (kc * 2 + mc) * 8192), &map_w, 64 * mc, s * kDc + 64 * kc, smem_u32(&bar_w));
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(&tmem_slot), kCombRows);
     tmem_relinquish();
   }
-  // W_UV[s] (an input: no need to wait): row k, 16-byte group q (8 output columns) ->
-  // K-chunk k/64, M-chunk q/8, row k%64, group (q%8) XOR (k%8).
-  for (int c = tid; c < kDc * (kDv / 8); c += kCombThreads) {
-    const int k = c >> 4, q = c & 15;
-    const int kc = k >> 6, kr = k & 63, mc = q >> 3, qq = q & 7;
-    mma::cp16(wa + ((kc * 2 + mc) * 64 + kr) * 128 + ((qq ^ (kr & 7)) << 4), w + (int64_t)k * kDv + q * 8, true);
+  sm100::grid_dep_wait();   // o_lat comes from the merge kernel; out may still be read before it
+  // o_lat rows g0 .. g0 + 63 of head s, K-chunk c -> [64 rows x 128 B] at c * 8 KB (rows past the
+  // end are zero-filled by the copy).
+  if (tid == 0) {
+    mbar_expect_tx(smem_u32(&bar_o), kOlBytes);
+    for (int c = 0; c < kDc / 64; ++c) tma_load_3d(smem_u32(ol + c * 8192), &map_o, 64 * c, s, g0, smem_u32(&bar_o));
   }
-  mma::cp_commit();
-  sm100::grid_dep_wait();   // o_lat comes from the merge kernel
-  // Row rr, latent group c8 (8 columns) -> K-chunk c8/8, group (c8%8) XOR (rr%8) of the row's 128 bytes;
-  // rows past the end are zero.
-  for (int e = tid; e < kCombRows * (kDc / 8); e += kCombThreads) {
-    const int rr = e >> 6, c8 = e & 63, g = g0 + rr;
-    mma::cp16(ol + (c8 >> 3) * 8192 + rr * 128 + (((c8 & 7) ^ (rr & 7)) << 4),
-              o_lat + ((int64_t)(g < rows ? g : 0) * H + s) * kDc + c8 * 8, g < rows);
-  }
-  mma::cp_commit();
-  // Both operands written by this CTA's threads (generic proxy) -> visible to the tensor cores.
-  mma::cp_wait<0>();
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  int loaded = 1;
   if (tid == 0) {
+    if (!mbar_wait(smem_u32(&bar_w), 0, kWaitNs) || !mbar_wait(smem_u32(&bar_o), 0, kWaitNs)) {
+      report(dev_status, MLA_ERR_TIMEOUT);
+      loaded = 0;
+    }
+    s_loaded = loaded;
+  }
+  // Without its operands the MMA is skipped; its barrier is still completed (commit with nothing issued).
+  if (tid == 0) {
+    tc_fence_after();
     const uint32_t idesc = idesc_bf16_f32(128, kCombRows, true, false);
-    for (int kc = 0; kc < kDc / 64; ++kc)
+    for (int kc = 0; kc < kDc / 64 && loaded; ++kc)
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
         mma_ss(tmem, smem_desc_sw128(smem_u32(wa + kc * 16384) + kk * 2048, 8192, 1024),
@@ -1150,6 +1157,7 @@ tc_combine_kernel(int rows, int H, const __nv_bfloat16 *o_lat, const __nv_bfloat
     tmem_ld32(tmem + ((uint32_t)((warp & 3) * 32) << 16) + 32 * (warp >> 2), v);
     tmem_wait_ld();
     __syncthreads();   // every thread is past its reads of o_lat (the MMAs completed before the loads)
+    ok = ok && s_loaded;
 #pragma unroll
     for (int i = 0; i < 32; ++i)
       stg[(32 * (warp >> 2) + i) * lds + (warp & 3) * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
@@ -1166,6 +1174,10 @@ tc_combine_kernel(int rows, int H, const __nv_bfloat16 *o_lat, const __nv_bfloat
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kCombRows);
+  }
+  if (tid == 0 && !loaded) {   // the copies must have landed before this CTA's shared memory goes away
+    mbar_wait(smem_u32(&bar_w), 0, kWaitNs);
+    mbar_wait(smem_u32(&bar_o), 0, kWaitNs);
   }
 }
 
@@ -1191,6 +1203,21 @@ int make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, ui
   cuuint32_t box[2] = {64, 64};
   cuuint32_t es[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// 3-D map over a [d2][d1][d0] bf16 array (d0 contiguous), box [64 x 1 x 64], 128-byte swizzle.
+int make_map3(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+              uint64_t stride2_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return MLA_ERR_CUDA;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {64, 1, 64};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
@@ -1355,12 +1382,16 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
                  o_lat, lse) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (!w_uv) return MLA_OK;
+  // W_UV as [H * 512 rows][128] (boxes of 64 rows x 64 columns); o_lat as [rows][H][512].
+  CUtensorMap mw, mo;
+  int rc = make_map(&mw, w_uv, kDv, (uint64_t)d.n_heads * kDc, (uint64_t)kDv * 2);
+  if (rc) return rc;
+  if ((rc = make_map3(&mo, o_lat, kDc, d.n_heads, rows, (uint64_t)kDc * 2, (uint64_t)d.n_heads * kDc * 2))) return rc;
   const size_t smem = 1024 + kOlBytes + kWuvBytes;
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid(d.n_heads, (rows + kCombRows - 1) / kCombRows);
-  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, rows, d.n_heads,
-                    static_cast<const __nv_bfloat16 *>(o_lat), static_cast<const __nv_bfloat16 *>(w_uv),
+  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, mw, mo, rows, d.n_heads,
                     static_cast<__nv_bfloat16 *>(out), dev_status) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
