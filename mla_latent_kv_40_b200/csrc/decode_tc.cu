@@ -32,16 +32,19 @@
 // Online softmax uses a lazy reference maximum (kept in log2 units): P is
 // exp2(s - m_ref) and m_ref only moves when a tile's maximum exceeds it by more
 // than 8, so the O accumulator is rescaled (tcgen05.ld / st by the value CTA)
-// only on those rare tiles; the final normalisation by the row sum is exact.
+// only on those rare tiles.  The row sum adds P in fp32 (before its rounding to bf16), and O is
+// divided by it once, at the end.
 //
-// Work is split evenly over the persistent clusters by 64-key tiles across all
-// (sequence, 128-row block) units; a unit cut between clusters leaves one
-// partial (O / l, lse) per piece, merged by the combine kernel.  Every wait on
+// Work is split over the persistent clusters by 64-key tiles across all
+// (sequence, 128-row block) units, at about equal cost (a unit start costs a few
+// tiles: see Split); a unit cut between clusters leaves one partial (O / l, lse)
+// per piece, merged by the merge kernel.  Every wait on
 // an mbarrier is bounded in time: on expiry the kernel reports MLA_ERR_TIMEOUT,
 // drains its in-flight copies, frees its tensor memory and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math_constants.h>
+#include <type_traits>
 
 #include <atomic>
 #include <cstring>
@@ -806,15 +809,23 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
           };
           // Valid while below the row's causal limit and inside the pages this tile holds.
           const int nvalid = min(vis_end - (T + h) * kTileKeys, (npg - h) * kTileKeys);
+          // Only a sequence's last page has keys past some row's limit: warps whose rows all see
+          // the whole page skip the per-key mask.
+          const bool whole = __all_sync(0xffffffffu, nvalid >= kTileKeys);
           float mx = -CUDART_INF_F;
 #pragma unroll 1
           for (int c2 = 0; c2 < 2; ++c2) {
             uint32_t v[32];
             tmem_ld32(scol + 32 * c2, v);
             tmem_wait_ld();
+            if (whole) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k)   // a select, not a branch: nvalid differs between rows
-              mx = fmaxf(mx, 32 * c2 + k < nvalid ? __uint_as_float(v[k]) : -CUDART_INF_F);
+              for (int k = 0; k < 32; k += 2) mx = max3f(mx, __uint_as_float(v[k]), __uint_as_float(v[k + 1]));
+            } else {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)   // a select, not a branch: nvalid differs between rows
+                mx = fmaxf(mx, 32 * c2 + k < nvalid ? __uint_as_float(v[k]) : -CUDART_INF_F);
+            }
           }
           // The scale is positive: the scaled maximum is the maximum of the scaled scores.
           mx *= p.scale_log2;
@@ -840,29 +851,39 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             // 32q..32q+31 are its bytes 4096q..4096q+4095), then the rows' rescale factors (the first
             // page of a score tile carries the tile's factors) and the warp's flag word.
             unsigned char *prow = stgp + 4096 * q4 + (lane >> 3) * 1024 + (lane & 7) * 128;
-            float psum = 0.f;
+            float psum0 = 0.f, psum1 = 0.f;   // the row sum, from P before its rounding to bf16
 #pragma unroll 1
             for (int c2 = 0; c2 < 2; ++c2) {
               uint32_t v[32];
               tmem_ld32(scol + 32 * c2, v);
               tmem_wait_ld();
               if (c2 == 1) release_s();
+              // Keys past the row's limit get exponent -inf: exp2 gives exactly 0, without a branch.
+              auto p_half = [&](auto masked) {
 #pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                uint32_t pk[4];
+                for (int c = 0; c < 4; ++c) {
+                  uint32_t pk[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const int k = 8 * c + 2 * e, kk = 32 * c2 + k;
-                  // Keys past the row's limit get exponent -inf: exp2 gives exactly 0, without a branch.
-                  const float p0 = exp2f(kk < nvalid ? __uint_as_float(v[k]) * p.scale_log2 - m_ref : -CUDART_INF_F);
-                  const float p1 = exp2f(kk + 1 < nvalid ? __uint_as_float(v[k + 1]) * p.scale_log2 - m_ref : -CUDART_INF_F);
-                  pk[e] = pack_bf16x2(p0, p1);
-                  psum += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xffff0000u);
+                  for (int e = 0; e < 4; ++e) {
+                    const int k = 8 * c + 2 * e, kk = 32 * c2 + k;
+                    float x0 = __uint_as_float(v[k]) * p.scale_log2 - m_ref;
+                    float x1 = __uint_as_float(v[k + 1]) * p.scale_log2 - m_ref;
+                    if (decltype(masked)::value) {
+                      x0 = kk < nvalid ? x0 : -CUDART_INF_F;
+                      x1 = kk + 1 < nvalid ? x1 : -CUDART_INF_F;
+                    }
+                    const float p0 = exp2f(x0), p1 = exp2f(x1);
+                    pk[e] = pack_bf16x2(p0, p1);
+                    psum0 += p0;
+                    psum1 += p1;
+                  }
+                  *reinterpret_cast<uint4 *>(prow + (((4 * c2 + c) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
-                *reinterpret_cast<uint4 *>(prow + (((4 * c2 + c) ^ (lane & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-              }
+              };
+              if (whole) p_half(std::false_type{});
+              else p_half(std::true_type{});
             }
-            l += psum;
+            l += psum0 + psum1;
             float *pa = reinterpret_cast<float *>(stga) + q4 * kPaWords;
             pa[lane] = h == 0 ? alpha : 1.f;
             const unsigned moved = __ballot_sync(0xffffffffu, need && h == 0 && T != t0);
