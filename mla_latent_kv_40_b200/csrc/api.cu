@@ -296,14 +296,14 @@ int mla_decode_absorbed(const mla_dims *dims, int d_cq, int B, int n_q, const vo
   float *part = reinterpret_cast<float *>(ws + L.part_off);
   // (1) c_Q = h W_DQ.
   L.g_cq.A = h; L.g_cq.B = w_dq; L.g_cq.C = c_q; L.g_cq.part = part;
-  if ((rc = launch_gemm_simt(L.g_cq, bf16, st))) return rc;
+  if ((rc = launch_gemm(L.g_cq, bf16, st))) return rc;
   // (2) latent queries q_lat^(s) = c_Q W_UQK^(s), straight into the absorbed query buffer.
   L.g_qlat.A = c_q; L.g_qlat.B = w_uqk; L.g_qlat.C = q_abs; L.g_qlat.part = part;
-  if ((rc = launch_gemm_simt(L.g_qlat, bf16, st))) return rc;
+  if ((rc = launch_gemm(L.g_qlat, bf16, st))) return rc;
   // (3) RoPE queries q_pe^(s) = RoPE(c_Q W_QR^(s), position), into the query buffer's RoPE slots.
   if (dims->d_rope) {
     L.g_qpe.A = c_q; L.g_qpe.B = w_qr; L.g_qpe.C = q_pe; L.g_qpe.part = part;
-    if ((rc = launch_gemm_simt(L.g_qpe, bf16, st))) return rc;
+    if ((rc = launch_gemm(L.g_qpe, bf16, st))) return rc;
     if ((rc = launch_rope_into_query(B, n_q, dims->n_heads, dims->d_c, dims->d_rope, q_pe, seqlens, q_abs,
                                      dims->rope_base, bf16, st)))
       return rc;
@@ -315,7 +315,7 @@ int mla_decode_absorbed(const mla_dims *dims, int d_cq, int B, int n_q, const vo
   if ((rc = combine_impl(dims, B, n_q, seqlens, max_seqlen, nullptr, o_lat, lse, L.dec, ws, dev_status, st))) return rc;
   // (5) u = sum_s o_lat^(s) W_UVO^(s).
   L.g_out.A = o_lat; L.g_out.B = w_uvo; L.g_out.C = out; L.g_out.part = part;
-  return launch_gemm_simt(L.g_out, bf16, st);
+  return launch_gemm(L.g_out, bf16, st);
 }
 
 int mla_decode_sparse_workspace_size(const mla_dims *dims, int B, int n_q, int topk, size_t *bytes) {

@@ -116,6 +116,17 @@ int launch_gemm_simt(const GemmArgs &g, bool bf16, cudaStream_t st) {
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
 }
 
+int launch_gemm_reduce(const GemmArgs &g, bool bf16, cudaStream_t st) {
+  if (bf16) gemm_reduce_kernel<__nv_bfloat16><<<592, 256, 0, st>>>(g);
+  else gemm_reduce_kernel<float><<<592, 256, 0, st>>>(g);
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+int launch_gemm(const GemmArgs &g, bool bf16, cudaStream_t st) {
+  const int rc = launch_gemm_tc(g, bf16, st);
+  return rc == MLA_ERR_UNSUPPORTED ? launch_gemm_simt(g, bf16, st) : rc;
+}
+
 int launch_rope_into_query(int B, int n_q, int H, int d_c, int d_rope, const void *q_pe_raw, const int32_t *seqlens,
                            void *q_abs, float rope_base, bool bf16, cudaStream_t st) {
   if (d_rope == 0) return MLA_OK;

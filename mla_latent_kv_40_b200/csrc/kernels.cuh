@@ -166,6 +166,12 @@ struct GemmArgs {
 };
 size_t gemm_simt_workspace(const GemmArgs &g);
 int launch_gemm_simt(const GemmArgs &g, bool bf16, cudaStream_t st);
+// The tensor-core product for weight-streaming shapes (MLA_ERR_UNSUPPORTED, nothing launched, when
+// the layout does not fit); the in-order sum of K-split partials into C; and the dispatcher that tries
+// the tensor cores first.  All use the same partial buffer (gemm_simt_workspace).
+int launch_gemm_tc(const GemmArgs &g, bool bf16, cudaStream_t st);
+int launch_gemm_reduce(const GemmArgs &g, bool bf16, cudaStream_t st);
+int launch_gemm(const GemmArgs &g, bool bf16, cudaStream_t st);
 // RoPE of the query-latent path's q_pe [T, H, d_R] into the RoPE slots of q_abs [T, H, d_c + d_R].
 int launch_rope_into_query(int B, int n_q, int H, int d_c, int d_rope, const void *q_pe_raw, const int32_t *seqlens,
                            void *q_abs, float rope_base, bool bf16, cudaStream_t st);
