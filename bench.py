@@ -343,6 +343,66 @@ def measure_decode_configs(mla, torch, peaks, steps, names=("v2lite_bf16", "v3_r
     return res
 
 
+def measure_absorbed(mla, torch, peaks, steps, d_cq=1536):
+    """Decode from hidden states with folded weights (mla_decode_absorbed) on the V3 batch-64 x 4096
+    workload, d_cq = 1536: c_Q = h W_DQ, latent and RoPE queries through W_UQK and W_QR, attention, the
+    merge, and the output through W_UVO, per call (the weight folds run once, untimed).  Roofline: the
+    four weights and the latent cache read once against HBM, or the products' FLOPs against bf16."""
+    from workloads import DECODE_CASES, make_decode_inputs_device, make_query_path_inputs, latent_bytes, decode_flops
+    case = DECODE_CASES["v3_bf16"]
+    d = case.dims
+    inp = make_decode_inputs_device(case)
+    qp = {k: v.cuda() for k, v in make_query_path_inputs(case, d_cq, seed=case.seed + 1).items()}
+    dims = mla.make_dims(d.n_heads, d.d_c, d.d_rope, d.d_nope, d.d_v, d.d_model, case.block_size, d.dtype,
+                         rope_base=d.rope_base, rms_eps=d.rms_eps, cache_layout=1)
+    packed = torch.empty_like(inp["pool"])
+    mla.mla_cache_pack(dims, inp["pool"], packed)
+    torch.cuda.synchronize()
+    inp["pool"] = packed
+    B, n_q, H, D = case.batch, case.n_q, d.n_heads, d.d_model
+    w_uqk = torch.empty(H, d_cq, d.d_c, dtype=d.torch_dtype, device="cuda")
+    w_uvo = torch.empty(H, d.d_c, D, dtype=d.torch_dtype, device="cuda")
+    mla.mla_fold_query_weights(dims, qp["w_uq"], inp["w_uk"], w_uqk)
+    mla.mla_fold_output_weights(dims, inp["w_uv"], qp["w_o"], w_uvo)
+    w_qr = qp["w_qr"].reshape(d_cq, H * d.d_rope).contiguous()
+    sl = inp["seqlens"]
+    ws = mla.alloc_workspace(mla.mla_decode_absorbed_workspace_size(dims, d_cq, B, n_q, int(sl.max())))
+    out = torch.empty((B, n_q, D), dtype=d.torch_dtype, device="cuda")
+    lse = torch.empty((B, n_q, H), dtype=torch.float32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bt, sl_d = inp["block_table"].cuda(), sl.cuda()
+
+    def run():
+        mla.mla_decode_absorbed(dims, qp["h"], qp["w_dq"], w_uqk, w_qr, packed, packed, bt, inp["max_blocks_per_seq"],
+                                inp["num_blocks"], sl_d, int(sl.max()), w_uvo, out, lse, ws, st)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the absorbed decode")
+    ms = e0.elapsed_time(e1) / steps
+    T = B * n_q
+    w_bytes = 2 * (D * d_cq + H * d_cq * d.d_c + d_cq * H * d.d_rope + H * d.d_c * D)
+    seqlens = [int(x) for x in sl]
+    bytes_ = w_bytes + latent_bytes(d, seqlens)
+    flops = 2 * T * (D * d_cq + H * d_cq * d.d_c + d_cq * H * d.d_rope + H * d.d_c * D) + decode_flops(d, seqlens, n_q)["attention"]
+    t_roof = max(bytes_ / (peaks["hbm_gbs"] * 1e9), flops / (peaks["bf16_tflops"] * 1e12))
+    res = {"workload": f"v3_bf16 from hidden states, d_cq {d_cq}, folded W_UQK and W_UVO", "ms": ms,
+           "tflops": flops / (ms * 1e-3) / 1e12, "gbs": bytes_ / (ms * 1e-3) / 1e9, "bytes": bytes_,
+           "decode_tokens_per_s": T / (ms * 1e-3), "roofline_us": t_roof * 1e6, "roofline_frac": t_roof / (ms * 1e-3),
+           "call": "mla_decode_absorbed (c_Q, queries, attention, merge, output through W_UVO)"}
+    del inp, packed, ws, w_uqk, w_uvo, qp
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_sparse(mla, torch, peaks, steps, topk=2048):
     """Sparse decode (mla_decode_sparse) on the V3 batch-64 x 4096 workload with `topk` tokens selected
     per query token (seeded random distinct positions): the gather of the selected rows, absorption,
@@ -761,6 +821,7 @@ def run_mla(args):
         torch.cuda.empty_cache()
         line["configs"] = measure_decode_configs(mla, torch, peaks, max(args.steps, 5))
         line["sparse"] = measure_sparse(mla, torch, peaks, max(args.steps, 5))
+        line["absorbed"] = measure_absorbed(mla, torch, peaks, max(args.steps, 5))
         line["split_kv"] = measure_split_kv(mla, torch, peaks, max(args.steps, 5))
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(case)
