@@ -303,7 +303,10 @@ MLA_API int mla_decode_partial(const mla_dims *dims, int B, int n_q, const void 
  *   o_lat_parts [n_parts, B, n_q, H, d_c] (dims->dtype), lse_parts
  *   [n_parts, B, n_q, H] (float), both device memory (the caller gathers them,
  *   e.g. with an all-gather over NCCL).  Writes out [B, n_q, H, d_v] and, if
- *   non-NULL, lse [B, n_q, H].  Runs on CUDA cores (the merge is small).
+ *   non-NULL, lse [B, n_q, H].  bf16 with d_c = 512 (and d_v = 128 when w_uv
+ *   is given) and 16-byte aligned buffers: the merged rows are rounded to
+ *   bf16, as in mla_decode, and go through W_UV on the tensor cores (two
+ *   kernels); other shapes merge in fp32 on CUDA cores (two kernels).
  */
 MLA_API int mla_merge_workspace_size(const mla_dims *dims, int B, int n_q, int n_parts, size_t *bytes);
 MLA_API int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts, const void *o_lat_parts,

@@ -580,8 +580,12 @@ int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts, const 
   if (rc) return rc;
   if (!o_lat_parts || !lse_parts || !out) return MLA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
-  if ((size_t)16 * (dims->d_c + n_parts) * sizeof(float) > 220 * 1024) return MLA_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // bf16 rows of 512: merged by log-sum-exp into bf16 rows (in the workspace, which holds them with
+  // room to spare), then through W_UV on the tensor cores.
+  if (tc_merge_parts_supported(*dims, o_lat_parts, w_uv, out))
+    return launch_tc_merge_parts(*dims, B, n_q, n_parts, o_lat_parts, lse_parts, w_uv, out, lse, workspace, st);
+  if ((size_t)16 * (dims->d_c + n_parts) * sizeof(float) > 220 * 1024) return MLA_ERR_UNSUPPORTED;
   const size_t rows = (size_t)B * n_parts * n_q * dims->n_heads;
   float *o_part = static_cast<float *>(workspace);
   float *lse_part = reinterpret_cast<float *>(static_cast<char *>(workspace) + align256(rows * dims->d_c * sizeof(float)));

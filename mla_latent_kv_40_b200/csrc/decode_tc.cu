@@ -1010,14 +1010,71 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
 }
 
 // ------------------------------------------------------------ merge of the split partials
-// One warp per (query row g = (b, j), head s): the pieces of g's unit are merged by their
-// log-sum-exps into o_lat[g][s][0 .. 512) (bf16) and lse_out[g][s] = log of the summed exp.  Each
-// lane owns 16 latent columns (8 in each half of the row), and the loads of up to kMergeUnroll
-// pieces are in flight together, so a unit cut into a few pieces costs one round of loads.
+// One warp merges the ns pieces of one (query row, head) by their log-sum-exps: piece k is the bf16
+// row part[k * part_stride][0 .. 512) with log-sum-exp lse[k * lse_stride].  It writes the merged
+// row (bf16) and, if lse_dst is non-null, the log of the summed exp (-inf, with a zero row, where no
+// piece saw a key).  Each lane owns 16 latent columns (8 in each half of the row), and the loads of
+// up to kMergeUnroll pieces are in flight together, so a row cut into a few pieces costs one round
+// of loads.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeUnroll = 4;
 constexpr int kMaxSegPerUnit = kMaxClusters + 1;
 
+__device__ __forceinline__ void merge_row(int lane, int ns, const __nv_bfloat16 *part, int64_t part_stride,
+                                          const float *lse, int64_t lse_stride, __nv_bfloat16 *dst,
+                                          float *lse_dst) {
+  float m = -CUDART_INF_F;
+  for (int k = lane; k < ns; k += 32) m = fmaxf(m, lse[(int64_t)k * lse_stride]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float sum = 0.f;
+  if (m != -CUDART_INF_F)
+    for (int k = lane; k < ns; k += 32) sum += __expf(lse[(int64_t)k * lse_stride] - m);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  const float inv = sum > 0.f ? 1.f / sum : 0.f;
+  float v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = 0.f;
+  for (int k0 = 0; k0 < ns; k0 += kMergeUnroll) {
+    uint4 x[kMergeUnroll][2];
+    float wk[kMergeUnroll];
+#pragma unroll
+    for (int i = 0; i < kMergeUnroll; ++i) {
+      const int k = k0 + i;
+      const bool have = k < ns;
+      const __nv_bfloat16 *src = part + (int64_t)(have ? k : 0) * part_stride + 8 * lane;
+      x[i][0] = have ? *reinterpret_cast<const uint4 *>(src) : make_uint4(0, 0, 0, 0);
+      x[i][1] = have ? *reinterpret_cast<const uint4 *>(src + 256) : make_uint4(0, 0, 0, 0);
+      wk[i] = have && m != -CUDART_INF_F ? __expf(lse[(int64_t)k * lse_stride] - m) * inv : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kMergeUnroll; ++i)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[i][hh]);
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 f = __bfloat1622float2(xh[e2]);
+          v[8 * hh + 2 * e2] = fmaf(wk[i], f.x, v[8 * hh + 2 * e2]);
+          v[8 * hh + 2 * e2 + 1] = fmaf(wk[i], f.y, v[8 * hh + 2 * e2 + 1]);
+        }
+      }
+  }
+  dst += 8 * lane;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint4 packed;
+    __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) ph[e2] = __floats2bfloat162_rn(v[8 * hh + 2 * e2], v[8 * hh + 2 * e2 + 1]);
+    *reinterpret_cast<uint4 *>(dst + 256 * hh) = packed;
+  }
+  if (lane == 0 && lse_dst) *lse_dst = sum > 0.f ? m + logf(sum) : -CUDART_INF_F;
+}
+
+// One warp per (query row g = (b, j), head s): the pieces of g's unit, listed by the attention
+// kernel's segment table, merged into o_lat[g][s] and lse_out[g][s].
 __global__ void __launch_bounds__(kMergeThreads)
 tc_merge_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_info, const __nv_bfloat16 *o_part,
                 const float *lse_part, __nv_bfloat16 *o_lat, float *lse_out) {
@@ -1036,55 +1093,23 @@ tc_merge_kernel(int B, int n_q, int H, int n_rb, int max_segs, const int *seg_in
     s0 = 0;
     ns = 0;
   }
-  const float *lse_row = lse_part + (int64_t)s0 * kRows + lr;
-  float m = -CUDART_INF_F;
-  for (int k = lane; k < ns; k += 32) m = fmaxf(m, lse_row[(int64_t)k * kRows]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  float sum = 0.f;
-  if (m != -CUDART_INF_F)
-    for (int k = lane; k < ns; k += 32) sum += __expf(lse_row[(int64_t)k * kRows] - m);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  const float inv = sum > 0.f ? 1.f / sum : 0.f;
-  float v[16];
-#pragma unroll
-  for (int e = 0; e < 16; ++e) v[e] = 0.f;
-  for (int k0 = 0; k0 < ns; k0 += kMergeUnroll) {
-    uint4 x[kMergeUnroll][2];
-    float wk[kMergeUnroll];
-#pragma unroll
-    for (int i = 0; i < kMergeUnroll; ++i) {
-      const int k = k0 + i;
-      const bool have = k < ns;
-      const __nv_bfloat16 *src = o_part + ((int64_t)(s0 + (have ? k : 0)) * kRows + lr) * kDc + 8 * lane;
-      x[i][0] = have ? *reinterpret_cast<const uint4 *>(src) : make_uint4(0, 0, 0, 0);
-      x[i][1] = have ? *reinterpret_cast<const uint4 *>(src + 256) : make_uint4(0, 0, 0, 0);
-      wk[i] = have && m != -CUDART_INF_F ? __expf(lse_row[(int64_t)k * kRows] - m) * inv : 0.f;
-    }
-#pragma unroll
-    for (int i = 0; i < kMergeUnroll; ++i)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[i][hh]);
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float2 f = __bfloat1622float2(xh[e2]);
-          v[8 * hh + 2 * e2] = fmaf(wk[i], f.x, v[8 * hh + 2 * e2]);
-          v[8 * hh + 2 * e2 + 1] = fmaf(wk[i], f.y, v[8 * hh + 2 * e2 + 1]);
-        }
-      }
-  }
-  __nv_bfloat16 *dst = o_lat + ((int64_t)g * H + s) * kDc + 8 * lane;
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    uint4 packed;
-    __nv_bfloat162 *ph = reinterpret_cast<__nv_bfloat162 *>(&packed);
-#pragma unroll
-    for (int e2 = 0; e2 < 4; ++e2) ph[e2] = __floats2bfloat162_rn(v[8 * hh + 2 * e2], v[8 * hh + 2 * e2 + 1]);
-    *reinterpret_cast<uint4 *>(dst + 256 * hh) = packed;
-  }
-  if (lane == 0 && lse_out) lse_out[(int64_t)g * H + s] = sum > 0.f ? m + logf(sum) : -CUDART_INF_F;
+  merge_row(lane, ns, o_part + ((int64_t)s0 * kRows + lr) * kDc, (int64_t)kRows * kDc,
+            lse_part + (int64_t)s0 * kRows + lr, kRows, o_lat + item * kDc, lse_out ? lse_out + item : nullptr);
+}
+
+// One warp per row r = ((b, j), s) of n_parts stacked partials (one per key range, e.g. gathered
+// from the devices that each decoded one range): o_parts [n_parts][rows][512], lse_parts
+// [n_parts][rows], merged into o_lat[r] and lse_out[r].
+__global__ void __launch_bounds__(kMergeThreads)
+parts_merge_kernel(int64_t rows, int n_parts, const __nv_bfloat16 *o_parts, const float *lse_parts,
+                   __nv_bfloat16 *o_lat, float *lse_out) {
+  sm100::grid_dep_launch();
+  sm100::grid_dep_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t)blockIdx.x * (kMergeThreads / 32) + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  merge_row(lane, n_parts, o_parts + r * kDc, rows * kDc, lse_parts + r, rows, o_lat + r * kDc,
+            lse_out ? lse_out + r : nullptr);
 }
 
 // ------------------------------------------------------------ W_UV product
@@ -1384,6 +1409,28 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
   return MLA_OK;
 }
 
+namespace {
+
+// out [rows][H][128] = o_lat [rows][H][512] . W_UV^(s) per head s, on the tensor cores.
+int launch_wuv_product(const mla_dims &d, int rows, const __nv_bfloat16 *o_lat, const void *w_uv, void *out,
+                       int *dev_status, cudaStream_t st) {
+  // W_UV as [H * 512 rows][128] (boxes of 64 rows x 64 columns); o_lat as [rows][H][512].
+  CUtensorMap mw, mo;
+  int rc = make_map(&mw, w_uv, kDv, (uint64_t)d.n_heads * kDc, (uint64_t)kDv * 2);
+  if (rc) return rc;
+  if ((rc = make_map3(&mo, o_lat, kDc, d.n_heads, rows, (uint64_t)kDc * 2, (uint64_t)d.n_heads * kDc * 2))) return rc;
+  const size_t smem = 1024 + kOlBytes + kWuvBytes;
+  if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+    return MLA_ERR_CUDA;
+  const dim3 grid(d.n_heads, (rows + kCombRows - 1) / kCombRows);
+  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, mw, mo, rows, d.n_heads,
+                    static_cast<__nv_bfloat16 *>(out), dev_status) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+
+}  // namespace
+
 int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens, int max_seqlen, const void *w_uv,
                       void *out, float *lse, void *ws, int *dev_status, cudaStream_t st) {
   (void)seqlens;
@@ -1403,19 +1450,27 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
                  o_lat, lse) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (!w_uv) return MLA_OK;
-  // W_UV as [H * 512 rows][128] (boxes of 64 rows x 64 columns); o_lat as [rows][H][512].
-  CUtensorMap mw, mo;
-  int rc = make_map(&mw, w_uv, kDv, (uint64_t)d.n_heads * kDc, (uint64_t)kDv * 2);
-  if (rc) return rc;
-  if ((rc = make_map3(&mo, o_lat, kDc, d.n_heads, rows, (uint64_t)kDc * 2, (uint64_t)d.n_heads * kDc * 2))) return rc;
-  const size_t smem = 1024 + kOlBytes + kWuvBytes;
-  if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+  return launch_wuv_product(d, rows, o_lat, w_uv, out, dev_status, st);
+}
+
+bool tc_merge_parts_supported(const mla_dims &d, const void *o_parts, const void *w_uv, const void *out) {
+  const bool aligned = !(reinterpret_cast<uintptr_t>(o_parts) & 15) && !(reinterpret_cast<uintptr_t>(out) & 15) &&
+                       !(reinterpret_cast<uintptr_t>(w_uv) & 15);
+  return d.dtype == MLA_BF16 && d.d_c == kDc && (!w_uv || d.d_v == kDv) && aligned;
+}
+
+int launch_tc_merge_parts(const mla_dims &d, int B, int n_q, int n_parts, const void *o_parts, const float *lse_parts,
+                          const void *w_uv, void *out, float *lse, void *o_lat_ws, cudaStream_t st) {
+  if (!tc_merge_parts_supported(d, o_parts, w_uv, out) || n_parts <= 0) return MLA_ERR_UNSUPPORTED;
+  const int rows = B * n_q;
+  const int64_t R = (int64_t)rows * d.n_heads;
+  __nv_bfloat16 *o_lat = static_cast<__nv_bfloat16 *>(w_uv ? o_lat_ws : out);
+  const dim3 mgrid((unsigned)((R + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
+  if (launch_pdl(parts_merge_kernel, mgrid, dim3(kMergeThreads), 0, st, R, n_parts,
+                 static_cast<const __nv_bfloat16 *>(o_parts), lse_parts, o_lat, lse) != cudaSuccess)
     return MLA_ERR_CUDA;
-  const dim3 grid(d.n_heads, (rows + kCombRows - 1) / kCombRows);
-  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, mw, mo, rows, d.n_heads,
-                    static_cast<__nv_bfloat16 *>(out), dev_status) == cudaSuccess
-             ? MLA_OK
-             : MLA_ERR_CUDA;
+  if (!w_uv) return MLA_OK;
+  return launch_wuv_product(d, rows, o_lat, w_uv, out, nullptr, st);
 }
 
 }  // namespace mla
