@@ -304,9 +304,9 @@ MLA_API int mla_decode_partial(const mla_dims *dims, int B, int n_q, const void 
  *   [n_parts, B, n_q, H] (float), both device memory (the caller gathers them,
  *   e.g. with an all-gather over NCCL).  Writes out [B, n_q, H, d_v] and, if
  *   non-NULL, lse [B, n_q, H].  bf16 with d_c = 512 (and d_v = 128 when w_uv
- *   is given) and 16-byte aligned buffers: the merged rows are rounded to
- *   bf16, as in mla_decode, and go through W_UV on the tensor cores (two
- *   kernels); other shapes merge in fp32 on CUDA cores (two kernels).
+ *   is given) and 16-byte aligned buffers: one kernel merges the rows,
+ *   rounds them to bf16 as mla_decode does, and applies W_UV on the tensor
+ *   cores; other shapes merge in fp32 on CUDA cores (two kernels).
  */
 MLA_API int mla_merge_workspace_size(const mla_dims *dims, int B, int n_q, int n_parts, size_t *bytes);
 MLA_API int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts, const void *o_lat_parts,
@@ -414,8 +414,9 @@ MLA_API int mla_prefill(const mla_dims *dims, int B, const int32_t *cu_seqlens, 
 /*
  * mla_decode_launches — how many kernels one mla_decode call launches for this
  *   shape (query absorption, attention, and the combine: on the tensor-core
- *   path a merge of the split partials and the W_UV product, on the CUDA-core
- *   path one kernel); for launch accounting in profilers and benchmarks.
+ *   path one kernel that merges the split partials and applies W_UV, on the
+ *   CUDA-core path one kernel); for launch accounting in profilers and
+ *   benchmarks.
  *   Writes *count; no device work.
  */
 MLA_API int mla_decode_launches(const mla_dims *dims, int n_q, int *count);

@@ -581,10 +581,10 @@ int mla_merge_partials(const mla_dims *dims, int B, int n_q, int n_parts, const 
   if (!o_lat_parts || !lse_parts || !out) return MLA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255)) return MLA_ERR_WORKSPACE;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // bf16 rows of 512: merged by log-sum-exp into bf16 rows (in the workspace, which holds them with
-  // room to spare), then through W_UV on the tensor cores.
+  // bf16 rows of 512: merged by log-sum-exp into bf16 rows and, with W_UV, multiplied by it on the
+  // tensor cores in the same kernel (the workspace is not used).
   if (tc_merge_parts_supported(*dims, o_lat_parts, w_uv, out))
-    return launch_tc_merge_parts(*dims, B, n_q, n_parts, o_lat_parts, lse_parts, w_uv, out, lse, workspace, st);
+    return launch_tc_merge_parts(*dims, B, n_q, n_parts, o_lat_parts, lse_parts, w_uv, out, lse, st);
   if ((size_t)16 * (dims->d_c + n_parts) * sizeof(float) > 220 * 1024) return MLA_ERR_UNSUPPORTED;
   const size_t rows = (size_t)B * n_parts * n_q * dims->n_heads;
   float *o_part = static_cast<float *>(workspace);

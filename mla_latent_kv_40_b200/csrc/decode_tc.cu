@@ -1112,29 +1112,61 @@ parts_merge_kernel(int64_t rows, int n_parts, const __nv_bfloat16 *o_parts, cons
             lse_out ? lse_out + r : nullptr);
 }
 
-// ------------------------------------------------------------ W_UV product
-// CTA = (head s, 64 query rows (b, j)): out^T [d_v x 64] = W_UV^(s)T . o_lat^T on the tensor cores,
-// with W_UV supplying the 128-row M side (A = W_UV^T, M-major; B = o_lat, K-major; fp32
-// accumulator in 64 tensor-memory columns).  All of W_UV[s] (128 KB) is requested by TMA before the
-// kernel waits for the merge, straight into the MMA's 128-byte-swizzled operand layout, so its
-// transfer overlaps the merge; the 64 rows of o_lat follow the same way.
+// ------------------------------------------------------------ merge + W_UV product
+// Where the pieces of output row (g, s) live: the attention kernel's per-unit segment list
+// (seg_info != NULL: piece k is row (s0 + k) * 128 + lr of the segment partials), or n_parts stacked
+// partials (piece k is row k * rows * H + g * H + s).
+struct Pieces {
+  const __nv_bfloat16 *part;   // rows of 512 bf16
+  const float *lse;            // one log-sum-exp per row of `part`
+  const int *seg_info;         // [units][2], or NULL for stacked partials
+  int n_q, H, n_rb, max_segs, n_parts;
+};
+
+// Number of pieces of row (g, s) and the index of its first piece row; pieces are `stride` rows apart.
+__device__ __forceinline__ int piece_rows(const Pieces &pc, int rows, int g, int s, int64_t &first, int64_t &stride) {
+  if (!pc.seg_info) {
+    first = (int64_t)g * pc.H + s;
+    stride = (int64_t)rows * pc.H;
+    return pc.n_parts;
+  }
+  const int b = g / pc.n_q, j = g % pc.n_q;
+  const int gr = j * pc.H + s;
+  const int u = b * pc.n_rb + gr / kRows;
+  int s0 = pc.seg_info[2 * u], ns = pc.seg_info[2 * u + 1];
+  ns = ns < 0 ? 0 : (ns > kMaxSegPerUnit ? kMaxSegPerUnit : ns);
+  if (s0 < 0 || s0 + ns > pc.max_segs) return 0;
+  first = (int64_t)s0 * kRows + gr % kRows;
+  stride = kRows;
+  return ns;
+}
+
+// CTA = (head s, 64 query rows (b, j)): the rows' pieces are merged by their log-sum-exps straight
+// into the B operand tile of the W_UV product (o_lat [64 rows x 512], K-major, 128-byte swizzled,
+// bf16), then out^T [d_v x 64] = W_UV^(s)T . o_lat^T on the tensor cores, with W_UV supplying the
+// 128-row M side (A = W_UV^T, M-major; fp32 accumulator in 64 tensor-memory columns).  All of
+// W_UV[s] (128 KB) is requested by TMA before the kernel waits for the attention kernel, so its
+// transfer overlaps that kernel's tail.  The merge runs on all 256 threads at once: four threads
+// per row, each owning 16 of the row's 64 16-byte column blocks (blocks 4 i + q), so that the four
+// threads of a row read 64 contiguous bytes per load.
 constexpr int kCombRows = 64;
 constexpr int kCombThreads = 256;
 constexpr int kDv = 128;                                   // the W_UV tile width this kernel takes
 constexpr uint32_t kOlBytes = kCombRows * kDc * 2;         // o_lat: [8 K-chunks][64 rows][128 B]
 constexpr uint32_t kWuvBytes = kDc * kDv * 2;              // W_UV^T: [8 K-chunks][2 M-chunks][64 K rows][128 B]
+static_assert(kCombThreads == 4 * kCombRows, "four merging threads per row");
 
 __global__ void __launch_bounds__(kCombThreads)
-tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_o, int rows, int H,
+tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const Pieces pc, int rows, float *lse_out,
                   __nv_bfloat16 *out, int *dev_status) {
   extern __shared__ unsigned char csm_raw[];
   unsigned char *csm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~uintptr_t(1023));
   unsigned char *ol = csm;                                                          // o_lat, K-major, swizzled
   unsigned char *wa = csm + kOlBytes;                                               // W_UV^T, M-major, swizzled
-  __shared__ __align__(8) uint64_t bar_w, bar_o, bar_mma;
+  __shared__ __align__(8) uint64_t bar_w, bar_mma;
   __shared__ uint32_t tmem_slot;
   __shared__ int s_loaded;
-  const int s = blockIdx.x;
+  const int s = blockIdx.x, H = pc.H;
   const int g0 = blockIdx.y * kCombRows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   sm100::grid_dep_launch();
@@ -1142,11 +1174,9 @@ tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
   // MMA's M-major, 128-byte-swizzled layout: box (K-chunk kc, M-chunk mc) at (kc * 2 + mc) * 8 KB.
   if (tid == 0) {
     mbar_init(smem_u32(&bar_w), 1);
-    mbar_init(smem_u32(&bar_o), 1);
     mbar_init(smem_u32(&bar_mma), 1);
     fence_mbar_init();
     tma_prefetch_desc(&map_w);
-    tma_prefetch_desc(&map_o);
     mbar_expect_tx(smem_u32(&bar_w), kWuvBytes);
     for (int kc = 0; kc < kDc / 64; ++kc)
       for (int mc = 0; mc < 2; ++mc)
@@ -1156,12 +1186,64 @@ tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
     tmem_alloc(smem_u32(&tmem_slot), kCombRows);
     tmem_relinquish();
   }
-  sm100::grid_dep_wait();   // o_lat comes from the merge kernel; out may still be read before it
-  // o_lat rows g0 .. g0 + 63 of head s, K-chunk c -> [64 rows x 128 B] at c * 8 KB (rows past the
-  // end are zero-filled by the copy).
-  if (tid == 0) {
-    mbar_expect_tx(smem_u32(&bar_o), kOlBytes);
-    for (int c = 0; c < kDc / 64; ++c) tma_load_3d(smem_u32(ol + c * 8192), &map_o, 64 * c, s, g0, smem_u32(&bar_o));
+  sm100::grid_dep_wait();   // the partials and the segment list come from the attention kernel
+  {
+    // Merge of row rr (output row g = g0 + rr); rows past the end become zero rows of the tile.
+    const int rr = tid >> 2, q = tid & 3, g = g0 + rr;
+    int64_t first = 0, stride = 0;
+    const int ns = g < rows ? piece_rows(pc, rows, g, s, first, stride) : 0;
+    float m = -CUDART_INF_F;
+    for (int k = 0; k < ns; ++k) m = fmaxf(m, pc.lse[first + k * stride]);
+    float sum = 0.f;
+    if (m != -CUDART_INF_F)
+      for (int k = 0; k < ns; ++k) sum += __expf(pc.lse[first + k * stride] - m);
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+      // this round: column blocks cb = 4 (8 hh + i) + q, i < 8 (8 bf16 each)
+      float acc[8][8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+      for (int k0 = 0; k0 < ns; k0 += 2) {
+        uint4 x[2][8];
+        float wk[2];
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const bool have = k0 + kk < ns;
+          const __nv_bfloat16 *src = pc.part + (first + (int64_t)(have ? k0 + kk : 0) * stride) * kDc;
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            x[kk][i] = have ? *reinterpret_cast<const uint4 *>(src + 8 * (4 * (8 * hh + i) + q)) : make_uint4(0, 0, 0, 0);
+          wk[kk] = have && m != -CUDART_INF_F ? __expf(pc.lse[first + (int64_t)(k0 + kk) * stride] - m) * inv : 0.f;
+        }
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const __nv_bfloat162 *xh = reinterpret_cast<const __nv_bfloat162 *>(&x[kk][i]);
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const float2 f = __bfloat1622float2(xh[e2]);
+              acc[i][2 * e2] = fmaf(wk[kk], f.x, acc[i][2 * e2]);
+              acc[i][2 * e2 + 1] = fmaf(wk[kk], f.y, acc[i][2 * e2 + 1]);
+            }
+          }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int cb = 4 * (8 * hh + i) + q, kc = cb >> 3, jj = cb & 7;
+        uint4 packed;
+        packed.x = pack_bf16x2(acc[i][0], acc[i][1]);
+        packed.y = pack_bf16x2(acc[i][2], acc[i][3]);
+        packed.z = pack_bf16x2(acc[i][4], acc[i][5]);
+        packed.w = pack_bf16x2(acc[i][6], acc[i][7]);
+        *reinterpret_cast<uint4 *>(ol + kc * 8192 + (rr >> 3) * 1024 + (rr & 7) * 128 + ((jj ^ (rr & 7)) << 4)) = packed;
+      }
+    }
+    if (q == 0 && lse_out && g < rows) lse_out[(int64_t)g * H + s] = sum > 0.f ? m + logf(sum) : -CUDART_INF_F;
+    fence_proxy_async_smem();   // the merged tile is read by the MMA (async proxy)
   }
   tc_fence_before();
   __syncthreads();
@@ -1169,7 +1251,7 @@ tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
   const uint32_t tmem = tmem_slot;
   int loaded = 1;
   if (tid == 0) {
-    if (!mbar_wait(smem_u32(&bar_w), 0, kWaitNs) || !mbar_wait(smem_u32(&bar_o), 0, kWaitNs)) {
+    if (!mbar_wait(smem_u32(&bar_w), 0, kWaitNs)) {
       report(dev_status, MLA_ERR_TIMEOUT);
       loaded = 0;
     }
@@ -1221,10 +1303,8 @@ tc_combine_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_consta
     tc_fence_after();
     tmem_dealloc(tmem, kCombRows);
   }
-  if (tid == 0 && !loaded) {   // the copies must have landed before this CTA's shared memory goes away
+  if (tid == 0 && !loaded)   // the copies must have landed before this CTA's shared memory goes away
     mbar_wait(smem_u32(&bar_w), 0, kWaitNs);
-    mbar_wait(smem_u32(&bar_o), 0, kWaitNs);
-  }
 }
 
 // ------------------------------------------------------------ host side
@@ -1254,23 +1334,8 @@ int make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, ui
   return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
 }
 
-// 3-D map over a [d2][d1][d0] bf16 array (d0 contiguous), box [64 x 1 x 64], 128-byte swizzle.
-int make_map3(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
-              uint64_t stride2_bytes) {
-  auto fn = encode_fn();
-  if (!fn) return MLA_ERR_CUDA;
-  cuuint64_t dims[3] = {d0, d1, d2};
-  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
-  cuuint32_t box[3] = {64, 1, 64};
-  cuuint32_t es[3] = {1, 1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MLA_OK : MLA_ERR_CUDA;
-}
-
 struct WsLayout {
-  size_t seg_info, o_part, lse_part, o_lat, total;
+  size_t seg_info, o_part, lse_part, total;
 };
 
 int clusters_for_device();
@@ -1285,8 +1350,7 @@ WsLayout ws_layout(int B, int n_rb) {
   L.seg_info = 0;
   L.o_part = a256(U * 2 * sizeof(int) + kTimeoutRecInts * sizeof(int));
   L.lse_part = L.o_part + a256(segs * kRows * kDc * sizeof(__nv_bfloat16));
-  L.o_lat = L.lse_part + a256(segs * kRows * sizeof(float));           // merged rows, [B n_q][H][512]
-  L.total = L.o_lat + a256(U * kRows * kDc * sizeof(__nv_bfloat16));
+  L.total = L.lse_part + a256(segs * kRows * sizeof(float));
   return L;
 }
 
@@ -1341,7 +1405,7 @@ bool tc_decode_supported(const mla_dims &d, int n_q) {
          d.d_v == 128 && n_q * d.n_heads <= 2 * kRows;
 }
 
-int tc_decode_kernel_launches() { return 3; }   // attention, merge, W_UV product
+int tc_decode_kernel_launches() { return 2; }   // attention; merge (+ W_UV product)
 
 size_t tc_decode_workspace_bytes(const mla_dims &d, int B, int n_q) {
   const int n_rb = (n_q * d.n_heads + kRows - 1) / kRows;
@@ -1411,19 +1475,19 @@ int launch_tc_attention(const mla_dims &d, int B, int n_q, const void *q_abs, co
 
 namespace {
 
-// out [rows][H][128] = o_lat [rows][H][512] . W_UV^(s) per head s, on the tensor cores.
-int launch_wuv_product(const mla_dims &d, int rows, const __nv_bfloat16 *o_lat, const void *w_uv, void *out,
-                       int *dev_status, cudaStream_t st) {
-  // W_UV as [H * 512 rows][128] (boxes of 64 rows x 64 columns); o_lat as [rows][H][512].
-  CUtensorMap mw, mo;
+// out [rows][H][128] = (pieces of each row, merged) . W_UV^(s) per head s, on the tensor cores;
+// lse (if non-null) gets the merged log-sum-exps.
+int launch_merge_wuv(const mla_dims &d, int rows, const Pieces &pc, const void *w_uv, void *out, float *lse,
+                     int *dev_status, cudaStream_t st) {
+  // W_UV as [H * 512 rows][128] (boxes of 64 rows x 64 columns).
+  CUtensorMap mw;
   int rc = make_map(&mw, w_uv, kDv, (uint64_t)d.n_heads * kDc, (uint64_t)kDv * 2);
   if (rc) return rc;
-  if ((rc = make_map3(&mo, o_lat, kDc, d.n_heads, rows, (uint64_t)kDc * 2, (uint64_t)d.n_heads * kDc * 2))) return rc;
   const size_t smem = 1024 + kOlBytes + kWuvBytes;
   if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
     return MLA_ERR_CUDA;
   const dim3 grid(d.n_heads, (rows + kCombRows - 1) / kCombRows);
-  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, mw, mo, rows, d.n_heads,
+  return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, mw, pc, rows, lse,
                     static_cast<__nv_bfloat16 *>(out), dev_status) == cudaSuccess
              ? MLA_OK
              : MLA_ERR_CUDA;
@@ -1440,17 +1504,20 @@ int launch_tc_combine(const mla_dims &d, int B, int n_q, const int32_t *seqlens,
   char *w = static_cast<char *>(ws);
   if (w_uv && (d.d_v != kDv || (reinterpret_cast<uintptr_t>(w_uv) & 15))) return MLA_ERR_UNSUPPORTED;
   const int rows = B * n_q;
-  // Merge into o_lat: the output itself when no W_UV is given, else the workspace's row buffer.
-  __nv_bfloat16 *o_lat = w_uv ? reinterpret_cast<__nv_bfloat16 *>(w + L.o_lat) : static_cast<__nv_bfloat16 *>(out);
+  const int max_segs = B * n_rb + clusters_for_device();
+  if (w_uv) {   // merge and W_UV product in one kernel
+    const Pieces pc{reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part), reinterpret_cast<const float *>(w + L.lse_part),
+                    reinterpret_cast<const int *>(w + L.seg_info), n_q, d.n_heads, n_rb, max_segs, 0};
+    return launch_merge_wuv(d, rows, pc, w_uv, out, lse, dev_status, st);
+  }
+  // Without W_UV the merged rows are the output.
   const int64_t warps = (int64_t)rows * d.n_heads;
   const dim3 mgrid((unsigned)((warps + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
-  if (launch_pdl(tc_merge_kernel, mgrid, dim3(kMergeThreads), 0, st, B, n_q, d.n_heads, n_rb,
-                 B * n_rb + clusters_for_device(), reinterpret_cast<const int *>(w + L.seg_info),
-                 reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part), reinterpret_cast<const float *>(w + L.lse_part),
-                 o_lat, lse) != cudaSuccess)
-    return MLA_ERR_CUDA;
-  if (!w_uv) return MLA_OK;
-  return launch_wuv_product(d, rows, o_lat, w_uv, out, dev_status, st);
+  return launch_pdl(tc_merge_kernel, mgrid, dim3(kMergeThreads), 0, st, B, n_q, d.n_heads, n_rb, max_segs,
+                    reinterpret_cast<const int *>(w + L.seg_info), reinterpret_cast<const __nv_bfloat16 *>(w + L.o_part),
+                    reinterpret_cast<const float *>(w + L.lse_part), static_cast<__nv_bfloat16 *>(out), lse) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 bool tc_merge_parts_supported(const mla_dims &d, const void *o_parts, const void *w_uv, const void *out) {
@@ -1460,17 +1527,20 @@ bool tc_merge_parts_supported(const mla_dims &d, const void *o_parts, const void
 }
 
 int launch_tc_merge_parts(const mla_dims &d, int B, int n_q, int n_parts, const void *o_parts, const float *lse_parts,
-                          const void *w_uv, void *out, float *lse, void *o_lat_ws, cudaStream_t st) {
+                          const void *w_uv, void *out, float *lse, cudaStream_t st) {
   if (!tc_merge_parts_supported(d, o_parts, w_uv, out) || n_parts <= 0) return MLA_ERR_UNSUPPORTED;
   const int rows = B * n_q;
+  if (w_uv) {
+    const Pieces pc{static_cast<const __nv_bfloat16 *>(o_parts), lse_parts, nullptr, n_q, d.n_heads, 0, 0, n_parts};
+    return launch_merge_wuv(d, rows, pc, w_uv, out, lse, nullptr, st);
+  }
   const int64_t R = (int64_t)rows * d.n_heads;
-  __nv_bfloat16 *o_lat = static_cast<__nv_bfloat16 *>(w_uv ? o_lat_ws : out);
   const dim3 mgrid((unsigned)((R + kMergeThreads / 32 - 1) / (kMergeThreads / 32)));
-  if (launch_pdl(parts_merge_kernel, mgrid, dim3(kMergeThreads), 0, st, R, n_parts,
-                 static_cast<const __nv_bfloat16 *>(o_parts), lse_parts, o_lat, lse) != cudaSuccess)
-    return MLA_ERR_CUDA;
-  if (!w_uv) return MLA_OK;
-  return launch_wuv_product(d, rows, o_lat, w_uv, out, nullptr, st);
+  return launch_pdl(parts_merge_kernel, mgrid, dim3(kMergeThreads), 0, st, R, n_parts,
+                    static_cast<const __nv_bfloat16 *>(o_parts), lse_parts, static_cast<__nv_bfloat16 *>(out), lse) ==
+                 cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
 }
 
 }  // namespace mla
