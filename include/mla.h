@@ -30,9 +30,11 @@
  *    share one library-owned scratch buffer per GPU (see there).  Besides that
  *    buffer, the library's only global state is per-device host-side caches
  *    filled on first use and read-only afterwards: the number of attention
- *    clusters that fit on the device, the driver's tensor-map encoder, and the
- *    device address of the no-allocation scratch buffer.  Each is guarded, so
- *    first calls from several host threads are safe.
+ *    clusters that fit on the device, the driver's tensor-map encoder, the
+ *    device address of the no-allocation scratch buffer, and, per kernel, the
+ *    dynamic shared-memory size already requested from the driver.  Each is
+ *    guarded (a mutex or atomics), so first calls from several host threads
+ *    are safe.
  *  - There is no CPU fallback: a shape the CUDA kernels do not handle returns
  *    MLA_ERR_UNSUPPORTED.
  *

@@ -1484,7 +1484,8 @@ int launch_merge_wuv(const mla_dims &d, int rows, const Pieces &pc, const void *
   int rc = make_map(&mw, w_uv, kDv, (uint64_t)d.n_heads * kDc, (uint64_t)kDv * 2);
   if (rc) return rc;
   const size_t smem = 1024 + kOlBytes + kWuvBytes;
-  if (cudaFuncSetAttribute(tc_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+  static std::atomic<int> smem_set[kSmemCacheDevs];
+  if (smem_limit(tc_combine_kernel, smem, smem_set) != cudaSuccess)
     return MLA_ERR_CUDA;
   const dim3 grid(d.n_heads, (rows + kCombRows - 1) / kCombRows);
   return launch_pdl(tc_combine_kernel, grid, dim3(kCombThreads), smem, st, mw, pc, rows, lse,

@@ -177,7 +177,8 @@ int launch_gemm_tc(const GemmArgs &g, bool bf16, cudaStream_t st) {
   p.sc_m = g.sc_m;
   p.dev_status = nullptr;
   const size_t smem = 1024 + (size_t)kGStages * kGStageBytes;
-  if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  static std::atomic<int> smem_set[kSmemCacheDevs];
+  if (smem_limit(gemm_tc_kernel, smem, smem_set) != cudaSuccess)
     return MLA_ERR_CUDA;
   const dim3 grid(g.N / 128, g.ksplit, g.batch * ((g.M + kGN - 1) / kGN));
   if (launch_pdl(gemm_tc_kernel, grid, dim3(kGThreads), smem, st, mb, ma, p) != cudaSuccess) return MLA_ERR_CUDA;

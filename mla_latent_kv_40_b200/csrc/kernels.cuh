@@ -1,6 +1,8 @@
 // Argument bundles and launchers of every libmla kernel (host side).
 #pragma once
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace mla {
@@ -21,6 +23,26 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device.  The driver is
+// called only the first time a launcher asks for that size (or more) on that device, since the
+// limit then stays set for the process; `cache` is the launcher's own record of the sizes set per
+// device.  Devices past the table's end always call the driver.
+constexpr int kSmemCacheDevs = 64;
+template <typename... KArgs>
+inline cudaError_t smem_limit(void (*kernel)(KArgs...), size_t bytes, std::atomic<int> (&cache)[kSmemCacheDevs]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const bool tracked = dev >= 0 && dev < kSmemCacheDevs;
+  if (tracked && cache[dev].load(std::memory_order_acquire) >= (int)bytes) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess && tracked) {
+    int cur = cache[dev].load(std::memory_order_relaxed);
+    while (cur < (int)bytes && !cache[dev].compare_exchange_weak(cur, (int)bytes, std::memory_order_release)) {
+    }
+  }
+  return e;
 }
 
 struct AppendArgs {

@@ -29,6 +29,8 @@ constexpr int kTcN = 64;                      // activation rows (tokens / query
 constexpr uint32_t kAChunk = 128 * 128;       // [128 rows x 64 K] bf16, 128B-swizzled: 16 KB
 constexpr uint32_t kBChunk = kTcN * 128;      // [64 rows x 64 K] bf16: 8 KB
 constexpr uint64_t kWaitNs = 2000000000ull;
+// The absorption's output staging tile reuses its operand tiles (one K-chunk at least).
+static_assert(sizeof(__nv_bfloat16) * kTcN * (128 + 8) <= kAChunk + kBChunk, "staging fits the operand tiles");
 
 // Bounded wait: on expiry report a timeout and let the caller skip its work.
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, int *dev_status) {
@@ -50,7 +52,9 @@ __device__ __forceinline__ void absorb_tc_body(const CUtensorMap &map_w, const C
   const int nkc = a.d_nope / 64;
   unsigned char *As = sm;                                  // [nkc][128 x 128 B]
   unsigned char *Bs = As + nkc * kAChunk;                  // [nkc][64 x 128 B]
-  __nv_bfloat16 *Os = reinterpret_cast<__nv_bfloat16 *>(Bs + nkc * kBChunk);   // [64][128 + 8]
+  // [64][128 + 8] output staging over the operand tiles, which are dead once the MMAs completed:
+  // 48 KB per CTA instead of 65 KB, so four CTAs fit on an SM and the grid runs in one wave.
+  __nv_bfloat16 *Os = reinterpret_cast<__nv_bfloat16 *>(sm);
   constexpr int ldo = 128 + 8;
   const int m0 = by * 128, r0 = bz * kTcN;
   const int R = a.B * a.n_q, W = a.d_c + a.d_rope;
@@ -380,8 +384,9 @@ int launch_absorb_tc(const AbsorbArgs &a, int *dev_status, cudaStream_t st) {
       !make_tmap_bf16(&mq, a.q_nope, (uint64_t)a.H * a.d_nope, R, (uint64_t)a.H * a.d_nope * 2, kTcN))
     return MLA_ERR_CUDA;
   const int nkc = a.d_nope / 64;
-  const size_t smem = 1024 + nkc * (kAChunk + kBChunk) + sizeof(__nv_bfloat16) * kTcN * (128 + 8);
-  if (cudaFuncSetAttribute(absorb_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+  const size_t smem = 1024 + nkc * (kAChunk + kBChunk);
+  static std::atomic<int> smem_set[kSmemCacheDevs];
+  if (smem_limit(absorb_tc_kernel, smem, smem_set) != cudaSuccess)
     return MLA_ERR_CUDA;
   const dim3 grid(a.H, a.d_c / 128, (R + kTcN - 1) / kTcN);
   return launch_pdl(absorb_tc_kernel, grid, dim3(kTcThreads), smem, st, mw, mq, a, dev_status) == cudaSuccess
@@ -403,7 +408,8 @@ int launch_append_tc(const AppendArgs &a, void *ws, int nsplit, int k_per_split,
       !make_tmap_bf16(&mh, a.h, a.d_model, a.T, (uint64_t)a.d_model * 2, kTcN))
     return MLA_ERR_CUDA;
   const size_t smem = 1024 + kApStages * kApStageBytes;
-  if (cudaFuncSetAttribute(append_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+  static std::atomic<int> smem_set[kSmemCacheDevs];
+  if (smem_limit(append_tc_kernel, smem, smem_set) != cudaSuccess)
     return MLA_ERR_CUDA;
   const dim3 grid((W + 127) / 128, nsplit, (a.T + kTcN - 1) / kTcN);
   return launch_pdl(append_tc_kernel, grid, dim3(kTcThreads), smem, st, mwd, mwr, mh, a.T, a.d_c, a.d_rope,
@@ -440,10 +446,11 @@ int launch_decode_prep(const AppendArgs &ap, const AbsorbArgs &ab, void *part, i
   pp.nB = ab.H * pp.b_ny * pp.b_nz;
   pp.counter = counter;
   const int nkc = ab.d_nope / 64;
-  const size_t smem_ab = 1024 + nkc * (kAChunk + kBChunk) + sizeof(__nv_bfloat16) * kTcN * (128 + 8);
+  const size_t smem_ab = 1024 + nkc * (kAChunk + kBChunk);
   const size_t smem_ap = 1024 + kApStages * kApStageBytes;
   const size_t smem = smem_ab > smem_ap ? smem_ab : smem_ap;
-  if (cudaFuncSetAttribute(decode_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem))
+  static std::atomic<int> smem_set[kSmemCacheDevs];
+  if (smem_limit(decode_prep_kernel, smem, smem_set) != cudaSuccess)
     return MLA_ERR_CUDA;
   if (cudaMemsetAsync(counter, 0, sizeof(unsigned), st) != cudaSuccess) return MLA_ERR_CUDA;
   return launch_pdl(decode_prep_kernel, dim3(pp.nA + pp.nB + ap.T), dim3(kTcThreads), smem, st, mwd, mwr, mh, mw, mq,
