@@ -758,28 +758,60 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
       // No early exit in this region: the eight warps meet at named barriers, so on a timeout they
       // keep walking the same (now wait-free: every wait returns at once) loop to the end.
       while (it.next(p, cid, b, rb, t0, t1, segid, first_u, nseg)) {
-        // Q row -> half h loads latent dims 256h..256h+255 into TMEM columns 128h..; half 0 also
-        // puts the RoPE dims into the shared [128 x 64] A tile.  The previous unit's MMAs are
-        // complete (its last S was consumed), so both may be overwritten.
+        // Q rows -> half h loads latent dims 256h..256h+255 of its warp's 32 rows into TMEM columns
+        // 128h..; half 0 also puts the RoPE dims into the shared [128 x 64] A tile.  The previous
+        // unit's MMAs are complete (its last S was consumed), so both may be overwritten.  The loads
+        // are coalesced (eight lanes per 128-byte row segment) and pass through the warp's 4 KB of
+        // the half's P staging tile, 128-byte swizzled, from which each thread reads its own row for
+        // the tensor-memory store; the last P copy out of that tile must have read it first.
         const int gr = rb * kRows + r;
         const bool real = gr < nrows;
         {
-          const uint4 *src = reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * nrows + (real ? gr : 0)) * kW);
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
+          if (q4 == 0 && lane == 0) bulk_wait_read_all();
+          asm volatile("bar.sync %0, 128;" ::"r"(2 + h) : "memory");
+          unsigned char *stg_w = stgp + q4 * 4096;
+          const int j = lane & 7;
+          const uint4 *rowp[8];
+          bool live[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              uint4 x = real ? __ldg(src + h * 32 + c * 8 + i) : make_uint4(0, 0, 0, 0);
-              v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+          for (int k = 0; k < 8; ++k) {
+            const int g = rb * kRows + q4 * 32 + 4 * k + (lane >> 3);
+            live[k] = g < nrows;
+            rowp[k] = reinterpret_cast<const uint4 *>(p.q + ((int64_t)b * nrows + (live[k] ? g : 0)) * kW);
+          }
+#pragma unroll 1
+          for (int cb = 0; cb < 4; cb += 2) {
+            uint4 x[2][8];
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr)
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                x[rr][k] = live[k] ? __ldg(rowp[k] + h * 32 + (cb + rr) * 8 + j) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int lr = 4 * k + (lane >> 3);
+                *reinterpret_cast<uint4 *>(stg_w + (lr >> 3) * 1024 + (lr & 7) * 128 + ((j ^ (lr & 7)) << 4)) = x[rr][k];
+              }
+              __syncwarp();
+              uint32_t v[32];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const uint4 y = *reinterpret_cast<const uint4 *>(stg_w + (lane >> 3) * 1024 + (lane & 7) * 128 + ((i ^ (lane & 7)) << 4));
+                v[4 * i] = y.x; v[4 * i + 1] = y.y; v[4 * i + 2] = y.z; v[4 * i + 3] = y.w;
+              }
+              tmem_st32(tbase + lane_off + kQCol + 128 * h + 32 * (cb + rr), v);
+              __syncwarp();
             }
-            tmem_st32(tbase + lane_off + kQCol + 128 * h + 32 * c, v);
           }
           if (h == 0) {
-            unsigned char *qpe = tiles + kQpeOff + (r >> 3) * 1024 + (r & 7) * 128;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<uint4 *>(qpe + ((c ^ (r & 7)) << 4)) = real ? __ldg(src + 64 + c) : make_uint4(0, 0, 0, 0);
+            for (int k = 0; k < 8; ++k) {
+              const int rq = q4 * 32 + 4 * k + (lane >> 3);
+              *reinterpret_cast<uint4 *>(tiles + kQpeOff + (rq >> 3) * 1024 + (rq & 7) * 128 + ((j ^ (rq & 7)) << 4)) =
+                  live[k] ? __ldg(rowp[k] + 64 + j) : make_uint4(0, 0, 0, 0);
+            }
             fence_proxy_async_smem();
           }
           tmem_wait_st();
