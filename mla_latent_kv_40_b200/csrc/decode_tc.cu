@@ -1014,13 +1014,20 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap map_c, const __grid_con
             uint32_t v[32];
             tmem_ld32(tbase + lane_off + ocol + 32 * c, v);
             tmem_wait_ld();
+            // 32-byte stores: the row's 64 bytes leave in two whole sectors (rows are 1 KB apart, the
+            // O halves start at 512 bytes, so every store is 32-byte aligned).
 #pragma unroll
-            for (int i = 0; i < 32; i += 8)
-              *reinterpret_cast<uint4 *>(dst + 32 * c + i) =
-                  make_uint4(pack_bf16x2(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
-                             pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
-                             pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
-                             pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
+            for (int i = 0; i < 32; i += 16) {
+              const uint4 lo = make_uint4(pack_bf16x2(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv),
+                                          pack_bf16x2(__uint_as_float(v[i + 2]) * inv, __uint_as_float(v[i + 3]) * inv),
+                                          pack_bf16x2(__uint_as_float(v[i + 4]) * inv, __uint_as_float(v[i + 5]) * inv),
+                                          pack_bf16x2(__uint_as_float(v[i + 6]) * inv, __uint_as_float(v[i + 7]) * inv));
+              const uint4 hi = make_uint4(pack_bf16x2(__uint_as_float(v[i + 8]) * inv, __uint_as_float(v[i + 9]) * inv),
+                                          pack_bf16x2(__uint_as_float(v[i + 10]) * inv, __uint_as_float(v[i + 11]) * inv),
+                                          pack_bf16x2(__uint_as_float(v[i + 12]) * inv, __uint_as_float(v[i + 13]) * inv),
+                                          pack_bf16x2(__uint_as_float(v[i + 14]) * inv, __uint_as_float(v[i + 15]) * inv));
+              st_global_v8(dst + 32 * c + i, lo, hi);
+            }
           }
           if (g == 0) p.lse_part[(int64_t)q.segid * kRows + r] = l > 0.f ? (m + __log2f(l)) * 0.69314718055994531f : -CUDART_INF_F;
           tc_fence_before();
