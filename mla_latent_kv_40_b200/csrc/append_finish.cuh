@@ -31,11 +31,19 @@ __device__ __forceinline__ void append_finish_token(const AppendArgs &a, const f
     const int j2 = tid + i * kThreads;
     float2 acc = make_float2(0.f, 0.f);
     if (j2 < npair) {
-#pragma unroll 8
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float2 x = __ldcg(pp + sp * split_stride + j2);
-        acc.x += x.x;
-        acc.y += x.y;
+      // Up to 32 partials' loads in flight at once, then added in split order (the same order for
+      // every caller, so the bits do not depend on the batching).
+      for (int s0 = 0; s0 < nsplit; s0 += 32) {
+        float2 xs[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          xs[k] = s0 + k < nsplit ? __ldcg(pp + (int64_t)(s0 + k) * split_stride + j2) : make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (s0 + k < nsplit) {
+            acc.x += xs[k].x;
+            acc.y += xs[k].y;
+          }
       }
       if (j2 < npc) red[j2] = acc.x * acc.x + acc.y * acc.y;
     }
