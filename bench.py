@@ -691,8 +691,8 @@ def run_mla(args):
     barrier()
     fused_ms = max_over_ranks(a0.elapsed_time(a1) / args.steps)
 
-    # End to end through the public calls: pinned host inputs in, result out, every step's copies inside the
-    # timed region.  The inputs of step i+1 are copied (copy stream) while step i computes, into the other of
+    # End to end through the public calls a user makes for a step (mla_append_latent, then mla_decode):
+    # pinned host inputs in, result out, every step's copies inside the timed region.  The inputs of step i+1 are copied (copy stream) while step i computes, into the other of
     # two device buffer sets, and step i's result goes back (a second copy stream) while step i+1 computes.
     e2e = None
     if not args.no_e2e:
@@ -715,6 +715,7 @@ def run_mla(args):
         h2d = nbytes   # the bytes of the one copy (inputs plus alignment padding)
         d2h = host_out[0].numel() * host_out[0].element_size()
         dev_blobs = [torch.empty(nbytes, dtype=torch.uint8, device="cuda") for _ in range(2)]
+        e2e_ws = mla.alloc_workspace(mla.mla_decode_workspace_size(dims, B, n_q, max_seqlen))
         bufs = [views(b) for b in dev_blobs]
         outs = [torch.empty_like(out) for _ in range(2)]
         h2d_s, d2h_s = torch.cuda.Stream(), torch.cuda.Stream()
@@ -739,16 +740,12 @@ def run_mla(args):
             x = bufs[j]
             stream.wait_event(in_ready[j])
             stream.wait_event(out_read[j])            # step i-2's result has left outs[j]
-            side.wait_stream(stream)
+            # The calls a user makes for a step: append the new tokens, then one mla_decode.
             mla.mla_append_latent(dims, x["h_new"], dev["w_dkv"], dev["w_kr"], dev["gamma"], x["seq_idx"], x["pos"],
                                   c_kv, k_pe, bt, B, inp["max_blocks_per_seq"], inp["num_blocks"], status,
-                                  workspace=app_ws, stream=side)
-            appended.record(side)
-            mla.mla_absorb_q(dims, x["q_nope"], x["q_pe"], dev["w_uk"], x["seqlens"], q_abs)
-            stream.wait_event(appended)
-            mla.mla_decode_attention(dims, q_abs, c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
-                                     x["seqlens"], max_seqlen, ws, status)
-            mla.mla_decode_combine(dims, B, n_q, x["seqlens"], max_seqlen, dev["w_uv"], outs[j], lse, ws)
+                                  workspace=app_ws)
+            mla.mla_decode(dims, x["q_nope"], x["q_pe"], c_kv, k_pe, bt, inp["max_blocks_per_seq"], inp["num_blocks"],
+                           x["seqlens"], max_seqlen, dev["w_uk"], dev["w_uv"], outs[j], lse, e2e_ws, status)
             in_free[j].record(stream)
             out_ready[j].record(stream)
             d2h_s.wait_event(out_ready[j])
