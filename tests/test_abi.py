@@ -222,3 +222,13 @@ def test_split_kv_host_validation():
     assert mla._lib.mla_merge_workspace_size(ctypes.byref(dims), 4, 2, 0, ctypes.byref(n)) == -1
     assert mla._lib.mla_merge_workspace_size(ctypes.byref(dims), 4, 2, 4, ctypes.byref(n)) == 0
     assert n.value >= 4 * 4 * 2 * 128 * 512 * 4
+    # mla_merge_partials refuses missing parts and a short or misaligned workspace before any launch.
+    merge = mla._lib.mla_merge_partials
+    ws = ctypes.c_void_p(1 << 20)
+    assert merge(ctypes.byref(dims), 4, 2, 4, None, fake, fake, fake, None, ws, n.value, None) == -1
+    assert merge(ctypes.byref(dims), 4, 2, 4, fake, None, fake, fake, None, ws, n.value, None) == -1
+    assert merge(ctypes.byref(dims), 4, 2, 4, fake, fake, fake, None, None, ws, n.value, None) == -1
+    assert merge(ctypes.byref(dims), 4, 2, 4, fake, fake, fake, fake, None, ws, n.value - 256, None) == -3
+    assert merge(ctypes.byref(dims), 4, 2, 4, fake, fake, fake, fake, None, ctypes.c_void_p((1 << 20) + 16), n.value,
+                 None) == -3
+    assert merge(ctypes.byref(dims), 4, 2, 0, fake, fake, fake, fake, None, ws, n.value, None) == -1
